@@ -1,0 +1,133 @@
+"""fp64 CPU oracle for the retention contraction -- test infrastructure only.
+
+This package is the checker: ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` are its only
+callers.  The product path (``retnet_retention_chunkwise_b200``) never imports
+it, and it imports nothing from there.
+
+The arithmetic lives in ``retention_oracle.c`` (plain C, fp64, one thread per
+(batch, head) pair); this module only compiles it with gcc and marshals numpy
+arrays.  Each C function cites the passage it follows:
+
+* ``recurrent``  -- S_n = gamma S_{n-1} + k_n^T v_n, y_n = q_n S_n (the
+  definition; page "Retentive Networks -- Microsoft Propone l'Alternativa
+  Architetturale ai Transformer", section "Il meccanismo: Multi-Scale
+  Retention").
+* ``parallel``   -- the double sum y_n = sum_{m<=n} gamma^(n-m) (q_n.k_m) v_m
+  (same section), plus gamma^(n+1) q_n S_in for a carried-in state.
+* ``chunkwise``  -- the block form of the same section, derived by splitting
+  the sum at each block start.
+
+Inputs are float64 numpy arrays (bf16 or fp32 values widen to fp64 exactly).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "retention_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_BUILD, "liboracle.so")
+
+_lib = None
+
+
+def build(src: str = _SRC, out: str = _LIB, extra_flags=()) -> str:
+    """Compile the C oracle with gcc (-O2, no fast-math: IEEE fp64)."""
+    os.makedirs(os.path.dirname(out), exist_ok=True)
+    cmd = ["gcc", "-O2", "-std=c99", "-D_POSIX_C_SOURCE=200809L", "-fPIC", "-shared",
+           "-fno-fast-math", "-ffp-contract=off", *extra_flags, src, "-o", out, "-lm", "-lpthread"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _needs_build() -> bool:
+    return (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+
+
+def load(path: str | None = None):
+    """Load (building first if stale) the oracle library and declare signatures."""
+    global _lib
+    if path is None:
+        if _lib is not None:
+            return _lib
+        if _needs_build():
+            build()
+        path = _LIB
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    i = ctypes.c_int
+    lib.oracle_recurrent.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
+    lib.oracle_parallel.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
+    lib.oracle_chunkwise.argtypes = [i, i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
+    for f in (lib.oracle_recurrent, lib.oracle_parallel, lib.oracle_chunkwise):
+        f.restype = ctypes.c_int
+    if path == _LIB:
+        _lib = lib
+    return lib
+
+
+def _f64(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor -> exact fp64 copy
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _run(form: str, q, k, v, gamma, state_in=None, chunk: int = 0,
+         nthreads: int = 0, lib=None):
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    gamma = _f64(gamma).reshape(-1)
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L) or gamma.shape[0] != H:
+        raise ValueError("oracle: shape mismatch")
+    s_in = _f64(state_in)
+    if s_in is not None and s_in.shape != (B, H, dk, dv):
+        raise ValueError("oracle: state_in must be [B,H,dk,dv]")
+    y = np.zeros((B, H, L, dv), dtype=np.float64)
+    s_out = np.zeros((B, H, dk, dv), dtype=np.float64)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(s_in), _ptr(y), _ptr(s_out), int(nthreads))
+    if form == "recurrent":
+        rc = lib.oracle_recurrent(B, H, L, dk, dv, *args)
+    elif form == "parallel":
+        rc = lib.oracle_parallel(B, H, L, dk, dv, *args)
+    elif form == "chunkwise":
+        rc = lib.oracle_chunkwise(B, H, L, dk, dv, int(chunk), *args)
+    else:
+        raise ValueError(form)
+    if rc != 0:
+        raise ValueError(f"oracle_{form}: invalid arguments")
+    return y, s_out
+
+
+def recurrent(q, k, v, gamma, state_in=None, nthreads: int = 0, lib=None):
+    """Recurrent definition in fp64.  Returns (y [B,H,L,dv], state_out [B,H,dk,dv])."""
+    return _run("recurrent", q, k, v, gamma, state_in, 0, nthreads, lib)
+
+
+def parallel(q, k, v, gamma, state_in=None, nthreads: int = 0, lib=None):
+    """Double-sum (parallel) form in fp64.  Same outputs as :func:`recurrent`."""
+    return _run("parallel", q, k, v, gamma, state_in, 0, nthreads, lib)
+
+
+def chunkwise(q, k, v, gamma, chunk: int, state_in=None, nthreads: int = 0, lib=None):
+    """Block (chunkwise) form in fp64 with block length ``chunk``."""
+    return _run("chunkwise", q, k, v, gamma, state_in, chunk, nthreads, lib)
+
+
+def recurrent_step(q, k, v, gamma, state, nthreads: int = 0, lib=None):
+    """One decode step (q, k, v of shape [B,H,1,d]) from ``state``; returns (y, new_state)."""
+    return _run("recurrent", q, k, v, gamma, state, 0, nthreads, lib)

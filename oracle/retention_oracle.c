@@ -1,0 +1,240 @@
+/*
+ * retention_oracle.c -- fp64 host reference for the retention contraction.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the checker the CUDA path is
+ * compared against.  Only tests/, the smoke check and the CPU-baseline leg of
+ * the benchmark load it.  It shares no code, header, table or constant with the
+ * CUDA library (retnet_retention_chunkwise_b200/csrc), and it never includes
+ * anything from there.
+ *
+ * What it computes (source: "Retentive Networks -- Microsoft Propone
+ * l'Alternativa Architetturale ai Transformer", aimpact.prandi.net, section
+ * "Il meccanismo: Multi-Scale Retention"):
+ *
+ *   retention sum       y_n = sum_{m<=n} gamma^(n-m) (q_n . k_m) v_m
+ *   recurrent form      S_n = gamma S_{n-1} + k_n^T v_n ,   y_n = q_n S_n
+ *   chunkwise form      blocks of length C: the parallel rule inside a block,
+ *                       the recurrence between blocks (stated in words only)
+ *
+ * Row vectors: q_n, k_n in R^{1 x dk}, v_n, y_n in R^{1 x dv}, S in R^{dk x dv}
+ * (the state shape "h x d" given in the author responses on paperhub.cn,
+ * "Retentive Network: A Successor to Transformer ...", reply on inference cost).
+ * One gamma per head (same page 1 section: each head has its own gamma).
+ *
+ * Readings where the pages are silent (all stated again in the design notes):
+ *   - gamma^0 = 1 also for gamma = 0 (the diagonal term is kept);
+ *   - the state before the first token is state_in, or zero when none is given;
+ *   - state_out is S after the last token of the call;
+ *   - no normalisation and no denominator (author responses on paperhub.cn,
+ *     reply comparing Eq. (1) with RFA-Gate);
+ *   - a chunk length that does not divide L leaves a shorter last chunk.
+ *
+ * Layout: q, k [B][H][L][dk], v, y [B][H][L][dv], state [B][H][dk][dv], all
+ * row-major doubles.  gamma [H].  Heads are independent; threads take whole
+ * (b, h) pairs.  Every function returns 0 on success, -1 on bad arguments.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+/* gamma^n for integer n >= 0, with gamma^0 = 1 for every gamma (0^0 = 1). */
+static double gpow(double g, long n) {
+    if (n == 0) return 1.0;
+    return pow(g, (double)n);
+}
+
+typedef struct {
+    int form;            /* 0 recurrent, 1 parallel (double sum), 2 chunkwise */
+    int B, H, L, dk, dv, C;
+    const double *q, *k, *v, *gamma, *state_in;
+    double *y, *state_out;
+    int next;            /* next (b,h) pair to take */
+    pthread_mutex_t lock;
+} job_t;
+
+/* Recurrent form: S <- gamma S + k_n^T v_n, then y_n = q_n S (page 1, the
+ * "forma ricorrente" sentence).  This is the definition itself: unrolling the
+ * recurrence gives S_n = sum_{m<=n} gamma^(n-m) k_m^T v_m, so q_n S_n is the
+ * retention sum plus gamma^(n+1) q_n S_in. */
+static void head_recurrent(const job_t* J, const double* q, const double* k,
+                           const double* v, double g, const double* s_in,
+                           double* y, double* s_out) {
+    const int L = J->L, dk = J->dk, dv = J->dv;
+    double* S = (double*)calloc((size_t)dk * dv, sizeof(double));
+    if (s_in) memcpy(S, s_in, sizeof(double) * (size_t)dk * dv);
+    for (int n = 0; n < L; ++n) {
+        const double* qn = q + (size_t)n * dk;
+        const double* kn = k + (size_t)n * dk;
+        const double* vn = v + (size_t)n * dv;
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j)
+                S[(size_t)i * dv + j] = g * S[(size_t)i * dv + j] + kn[i] * vn[j];
+        double* yn = y + (size_t)n * dv;
+        for (int j = 0; j < dv; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < dk; ++i) acc += qn[i] * S[(size_t)i * dv + j];
+            yn[j] = acc;
+        }
+    }
+    if (s_out) memcpy(s_out, S, sizeof(double) * (size_t)dk * dv);
+    free(S);
+}
+
+/* Parallel form as the plain double sum of the definition (page 1, the
+ * "Y_n = sum_(m<=n) gamma^(n-m) Q_n K_m^T V_m" sentence), plus the carried-in
+ * state term gamma^(n+1) q_n S_in. */
+static void head_parallel(const job_t* J, const double* q, const double* k,
+                          const double* v, double g, const double* s_in,
+                          double* y, double* s_out) {
+    const int L = J->L, dk = J->dk, dv = J->dv;
+    for (int n = 0; n < L; ++n) {
+        const double* qn = q + (size_t)n * dk;
+        double* yn = y + (size_t)n * dv;
+        for (int j = 0; j < dv; ++j) yn[j] = 0.0;
+        for (int m = 0; m <= n; ++m) {
+            const double* km = k + (size_t)m * dk;
+            const double* vm = v + (size_t)m * dv;
+            double s = 0.0;
+            for (int i = 0; i < dk; ++i) s += qn[i] * km[i];
+            s *= gpow(g, n - m);
+            for (int j = 0; j < dv; ++j) yn[j] += s * vm[j];
+        }
+        if (s_in) {
+            const double w = gpow(g, (long)n + 1);
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += qn[i] * s_in[(size_t)i * dv + j];
+                yn[j] += w * acc;
+            }
+        }
+    }
+    if (s_out) {
+        /* S_{L-1} = gamma^L S_in + sum_m gamma^(L-1-m) k_m^T v_m */
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j) {
+                double acc = s_in ? gpow(g, L) * s_in[(size_t)i * dv + j] : 0.0;
+                for (int m = 0; m < L; ++m)
+                    acc += gpow(g, (long)L - 1 - m) * k[(size_t)m * dk + i] * v[(size_t)m * dv + j];
+                s_out[(size_t)i * dv + j] = acc;
+            }
+    }
+}
+
+/* Chunkwise form (page 1, the "forma chunkwise" sentence: blocks of length C,
+ * parallel inside the block, recurrence between blocks).  Splitting the
+ * definition's sum at the block start t0 gives, for local index i < l:
+ *   y_{t0+i} = sum_{j<=i} gamma^(i-j) (q_i . k_j) v_j  +  gamma^(i+1) q_i S_prev
+ *   S_new    = gamma^l S_prev + sum_{j<l} gamma^(l-1-j) k_j^T v_j
+ * with l = C, or the remainder for the last block. */
+static void head_chunkwise(const job_t* J, const double* q, const double* k,
+                           const double* v, double g, const double* s_in,
+                           double* y, double* s_out) {
+    const int L = J->L, dk = J->dk, dv = J->dv, C = J->C;
+    double* S = (double*)calloc((size_t)dk * dv, sizeof(double));
+    double* Sn = (double*)malloc(sizeof(double) * (size_t)dk * dv);
+    if (s_in) memcpy(S, s_in, sizeof(double) * (size_t)dk * dv);
+    for (int t0 = 0; t0 < L; t0 += C) {
+        const int l = (L - t0 < C) ? (L - t0) : C;
+        for (int i = 0; i < l; ++i) {
+            const double* qi = q + (size_t)(t0 + i) * dk;
+            double* yi = y + (size_t)(t0 + i) * dv;
+            for (int c = 0; c < dv; ++c) yi[c] = 0.0;
+            for (int j = 0; j <= i; ++j) {
+                const double* kj = k + (size_t)(t0 + j) * dk;
+                const double* vj = v + (size_t)(t0 + j) * dv;
+                double s = 0.0;
+                for (int d = 0; d < dk; ++d) s += qi[d] * kj[d];
+                s *= gpow(g, i - j);
+                for (int c = 0; c < dv; ++c) yi[c] += s * vj[c];
+            }
+            const double xi = gpow(g, (long)i + 1);
+            for (int c = 0; c < dv; ++c) {
+                double acc = 0.0;
+                for (int d = 0; d < dk; ++d) acc += qi[d] * S[(size_t)d * dv + c];
+                yi[c] += xi * acc;
+            }
+        }
+        const double gl = gpow(g, l);
+        for (int d = 0; d < dk; ++d)
+            for (int c = 0; c < dv; ++c) {
+                double acc = gl * S[(size_t)d * dv + c];
+                for (int j = 0; j < l; ++j)
+                    acc += gpow(g, (long)l - 1 - j) * k[(size_t)(t0 + j) * dk + d] *
+                           v[(size_t)(t0 + j) * dv + c];
+                Sn[(size_t)d * dv + c] = acc;
+            }
+        memcpy(S, Sn, sizeof(double) * (size_t)dk * dv);
+    }
+    if (s_out) memcpy(s_out, S, sizeof(double) * (size_t)dk * dv);
+    free(Sn);
+    free(S);
+}
+
+static void* worker(void* arg) {
+    job_t* J = (job_t*)arg;
+    const size_t qs = (size_t)J->L * J->dk, vs = (size_t)J->L * J->dv;
+    const size_t ss = (size_t)J->dk * J->dv;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        const int p = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (p >= J->B * J->H) break;
+        const int h = p % J->H;
+        const double* si = J->state_in ? J->state_in + (size_t)p * ss : NULL;
+        double* so = J->state_out ? J->state_out + (size_t)p * ss : NULL;
+        const double* q = J->q + (size_t)p * qs;
+        const double* k = J->k + (size_t)p * qs;
+        const double* v = J->v + (size_t)p * vs;
+        double* y = J->y + (size_t)p * vs;
+        if (J->form == 0) head_recurrent(J, q, k, v, J->gamma[h], si, y, so);
+        else if (J->form == 1) head_parallel(J, q, k, v, J->gamma[h], si, y, so);
+        else head_chunkwise(J, q, k, v, J->gamma[h], si, y, so);
+    }
+    return NULL;
+}
+
+static int run(int form, int B, int H, int L, int dk, int dv, int C,
+               const double* q, const double* k, const double* v,
+               const double* gamma, const double* state_in, double* y,
+               double* state_out, int nthreads) {
+    if (B < 0 || H < 1 || L < 0 || dk < 1 || dv < 1 || !gamma) return -1;
+    if (form == 2 && C < 1) return -1;
+    if (L > 0 && (!q || !k || !v || !y)) return -1;
+    for (int h = 0; h < H; ++h)
+        if (!(gamma[h] >= 0.0 && gamma[h] <= 1.0)) return -1;
+    job_t J = {form, B, H, L, dk, dv, C, q, k, v, gamma, state_in, y, state_out, 0};
+    pthread_mutex_init(&J.lock, NULL);
+    if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads > B * H) nthreads = B * H;
+    if (nthreads < 1) nthreads = 1;
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, worker, &J);
+    worker(&J);
+    for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return 0;
+}
+
+int oracle_recurrent(int B, int H, int L, int dk, int dv, const double* q,
+                     const double* k, const double* v, const double* gamma,
+                     const double* state_in, double* y, double* state_out,
+                     int nthreads) {
+    return run(0, B, H, L, dk, dv, 1, q, k, v, gamma, state_in, y, state_out, nthreads);
+}
+
+int oracle_parallel(int B, int H, int L, int dk, int dv, const double* q,
+                    const double* k, const double* v, const double* gamma,
+                    const double* state_in, double* y, double* state_out,
+                    int nthreads) {
+    return run(1, B, H, L, dk, dv, 1, q, k, v, gamma, state_in, y, state_out, nthreads);
+}
+
+int oracle_chunkwise(int B, int H, int L, int dk, int dv, int C, const double* q,
+                     const double* k, const double* v, const double* gamma,
+                     const double* state_in, double* y, double* state_out,
+                     int nthreads) {
+    return run(2, B, H, L, dk, dv, C, q, k, v, gamma, state_in, y, state_out, nthreads);
+}
