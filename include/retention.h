@@ -1,0 +1,137 @@
+/*
+ * retention.h -- C ABI of libretention, the B200 (sm_100a) implementation of the
+ * retention contraction of Multi-Scale Retention (RetNet).
+ *
+ * The operation (page "Retentive Networks -- Microsoft Propone l'Alternativa
+ * Architetturale ai Transformer", aimpact.prandi.net, section "Il meccanismo:
+ * Multi-Scale Retention"), per batch row b and head h with decay gamma_h:
+ *
+ *     y_n = sum_{m <= n} gamma_h^(n-m) (q_n . k_m) v_m  +  gamma_h^(n+1) q_n S_in
+ *
+ * computed in three equivalent forms named by the same section: parallel
+ * (the whole decayed score matrix at once), chunkwise (blocks of length C:
+ * parallel inside a block, recurrence between blocks) and recurrent
+ * (S_n = gamma S_{n-1} + k_n^T v_n, y_n = q_n S_n; one token per call).
+ * gamma^0 is taken as 1, also for gamma = 0.  There is no normalisation and no
+ * denominator (author responses on paperhub.cn, "Retentive Network: A
+ * Successor to Transformer ...", reply comparing Eq. (1) with RFA-Gate).
+ *
+ * Layouts (all row-major and contiguous, element = the call's dtype unless
+ * stated):
+ *     q, k   [B][H][L][dk]          v, y   [B][H][L][dv]
+ *     state  [B][H][dk][dv]  always fp32 (the "h x d" state shape from the
+ *                            paperhub.cn author responses, reply on inference cost)
+ *     gamma  [H]             HOST array of fp32, each finite and in [0, 1]
+ * Ownership: the caller owns every buffer.  q, k, v, y, state and workspace are
+ * DEVICE pointers (from cudaMalloc, torch, ...); gamma is a HOST pointer read
+ * during the call.  Every call is asynchronous on `stream` (a cudaStream_t;
+ * NULL = legacy default stream) and allocates nothing.
+ *
+ * Precision: RET_BF16 runs the tensor-core path (bf16 operands, fp32
+ * accumulation, fp32 state, y rounded to bf16).  RET_F32 runs fp32 CUDA-core
+ * kernels (fp32 throughout).
+ *
+ * Errors: every argument is validated before anything is launched; a call that
+ * returns anything but RET_OK has launched nothing.  RET_EUNSUPPORTED marks a
+ * shape/dtype combination this library does not implement (there is no
+ * fallback).  Kernels never trap: a wait that runs out of time sets a device
+ * status word instead, read with retention_get_device_status().
+ */
+#ifndef RETENTION_H
+#define RETENTION_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define RET_API __attribute__((visibility("default")))
+#else
+#define RET_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RET_OK = 0,
+  RET_EINVAL = 1,        /* null pointer, bad size, gamma outside [0,1], misalignment */
+  RET_EUNSUPPORTED = 2,  /* valid request that this library does not implement */
+  RET_ECUDA = 3,         /* a CUDA runtime call failed (launch, attribute, copy) */
+  RET_ETIMEOUT = 4       /* a kernel's bounded wait expired (device status) */
+} ret_status;
+
+typedef enum { RET_F32 = 0, RET_BF16 = 1 } ret_dtype;
+
+/* L is ignored by retention_recurrent_step (one token per call). */
+typedef struct {
+  int B, H, L, dk, dv;
+} ret_shape;
+
+/* Largest head count one call accepts (per-head decay travels in the launch). */
+#define RET_MAX_HEADS 1024
+
+/*
+ * Parallel form: y = (Q K^T (.) D) V per (b, h), D[n][m] = gamma_h^(n-m) for
+ * m <= n and 0 above the diagonal.  Same page and section, "forma parallela";
+ * it is Eq. (5) / Fig. 2a in the paperhub.cn author responses (reply on why the
+ * two forms of Fig. 2 are equivalent).  No state in or out.
+ * Supported: RET_F32 with dk <= 256; RET_BF16 with dk in {64, 128, 256} and
+ * dv a multiple of 128.  Pointers must be 16-byte aligned.
+ */
+RET_API ret_status retention_parallel(const void* q, const void* k, const void* v, const float* gamma,
+                              void* y, ret_shape s, ret_dtype dt, void* stream);
+
+/*
+ * Chunkwise form with block length `chunk` (C): inside a block of length l
+ * (C, or the remainder for the last block) starting at t0, for i < l,
+ *     y_{t0+i} = sum_{j<=i} gamma^(i-j) (q_i . k_j) v_j + gamma^(i+1) q_i S_prev
+ *     S_new    = gamma^l S_prev + sum_{j<l} gamma^(l-1-j) k_j^T v_j
+ * (same page and section, "forma chunkwise"; the equations are the split of the
+ * definition's sum at each block start).
+ * state_in  : device fp32 [B][H][dk][dv], or NULL for a zero initial state.
+ * state_out : device fp32, or NULL; receives S after the last token.  It may be
+ *             the same buffer as state_in (in-place carry between calls).
+ * workspace : optional device scratch of workspace_bytes bytes (>= 256-byte
+ *             aligned).  With enough of it (see the query below) the sequence is
+ *             also split across CTAs for parallelism; with less, or NULL, the
+ *             call still runs, with fewer CTAs.  Results do not depend on it
+ *             beyond fp32 rounding.
+ * Supported: RET_F32 with 1 <= chunk <= 128, dk <= 256; RET_BF16 with chunk a
+ * multiple of 16 in [16, 128], dk in {64, 128, 256}, dv a multiple of 128.
+ */
+RET_API ret_status retention_chunkwise(const void* q, const void* k, const void* v, const float* gamma,
+                               void* y, const float* state_in, float* state_out, int chunk,
+                               ret_shape s, ret_dtype dt, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Workspace size that lets retention_chunkwise use its full sequence split for
+ * this shape (0 when the shape needs none). */
+RET_API size_t retention_chunkwise_workspace_bytes(int chunk, ret_shape s, ret_dtype dt);
+
+/*
+ * One recurrent (decode) step, in place on the state:
+ *     S <- gamma_h S + k^T v ;  y = q S        (same page and section, "forma ricorrente")
+ * q, k [B][H][1][dk], v, y [B][H][1][dv] in the call's dtype; state fp32
+ * [B][H][dk][dv], read and written in place.  Supported for both dtypes with
+ * dk <= 1024; state must be 16-byte aligned.
+ */
+RET_API ret_status retention_recurrent_step(const void* q, const void* k, const void* v,
+                                    const float* gamma, void* y, float* state, ret_shape s,
+                                    ret_dtype dt, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word:
+ * RET_OK, RET_ETIMEOUT if a kernel's bounded wait expired since the last
+ * query, or RET_ECUDA if the stream reported an error. */
+RET_API ret_status retention_get_device_status(void* stream);
+
+/* Static, NUL-terminated name of a status code. */
+RET_API const char* retention_status_str(ret_status st);
+
+/* ABI version of this header (major * 100 + minor). */
+RET_API int retention_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RETENTION_H */

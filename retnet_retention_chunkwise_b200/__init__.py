@@ -1,0 +1,192 @@
+"""retnet_retention_chunkwise_b200 -- the retention contraction of Multi-Scale
+Retention (RetNet) on NVIDIA B200 (sm_100a).
+
+    y_n = sum_{m<=n} gamma_h^(n-m) (q_n . k_m) v_m  (+ gamma_h^(n+1) q_n S_in)
+
+in its parallel, chunkwise and recurrent forms (page "Retentive Networks --
+Microsoft Propone l'Alternativa Architetturale ai Transformer", section "Il
+meccanismo: Multi-Scale Retention").  The work is done by the hand-written
+CUDA kernels of ``libretention.so`` behind the C ABI of ``include/retention.h``;
+this module only checks tensors and marshals pointers (PyTorch supplies device
+memory and the current stream).  There is no CPU path: without the compiled
+library every call raises.
+
+Tensors: q, k [B, H, L, dk]; v [B, H, L, dv]; state fp32 [B, H, dk, dv]; all
+contiguous CUDA tensors; bf16 (tensor-core path) or fp32 (CUDA-core path).
+``gamma`` is a host sequence / CPU tensor of H values in [0, 1].
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+
+import torch
+
+from . import _abi
+
+__all__ = ["parallel", "chunkwise", "recurrent_step", "device_status", "workspace_bytes",
+           "RetentionError", "library"]
+
+_LIB = None
+_LOCK = threading.Lock()
+
+
+class RetentionError(RuntimeError):
+    """A libretention call returned a status other than RET_OK."""
+
+    def __init__(self, status: int, where: str):
+        name = library().retention_status_str(status).decode()
+        super().__init__(f"{where}: {name}")
+        self.status = status
+
+
+def library() -> ctypes.CDLL:
+    """The loaded libretention.so (raises ImportError if it was not built)."""
+    global _LIB
+    if _LIB is None:
+        with _LOCK:
+            if _LIB is None:
+                _LIB = _abi.load()
+    return _LIB
+
+
+def _check(rc: int, where: str):
+    if rc != _abi.RET_OK:
+        raise RetentionError(rc, where)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return _abi.RET_BF16
+    if t.dtype == torch.float32:
+        return _abi.RET_F32
+    raise TypeError(f"retention: unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _cuda(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"retention: {name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"retention: {name} must be contiguous")
+
+
+def _gamma(gamma, H: int):
+    if isinstance(gamma, torch.Tensor):
+        if gamma.is_cuda:
+            raise ValueError("retention: gamma must be on the host (it is read at launch)")
+        g = gamma.detach().to(torch.float32).reshape(-1).tolist()
+    else:
+        g = [float(x) for x in gamma]
+    if len(g) != H:
+        raise ValueError(f"retention: gamma has {len(g)} values for {H} heads")
+    return (ctypes.c_float * H)(*g)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _shape(q, v):
+    B, H, L, dk = q.shape
+    return _abi.RetShape(B, H, L, dk, v.shape[-1])
+
+
+def _qkv(q, k, v):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _cuda(t, n)
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError("retention: expected q, k [B,H,L,dk] and v [B,H,L,dv]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("retention: q, k, v must share a dtype")
+    return _dtype(q)
+
+
+def parallel(q, k, v, gamma, *, out=None):
+    """Parallel form: y = (Q K^T (.) D) V per head.  Returns y [B,H,L,dv]."""
+    dt = _qkv(q, k, v)
+    s = _shape(q, v)
+    y = out if out is not None else torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    _cuda(y, "out")
+    _check(library().retention_parallel(_ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(y), s, dt,
+                                        _stream()), "retention_parallel")
+    return y
+
+
+_WS = {}
+
+
+def workspace_bytes(chunk: int, B: int, H: int, L: int, dk: int, dv: int,
+                    dtype: torch.dtype = torch.bfloat16) -> int:
+    """Scratch bytes that let the chunkwise call split long sequences across CTAs."""
+    code = _abi.RET_BF16 if dtype == torch.bfloat16 else _abi.RET_F32
+    return int(library().retention_chunkwise_workspace_bytes(chunk, _abi.RetShape(B, H, L, dk, dv), code))
+
+
+def _workspace(nbytes: int, device):
+    if nbytes == 0:
+        return None
+    key = (device.index if device.index is not None else torch.cuda.current_device())
+    ws = _WS.get(key)
+    if ws is None or ws.numel() * 4 < nbytes:
+        ws = torch.empty((nbytes + 3) // 4, dtype=torch.float32, device=device)
+        _WS[key] = ws
+    return ws
+
+
+def chunkwise(q, k, v, gamma, chunk: int, *, state_in=None, state_out=None, return_state=True,
+              out=None, workspace="auto"):
+    """Chunkwise form with block length ``chunk``.
+
+    Returns (y, state_out).  ``state_in`` (fp32 [B,H,dk,dv], optional) is the
+    state before the first token; ``state_out`` may be given (it may be the same
+    tensor as ``state_in``) or is allocated when ``return_state``.
+    ``workspace`` (CUDA tensor) enables the sequence split; the default "auto"
+    uses a cached buffer of ``workspace_bytes(...)``; None runs without one.
+    """
+    dt = _qkv(q, k, v)
+    s = _shape(q, v)
+    y = out if out is not None else torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    _cuda(y, "out")
+    sshape = (s.B, s.H, s.dk, s.dv)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        if t is not None:
+            _cuda(t, n)
+            if t.dtype != torch.float32 or tuple(t.shape) != sshape:
+                raise ValueError(f"retention: {n} must be fp32 {sshape}")
+    if state_out is None and return_state:
+        state_out = torch.empty(sshape, dtype=torch.float32, device=q.device)
+    if isinstance(workspace, str):
+        workspace = _workspace(int(library().retention_chunkwise_workspace_bytes(chunk, s, dt)), q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(library().retention_chunkwise(_ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(y),
+                                         _ptr(state_in), _ptr(state_out), int(chunk), s, dt,
+                                         _ptr(workspace), wbytes, _stream()), "retention_chunkwise")
+    return y, state_out
+
+
+def recurrent_step(q, k, v, gamma, state, *, out=None):
+    """One decode step in place on ``state``: S <- gamma S + k^T v, y = q S.
+
+    q, k [B,H,1,dk], v [B,H,1,dv]; state fp32 [B,H,dk,dv].  Returns y [B,H,1,dv].
+    """
+    dt = _qkv(q, k, v)
+    if q.shape[2] != 1:
+        raise ValueError("retention: recurrent_step takes one token (L == 1)")
+    s = _shape(q, v)
+    _cuda(state, "state")
+    if state.dtype != torch.float32 or tuple(state.shape) != (s.B, s.H, s.dk, s.dv):
+        raise ValueError("retention: state must be fp32 [B,H,dk,dv]")
+    y = out if out is not None else torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    _cuda(y, "out")
+    _check(library().retention_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(y),
+                                              _ptr(state), s, dt, _stream()), "retention_recurrent_step")
+    return y
+
+
+def device_status() -> int:
+    """Synchronise the current stream; return (and clear) the device status code."""
+    return int(library().retention_get_device_status(_stream()))

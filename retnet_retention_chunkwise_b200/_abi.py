@@ -1,0 +1,55 @@
+"""ctypes declarations for libretention.so (the C ABI in include/retention.h).
+
+Marshalling only: this module loads the in-tree shared library and declares the
+signatures.  There is no alternative implementation behind it; if the library
+is missing or fails to load, importing the package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libretention.so")
+
+RET_OK, RET_EINVAL, RET_EUNSUPPORTED, RET_ECUDA, RET_ETIMEOUT = 0, 1, 2, 3, 4
+RET_F32, RET_BF16 = 0, 1
+RET_MAX_HEADS = 1024
+
+# Every symbol include/retention.h declares.
+EXPORTS = (
+    "retention_parallel",
+    "retention_chunkwise",
+    "retention_chunkwise_workspace_bytes",
+    "retention_recurrent_step",
+    "retention_get_device_status",
+    "retention_status_str",
+    "retention_abi_version",
+)
+
+
+class RetShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("L", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int)]
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(
+            f"libretention.so not found at {path}; build it with "
+            "`python -m retnet_retention_chunkwise_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    vp, fp, i, sz = ctypes.c_void_p, ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.c_size_t
+    lib.retention_parallel.argtypes = [vp, vp, vp, fp, vp, RetShape, i, vp]
+    lib.retention_chunkwise.argtypes = [vp, vp, vp, fp, vp, vp, vp, i, RetShape, i, vp, sz, vp]
+    lib.retention_chunkwise_workspace_bytes.argtypes = [i, RetShape, i]
+    lib.retention_chunkwise_workspace_bytes.restype = sz
+    lib.retention_recurrent_step.argtypes = [vp, vp, vp, fp, vp, vp, RetShape, i, vp]
+    lib.retention_get_device_status.argtypes = [vp]
+    lib.retention_status_str.argtypes = [i]
+    lib.retention_status_str.restype = ctypes.c_char_p
+    lib.retention_abi_version.argtypes = []
+    for name in ("retention_parallel", "retention_chunkwise", "retention_recurrent_step",
+                 "retention_get_device_status", "retention_abi_version"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib

@@ -1,0 +1,582 @@
+// chunkwise_tc.cuh -- bf16 chunkwise retention on the sm_100a tensor cores.
+//
+// The form (page "Retentive Networks -- Microsoft ...", section "Il meccanismo:
+// Multi-Scale Retention": blocks of length C, parallel inside a block,
+// recurrence between blocks), written out for a block of length l at t0:
+//   P   = Q_c K_c^T                                   (scores, l x l)
+//   O   = (P (.) D) V_c  +  diag(xi) Q_c S_prev        D_ij = gamma^(i-j), j <= i
+//   S   = gamma^l S_prev + K_c^T diag(zeta) V_c        xi_i = gamma^(i+1), zeta_j = gamma^(l-1-j)
+//
+// One CTA owns (b, h, a 128-column slice of dv, a run of consecutive blocks)
+// and walks its blocks in order with the fp32 state slice resident in TMEM.
+// Warp roles (192 threads):
+//   warps 0-3  epilogue: TMEM lane r = thread r (0..127).  Turns P into the
+//              decayed bf16 P~ in place, scales rows of K_c by zeta, scales O
+//              by xi, keeps the state (rescale by gamma^l, bf16 copy for the
+//              next block's Q S term), writes y.
+//   warp 4     TMA producer: Q_c, K_c and the V_c slice per block, NS stages.
+//   warp 5     TMEM allocator; lane 0 issues every tcgen05.mma.
+// Per block the MMA warp issues, in order,
+//   MMA1  P[pb] = Q K^T            A = Q  (smem, K-major)   B = K  (smem, K-major)
+//   MMA4  O     = Q Sb             A = Q  (smem, K-major)   B = Sb (smem, K-major; bf16 S^T)
+//   MMA3  O    += P~ V             A = P~ (TMEM, bf16)      B = V  (smem, MN-major)
+//   MMA5  S^T  += V^T (zeta K)     A = V  (smem, MN-major)  B = zeta K (smem, MN-major)
+// with xi applied to O between MMA4 and MMA3 (a TMEM read-modify-write), so the
+// cross-block and intra-block terms share one accumulator.  The state is held
+// transposed (lanes = the 128 dv columns, columns = dk) so MMA5 has M = 128
+// for every dk.
+//
+// TMEM columns: S^T [0, DK), P buffers [DK, DK + 128*NP), O [DK + 128*NP, +128).
+// DK = 256 fits one P buffer (512 columns in all); DK <= 128 double-buffers P.
+//
+// Decay factors come from a per-CTA table pw[n] = gamma^n, n = 0..128 (exp2 of
+// n*log2(gamma), gamma^0 = 1): the intra-block mask uses pw[i-j], xi = pw[i+1],
+// zeta = pw[l-1-j], the state rescale pw[l].  No negative exponent appears, so
+// small gamma underflows to 0 instead of overflowing.
+//
+// Long sequences with few (b, h) are split into segments run by separate CTAs:
+// chunk_state_kernel computes each segment's decayed K^T V sum, state_scan_kernel
+// turns those into every segment's initial state, and the main kernel starts
+// each segment from its own state.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include "tc_common.cuh"
+
+namespace ret {
+
+constexpr int kCW_Threads = 192;
+constexpr int kCW_DVT = 128;       // dv columns per CTA
+constexpr int kCW_MaxStages = 4;
+constexpr uint32_t kSmemAlign = 1024;
+constexpr uint32_t kMiscBytes = 1024;
+
+struct CwDecay {
+  float l2g[1024];  // per-head log2(gamma); -inf for gamma = 0 (RET_MAX_HEADS)
+};
+
+struct CwArgs {
+  int B, H, L, dv, C;
+  int seg_chunks;           // blocks per segment
+  int n_seg;                // segments per (b, h)
+  int nstages;
+  __nv_bfloat16* y;
+  const float* state_in;    // initial state when n_seg == 1 (may be null = zeros)
+  float* state_out;         // may be null
+  const float* seg_state;   // [BH][n_seg][dk][dv] initial states when n_seg > 1
+  WaitLimit lim;
+};
+
+struct CwSmem {
+  uint32_t q, k, v, sb, misc, total;
+  uint32_t q_stage, k_stage, v_stage;
+};
+
+// Shared-memory plan (byte offsets from a 1024-aligned base).  Q stages keep
+// 128 rows per 64-column box so the M = 128 MMA reads only zeros past row C.
+__host__ __device__ inline CwSmem cw_smem_plan(int DK, int C, int ns) {
+  CwSmem s;
+  s.q_stage = (uint32_t)(DK / 64) * 128u * 128u;
+  s.k_stage = (uint32_t)(DK / 64) * (uint32_t)C * 128u;
+  s.v_stage = 2u * (uint32_t)C * 128u;
+  s.q = 0;
+  s.k = s.q + (uint32_t)ns * s.q_stage;
+  s.v = s.k + (uint32_t)ns * s.k_stage;
+  s.sb = s.v + (uint32_t)ns * s.v_stage;
+  s.misc = s.sb + (uint32_t)(DK / 64) * 128u * 128u;
+  s.total = s.misc + kMiscBytes + kSmemAlign;  // + slack for aligning the base
+  return s;
+}
+
+__device__ __forceinline__ uint8_t* align_smem(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + (kSmemAlign - 1)) &
+                                    ~uintptr_t(kSmemAlign - 1));
+}
+
+// Waits that ignore the abort flag (time-bounded only): used at teardown to
+// drain copies and MMAs still in flight before the CTA releases its memory.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, WaitLimit lim) {
+  int dummy = 0;
+  mbar_wait(bar, parity, &dummy, lim);
+}
+
+// Scale the 128-byte row r of a 128B-swizzled bf16 tile in place by f.
+__device__ __forceinline__ void scale_row_sw128(uint8_t* tile, uint32_t r, float f) {
+#pragma unroll
+  for (uint32_t c = 0; c < 8; ++c) {
+    uint4* p = reinterpret_cast<uint4*>(tile + sw128_off(r, c));
+    uint4 w = *p;
+    w.x = pack_bf16x2(bf16lo_to_f32(w.x) * f, bf16hi_to_f32(w.x) * f);
+    w.y = pack_bf16x2(bf16lo_to_f32(w.y) * f, bf16hi_to_f32(w.y) * f);
+    w.z = pack_bf16x2(bf16lo_to_f32(w.z) * f, bf16hi_to_f32(w.z) * f);
+    w.w = pack_bf16x2(bf16lo_to_f32(w.w) * f, bf16hi_to_f32(w.w) * f);
+    *p = w;
+  }
+}
+
+// Write 32 floats as bf16 into row r, columns [c0, c0+32) of a 128B-swizzled
+// tile made of 64-column boxes of `box_bytes` bytes each.
+__device__ __forceinline__ void store_row32_sw128(uint8_t* tile, uint32_t box_bytes, uint32_t r,
+                                                  uint32_t c0, const float* x) {
+  uint8_t* box = tile + (c0 / 64) * box_bytes;
+  const uint32_t ch0 = (c0 % 64) / 8;
+#pragma unroll
+  for (uint32_t q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(x[8 * q + 0], x[8 * q + 1]);
+    w.y = pack_bf16x2(x[8 * q + 2], x[8 * q + 3]);
+    w.z = pack_bf16x2(x[8 * q + 4], x[8 * q + 5]);
+    w.w = pack_bf16x2(x[8 * q + 6], x[8 * q + 7]);
+    *reinterpret_cast<uint4*>(box + sw128_off(r, ch0 + q)) = w;
+  }
+}
+
+template <int DK>
+__global__ void __launch_bounds__(kCW_Threads, 1)
+chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                    const __grid_constant__ CUtensorMap mapV, const CwArgs a,
+                    const __grid_constant__ CwDecay dec) {
+  static_assert(DK == 64 || DK == 128 || DK == 256, "dk must be 64, 128 or 256");
+  constexpr int NP = (DK <= 128) ? 2 : 1;
+  constexpr uint32_t TM_S = 0, TM_P = DK, TM_O = DK + 128 * NP;
+  constexpr uint32_t kTmemCols = 512;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align_smem(smem_raw);
+  const int C = a.C, NS = a.nstages;
+  const CwSmem sp = cw_smem_plan(DK, C, NS);
+  uint8_t* sQ = base + sp.q;
+  uint8_t* sK = base + sp.k;
+  uint8_t* sV = base + sp.v;
+  uint8_t* sSb = base + sp.sb;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + sp.misc);
+  uint64_t* full = bars;             // [4] TMA -> consumers
+  uint64_t* empty = bars + 4;        // [4] MMA5 done -> producer
+  uint64_t* pfull = bars + 8;        // [2] MMA1 done -> epilogue
+  uint64_t* pfree = bars + 10;       // [2] MMA3 done (P~ consumed) -> MMA1 of a later block
+  uint64_t* ocross = bars + 12;      // MMA4 done -> epilogue
+  uint64_t* e1done = bars + 13;      // epilogue (P~, zeta K, xi O ready) -> MMA3/MMA5
+  uint64_t* e2done = bars + 14;      // epilogue (Sb, rescaled S, O drained) -> MMA4 of next block
+  uint64_t* mma35 = bars + 15;       // MMA3+MMA5 done -> epilogue
+  uint64_t* fin = bars + 16;         // teardown drain of the MMA pipe
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17) + 1;
+  float* pw = reinterpret_cast<float*>(bars + 18);  // gamma^0..gamma^128
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int vt = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;
+  const float l2g = dec.l2g[bh % a.H];
+  const int n_total = (a.L + C - 1) / C;
+  const int c_begin = seg * a.seg_chunks;
+  const int c_end = min(c_begin + a.seg_chunks, n_total);
+  const int nck = max(c_end - c_begin, 0);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&pfull[i], 1);
+      mbar_init(&pfree[i], 1);
+    }
+    mbar_init(ocross, 1);
+    mbar_init(e1done, 128);
+    mbar_init(e2done, 128);
+    mbar_init(mma35, 1);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int n = threadIdx.x; n <= 128; n += kCW_Threads) pw[n] = n == 0 ? 1.f : exp2f((float)n * l2g);
+  if (C < 128) {  // rows C..127 of every Q box are read by the M = 128 MMA: keep them zero
+    const uint32_t rows_bytes = (128u - (uint32_t)C) * 128u;
+    const uint32_t per_stage = (uint32_t)(DK / 64) * rows_bytes / 16u;
+    for (uint32_t e = threadIdx.x; e < (uint32_t)NS * per_stage; e += kCW_Threads) {
+      const uint32_t s = e / per_stage, rem = e % per_stage;
+      const uint32_t b = rem / (rows_bytes / 16u), o = rem % (rows_bytes / 16u);
+      *reinterpret_cast<uint4*>(sQ + s * sp.q_stage + b * 16384u + (uint32_t)C * 128u + o * 16u) =
+          make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nck > 0) {
+      tma_prefetch_desc(&mapQ);
+      tma_prefetch_desc(&mapK);
+      tma_prefetch_desc(&mapV);
+      const uint32_t bytes = (uint32_t)(2 * DK + kCW_DVT) * (uint32_t)C * 2u;
+      int issued = 0;
+      for (int it = 0; it < nck; ++it) {
+        const int s = it % NS;
+        if (it >= NS && !mbar_wait(&empty[s], ((it / NS) - 1) & 1, abort_flag, a.lim)) break;
+        const int t0 = (c_begin + it) * C;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        for (int b = 0; b < DK / 64; ++b)
+          tma_load_3d(sQ + s * sp.q_stage + b * 16384, &mapQ, &full[s], b * 64, t0, bh);
+        for (int b = 0; b < DK / 64; ++b)
+          tma_load_3d(sK + s * sp.k_stage + b * C * 128, &mapK, &full[s], b * 64, t0, bh);
+        for (int b = 0; b < 2; ++b)
+          tma_load_3d(sV + s * sp.v_stage + b * C * 128, &mapV, &full[s], vt * kCW_DVT + b * 64, t0, bh);
+        issued = it + 1;
+      }
+      // every load issued must land before the CTA may exit
+      for (int it = max(0, issued - NS); it < issued; ++it) mbar_drain(&full[it % NS], (it / NS) & 1, a.lim);
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0 && nck > 0) {
+      const uint32_t id1 = idesc_bf16(128, C, false, false);
+      const uint32_t id4 = idesc_bf16(128, kCW_DVT, false, false);
+      const uint32_t id3 = idesc_bf16(128, kCW_DVT, false, true);
+      const uint32_t id5 = idesc_bf16(128, DK, true, true);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aSb = smem_u32(sSb);
+      for (int it = 0; it < nck; ++it) {
+        const int s = it % NS, pb = it % NP;
+        if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) break;
+        if (it >= NP && !mbar_wait(&pfree[pb], ((it / NP) - 1) & 1, abort_flag, a.lim)) break;
+        tc_fence_after();
+        const uint32_t q_s = aQ + s * sp.q_stage, k_s = aK + s * sp.k_stage, v_s = aV + s * sp.v_stage;
+        // MMA1: P = Q K^T
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(q_s + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(k_s + (kk / 4) * C * 128 + (kk % 4) * 32, 16, 1024);
+          mma_ss(tm + TM_P + pb * 128, ad, bd, id1, kk > 0);
+        }
+        mma_commit(&pfull[pb]);
+        // MMA4: O = Q S_prev (bf16 copy of the state, written by the epilogue)
+        if (!mbar_wait(e2done, it & 1, abort_flag, a.lim)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(q_s + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(aSb + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          mma_ss(tm + TM_O, ad, bd, id4, kk > 0);
+        }
+        mma_commit(ocross);
+        // MMA3: O += P~ V ; MMA5: S^T += V^T (zeta K)
+        if (!mbar_wait(e1done, it & 1, abort_flag, a.lim)) break;
+        tc_fence_after();
+        for (int kk = 0; kk < C / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(v_s + kk * 2048, C * 128, 1024);
+          mma_ts(tm + TM_O, tm + TM_P + pb * 128 + kk * 8, bd, id3, 1);
+        }
+        mma_commit(&pfree[pb]);
+        for (int kk = 0; kk < C / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(v_s + kk * 2048, C * 128, 1024);
+          const uint64_t bd = sdesc_sw128(k_s + kk * 2048, C * 128, 1024);
+          mma_ss(tm + TM_S, ad, bd, id5, 1);
+        }
+        mma_commit(mma35);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(fin);
+      mbar_drain(fin, 0, a.lim);
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const uint32_t r = threadIdx.x;                 // TMEM lane == row of P / O, column of S
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int v = vt * kCW_DVT + (int)r;            // this thread's dv column
+    const size_t dkdv = (size_t)DK * a.dv;
+    // initial state: S_prev (bf16 copy for MMA4) and gamma^l0 S_prev (accumulator for MMA5)
+    {
+      const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
+                                       : (a.state_in ? a.state_in + (size_t)bh * dkdv : nullptr);
+      const int l0 = min(C, a.L - c_begin * C);
+      const float g0 = pw[max(l0, 0)];
+      for (int d0 = 0; d0 < DK; d0 += 32) {
+        float x[32];
+        uint32_t w[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          x[u] = src ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
+          w[u] = __float_as_uint(g0 * x[u]);
+        }
+        store_row32_sw128(sSb, 16384, r, d0, x);
+        tmem_st32(tm + lane_off + TM_S + d0, w);
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(e2done);
+    }
+    for (int it = 0; it < nck; ++it) {
+      const int s = it % NS, pb = it % NP;
+      const int t0 = (c_begin + it) * C;
+      const int l = min(C, a.L - t0);
+      if (!mbar_wait(&pfull[pb], (it / NP) & 1, abort_flag, a.lim)) break;
+      if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) break;
+      tc_fence_after();
+      // E1a: P -> P~ = bf16(P * gamma^(r-j)) for j <= r < l, else 0 (in place, two per column)
+      const uint32_t tp = tm + lane_off + TM_P + pb * 128;
+      for (int j0 = 0; j0 < C; j0 += 32) {
+        uint32_t pr[32];
+        tmem_ld32(tp + j0, pr);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int u = 0; u < 32; u += 2) {
+          const int j = j0 + u;
+          const float f0 = (j <= (int)r && (int)r < l) ? pw[r - j] : 0.f;
+          const float f1 = (j + 1 <= (int)r && (int)r < l) ? pw[r - j - 1] : 0.f;
+          w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * f0, __uint_as_float(pr[u + 1]) * f1);
+        }
+        // When C % 32 == 16 the last piece also covers 16 columns past C; their
+        // packed results land at columns >= C/2, which MMA3 never reads.
+        tmem_st16(tp + j0 / 2, w);
+      }
+      // E1b: row j of K scaled by zeta_j = gamma^(l-1-j) (0 past the block end)
+      if ((int)r < C) {
+        const float zeta = ((int)r < l) ? pw[l - 1 - (int)r] : 0.f;
+        uint8_t* ks = sK + s * sp.k_stage;
+        for (int b = 0; b < DK / 64; ++b) scale_row_sw128(ks + b * C * 128, r, zeta);
+      }
+      fence_proxy_async_smem();
+      // E1c: O *= xi_r = gamma^(r+1)
+      if (!mbar_wait(ocross, it & 1, abort_flag, a.lim)) break;
+      tc_fence_after();
+      {
+        const float xi = pw[r + 1];
+        for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tm + lane_off + TM_O + c0, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * xi);
+          tmem_st32(tm + lane_off + TM_O + c0, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(e1done);
+      // E2: state -> bf16 copy + rescale (or state_out); O -> y
+      if (!mbar_wait(mma35, it & 1, abort_flag, a.lim)) break;
+      tc_fence_after();
+      const bool last = (it == nck - 1);
+      if (!last) {
+        const float gn = pw[min(C, a.L - t0 - C)];
+        for (int d0 = 0; d0 < DK; d0 += 32) {
+          uint32_t sr[32];
+          tmem_ld32(tm + lane_off + TM_S + d0, sr);
+          tmem_ld_wait();
+          float x[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            x[u] = __uint_as_float(sr[u]);
+            sr[u] = __float_as_uint(gn * x[u]);
+          }
+          store_row32_sw128(sSb, 16384, r, d0, x);
+          tmem_st32(tm + lane_off + TM_S + d0, sr);
+        }
+      } else if (a.state_out && seg == a.n_seg - 1) {
+        float* so = a.state_out + (size_t)bh * dkdv;
+        for (int d0 = 0; d0 < DK; d0 += 32) {
+          uint32_t sr[32];
+          tmem_ld32(tm + lane_off + TM_S + d0, sr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) so[(size_t)(d0 + u) * a.dv + v] = __uint_as_float(sr[u]);
+        }
+      }
+      {
+        __nv_bfloat16* yrow = a.y + ((size_t)bh * a.L + t0 + r) * a.dv + vt * kCW_DVT;
+        for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tm + lane_off + TM_O + c0, o);
+          tmem_ld_wait();
+          if ((int)r < l) {
+            uint4* dst = reinterpret_cast<uint4*>(yrow + c0);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * q4 + 0]), __uint_as_float(o[8 * q4 + 1]));
+              w.y = pack_bf16x2(__uint_as_float(o[8 * q4 + 2]), __uint_as_float(o[8 * q4 + 3]));
+              w.z = pack_bf16x2(__uint_as_float(o[8 * q4 + 4]), __uint_as_float(o[8 * q4 + 5]));
+              w.w = pack_bf16x2(__uint_as_float(o[8 * q4 + 6]), __uint_as_float(o[8 * q4 + 7]));
+              dst[q4] = w;
+            }
+          }
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(e2done);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tm, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------
+// Segment sums for the sequence split: for segment g of one (b, h) and one
+// 128-column dv slice,  D_g^T = sum_{t in g} gamma^(e_g - t) v_t^T k_t  with e_g
+// the segment's last token, written (as [dk][dv], like a state) to slot g+1 of
+// the workspace [BH][n_seg][dk][dv].  Rows of K are scaled by the decay to the
+// segment end in shared memory, then accumulated by tcgen05 into TMEM.
+template <int DK>
+__global__ void __launch_bounds__(kCW_Threads)
+chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                   const CwArgs a, const __grid_constant__ CwDecay dec, float* ws) {
+  constexpr uint32_t kTmemCols = DK;  // 64, 128 or 256: powers of two >= 32
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align_smem(smem_raw);
+  const int C = a.C, NS = a.nstages;
+  const uint32_t k_stage = (uint32_t)(DK / 64) * C * 128, v_stage = 2u * C * 128;
+  uint8_t* sK = base;
+  uint8_t* sV = base + NS * k_stage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + NS * (k_stage + v_stage));
+  uint64_t* full = bars;        // [4]
+  uint64_t* empty = bars + 4;   // [4]
+  uint64_t* kready = bars + 8;  // [4] epilogue scaled K -> MMA
+  uint64_t* done = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13) + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int vt = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;  // seg < n_seg - 1
+  const float l2g = dec.l2g[bh % a.H];
+  const int n_total = (a.L + C - 1) / C;
+  const int c_begin = seg * a.seg_chunks;
+  const int c_end = min(c_begin + a.seg_chunks, n_total);
+  const int nck = max(c_end - c_begin, 0);
+  const int seg_last = min(c_end * C, a.L) - 1;  // e_g
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+      mbar_init(&kready[i], 128);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0 && nck > 0) {
+      const uint32_t bytes = (uint32_t)(DK + kCW_DVT) * C * 2u;
+      int issued = 0;
+      for (int it = 0; it < nck; ++it) {
+        const int s = it % NS;
+        if (it >= NS && !mbar_wait(&empty[s], ((it / NS) - 1) & 1, abort_flag, a.lim)) break;
+        const int t0 = (c_begin + it) * C;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        for (int b = 0; b < DK / 64; ++b)
+          tma_load_3d(sK + s * k_stage + b * C * 128, &mapK, &full[s], b * 64, t0, bh);
+        for (int b = 0; b < 2; ++b)
+          tma_load_3d(sV + s * v_stage + b * C * 128, &mapV, &full[s], vt * kCW_DVT + b * 64, t0, bh);
+        issued = it + 1;
+      }
+      for (int it = max(0, issued - NS); it < issued; ++it) mbar_drain(&full[it % NS], (it / NS) & 1, a.lim);
+    }
+  } else if (warp == 5) {
+    if (lane == 0 && nck > 0) {
+      const uint32_t id5 = idesc_bf16(128, DK, true, true);
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+      for (int it = 0; it < nck; ++it) {
+        const int s = it % NS;
+        if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) break;
+        if (!mbar_wait(&kready[s], (it / NS) & 1, abort_flag, a.lim)) break;
+        tc_fence_after();
+        for (int kk = 0; kk < C / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(aV + s * v_stage + kk * 2048, C * 128, 1024);
+          const uint64_t bd = sdesc_sw128(aK + s * k_stage + kk * 2048, C * 128, 1024);
+          mma_ss(tm, ad, bd, id5, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(done);
+    }
+  } else {
+    const uint32_t r = threadIdx.x;
+    bool ok = true;
+    for (int it = 0; it < nck; ++it) {
+      const int s = it % NS;
+      if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) { ok = false; break; }
+      if ((int)r < C) {
+        const int t = (c_begin + it) * C + (int)r;
+        const float f = (t <= seg_last) ? (t == seg_last ? 1.f : exp2f((float)(seg_last - t) * l2g)) : 0.f;
+        for (int b = 0; b < DK / 64; ++b) scale_row_sw128(sK + s * k_stage + b * C * 128, r, f);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&kready[s]);
+    }
+    if (ok && nck > 0 && mbar_wait(done, 0, abort_flag, a.lim)) {
+      tc_fence_after();
+      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+      const size_t dkdv = (size_t)DK * a.dv;
+      float* dst = ws + ((size_t)bh * a.n_seg + seg + 1) * dkdv;
+      const int v = vt * kCW_DVT + (int)r;
+      for (int d0 = 0; d0 < DK; d0 += 32) {
+        uint32_t sr[32];
+        tmem_ld32(tm + lane_off + d0, sr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) dst[(size_t)(d0 + u) * a.dv + v] = __uint_as_float(sr[u]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    if (lane == 0 && nck > 0) {
+      // no MMA may still be running when TMEM is released
+      mbar_drain(done, 0, a.lim);
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tm, kTmemCols);
+  }
+}
+
+// Scan over segments, element-wise on the state: slot 0 <- S_in, and for
+// g = 1..n_seg-1, slot g <- gamma^len * slot(g-1) + D_(g-1) (D_(g-1) was stored in
+// slot g by chunk_state_kernel).  len = tokens per segment (all but the last
+// segment are full).
+__global__ void state_scan_kernel(const float* __restrict__ state_in, float* __restrict__ ws,
+                                  int BH, int H, int dkdv, int n_seg, int seg_len,
+                                  const __grid_constant__ CwDecay dec) {
+  const size_t total = (size_t)BH * dkdv;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (size_t)gridDim.x * blockDim.x) {
+    const int bh = (int)(e / dkdv);
+    const size_t off = e % dkdv;
+    const float gl = exp2f((float)seg_len * dec.l2g[bh % H]);
+    float S = state_in ? state_in[e] : 0.f;
+    float* slot = ws + (size_t)bh * n_seg * dkdv + off;
+    slot[0] = S;
+    for (int g = 1; g < n_seg; ++g) {
+      S = fmaf(gl, S, slot[(size_t)g * dkdv]);
+      slot[(size_t)g * dkdv] = S;
+    }
+  }
+}
+
+}  // namespace ret

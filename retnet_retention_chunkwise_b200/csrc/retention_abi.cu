@@ -1,0 +1,416 @@
+// retention_abi.cu -- the C ABI of libretention (declared in include/retention.h):
+// argument validation, TMA descriptor encoding, launch configuration.
+//
+// The whole library is this one translation unit (the kernels live in the
+// included .cuh files), so the device status word has a single definition.
+// No function here allocates memory; every launch goes to the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/retention.h"
+#include "chunkwise_tc.cuh"
+#include "decode.cuh"
+#include "parallel_tc.cuh"
+#include "simt_f32.cuh"
+#include "tc_common.cuh"
+
+namespace {
+
+using namespace ret;
+
+// Wall-clock budget of any single wait inside a kernel.  A healthy wait is
+// microseconds; this only bounds a kernel whose pipeline broke.
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
+constexpr uint32_t kWaitIter = 1u << 30;
+
+WaitLimit wait_limit() {
+  WaitLimit w{kWaitNs, kWaitIter};
+  static int env_ms = -1;
+  if (env_ms < 0) {
+    const char* e = getenv("RETENTION_WAIT_LIMIT_MS");
+    env_ms = e ? atoi(e) : 0;
+    if (env_ms < 0) env_ms = 0;
+  }
+  if (env_ms > 0) w.ns = (uint64_t)env_ms * 1000000ull;
+  return w;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 view [n_heads][rows][inner] with a 64 x box_rows box, 128-byte swizzle.
+// Rows past the end of a head read as zero.
+bool make_map(CUtensorMap* m, const void* ptr, int inner, int rows, int n_heads, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)n_heads};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * rows * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ret_status check_gamma(const float* gamma, int H) {
+  if (!gamma) return RET_EINVAL;
+  for (int h = 0; h < H; ++h)
+    if (!(gamma[h] >= 0.f && gamma[h] <= 1.f)) return RET_EINVAL;  // also rejects NaN
+  return RET_OK;
+}
+
+ret_status check_shape(const ret_shape& s, bool need_L) {
+  if (s.B < 1 || s.H < 1 || s.dk < 1 || s.dv < 1) return RET_EINVAL;
+  if (need_L && s.L < 0) return RET_EINVAL;
+  if (s.H > RET_MAX_HEADS) return RET_EUNSUPPORTED;
+  if ((long long)s.B * s.H > 65535) return RET_EUNSUPPORTED;  // grid.y / grid.z limit
+  return RET_OK;
+}
+
+// Tensor-core path requires an sm_100 device.
+bool device_is_sm100() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  return major == 10;
+}
+
+int max_smem_optin() {
+  int dev = 0, v = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  return v;
+}
+
+float log2_gamma(float g) {
+  // log2 in double, rounded once; gamma = 0 -> -inf so gamma^n = exp2(-inf) = 0 for n >= 1
+  return g == 0.f ? -INFINITY : (float)std::log2((double)g);
+}
+
+void fill_l2g(CwDecay& d, const float* gamma, int H) {
+  for (int h = 0; h < H; ++h) d.l2g[h] = log2_gamma(gamma[h]);
+}
+
+ret_status launch_status() { return cudaGetLastError() == cudaSuccess ? RET_OK : RET_ECUDA; }
+
+bool tc_shape_ok(const ret_shape& s) {
+  return (s.dk == 64 || s.dk == 128 || s.dk == 256) && (s.dv % kCW_DVT) == 0;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// Sequence split for the chunkwise tensor-core path: enough segments to give
+// every SM a CTA, each segment at least two blocks long.
+void plan_segments(const ret_shape& s, int C, int* n_seg, int* seg_chunks) {
+  const int n_chunks = (s.L + C - 1) / C;
+  const long long base = (long long)(s.dv / kCW_DVT) * s.B * s.H;
+  int g = 1;
+  if (base < sm_count()) g = (int)(sm_count() / base);
+  g = std::max(1, std::min(g, n_chunks / 2));
+  const int sc = (n_chunks + g - 1) / g;
+  *seg_chunks = std::max(sc, 1);
+  *n_seg = (n_chunks + *seg_chunks - 1) / *seg_chunks;
+}
+
+size_t seg_workspace_bytes(const ret_shape& s, int n_seg) {
+  if (n_seg <= 1) return 0;
+  return (size_t)s.B * s.H * n_seg * (size_t)s.dk * s.dv * sizeof(float);
+}
+
+template <int DK>
+ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, const float* gamma,
+                               void* y, const float* state_in, float* state_out, int C,
+                               const ret_shape& s, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int BH = s.B * s.H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, DK, s.L, BH, C) || !make_map(&mk, k, DK, s.L, BH, C) ||
+      !make_map(&mv, v, s.dv, s.L, BH, C))
+    return RET_ECUDA;
+  static CwDecay dec;  // staged on the host; copied into the launch's parameters
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  fill_l2g(dec, gamma, s.H);
+
+  const int smax = max_smem_optin();
+  int ns = 0;
+  for (int n = kCW_MaxStages; n >= 1; --n)
+    if ((int)cw_smem_plan(DK, C, n).total <= smax) { ns = n; break; }
+  if (ns == 0) return RET_EUNSUPPORTED;
+  CwSmem plan = cw_smem_plan(DK, C, ns);
+
+  int n_seg = 1, seg_chunks = 0;
+  plan_segments(s, C, &n_seg, &seg_chunks);
+  while (n_seg > 1 && (ws == nullptr || seg_workspace_bytes(s, n_seg) > ws_bytes)) {
+    // not enough workspace for this split: fall back to fewer segments
+    const int n_chunks = (s.L + C - 1) / C;
+    int g = n_seg - 1;
+    seg_chunks = (n_chunks + g - 1) / g;
+    n_seg = (n_chunks + seg_chunks - 1) / seg_chunks;
+  }
+  if (n_seg <= 1) {
+    n_seg = 1;
+    seg_chunks = (s.L + C - 1) / C;
+  }
+
+  CwArgs a;
+  a.B = s.B;
+  a.H = s.H;
+  a.L = s.L;
+  a.dv = s.dv;
+  a.C = C;
+  a.seg_chunks = seg_chunks;
+  a.n_seg = n_seg;
+  a.nstages = ns;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.state_in = state_in;
+  a.state_out = state_out;
+  a.seg_state = static_cast<const float*>(ws);
+  a.lim = wait_limit();
+
+  if (n_seg > 1) {
+    // segment sums -> workspace slots 1..n_seg-1, then the scan fills every slot
+    int ns2 = 0;
+    const uint32_t per = (uint32_t)(DK / 64) * C * 128 + 2u * C * 128;
+    for (int n = kCW_MaxStages; n >= 1; --n)
+      if ((int)(n * per + kMiscBytes + kSmemAlign) <= smax) { ns2 = n; break; }
+    CwArgs a2 = a;
+    a2.nstages = ns2;
+    const int smem2 = (int)(ns2 * per + kMiscBytes + kSmemAlign);
+    if (cudaFuncSetAttribute(chunk_state_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) !=
+        cudaSuccess)
+      return RET_ECUDA;
+    dim3 g2(s.dv / kCW_DVT, BH, n_seg - 1);
+    chunk_state_kernel<DK><<<g2, kCW_Threads, smem2, st>>>(mk, mv, a2, dec, static_cast<float*>(ws));
+    if (launch_status() != RET_OK) return RET_ECUDA;
+    const long long total = (long long)BH * DK * s.dv;
+    const int blocks = (int)std::min<long long>((total + 255) / 256, 4LL * sm_count());
+    state_scan_kernel<<<blocks, 256, 0, st>>>(state_in, static_cast<float*>(ws), BH, s.H, DK * s.dv,
+                                              n_seg, seg_chunks * C, dec);
+    if (launch_status() != RET_OK) return RET_ECUDA;
+  }
+  if (cudaFuncSetAttribute(chunkwise_tc_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)plan.total) != cudaSuccess)
+    return RET_ECUDA;
+  dim3 grid(s.dv / kCW_DVT, BH, n_seg);
+  chunkwise_tc_kernel<DK><<<grid, kCW_Threads, plan.total, st>>>(mq, mk, mv, a, dec);
+  return launch_status();
+}
+
+template <int DK>
+ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const float* gamma, void* y,
+                              const ret_shape& s, cudaStream_t st) {
+  const int BH = s.B * s.H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, DK, s.L, BH, 128) || !make_map(&mk, k, DK, s.L, BH, 128) ||
+      !make_map(&mv, v, s.dv, s.L, BH, 128))
+    return RET_ECUDA;
+  static CwDecay dec;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  fill_l2g(dec, gamma, s.H);
+  const int smax = max_smem_optin();
+  int ns = 0;
+  for (int n = kCW_MaxStages; n >= 1; --n)
+    if ((int)pa_smem_plan(DK, n).total <= smax) { ns = n; break; }
+  if (ns == 0) return RET_EUNSUPPORTED;
+  const PaSmem plan = pa_smem_plan(DK, ns);
+  PaArgs a;
+  a.B = s.B;
+  a.H = s.H;
+  a.L = s.L;
+  a.dv = s.dv;
+  a.n_qt = (s.L + 127) / 128;
+  a.nstages = ns;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.lim = wait_limit();
+  if (cudaFuncSetAttribute(parallel_tc_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)plan.total) != cudaSuccess)
+    return RET_ECUDA;
+  dim3 grid(s.dv / 128, a.n_qt, BH);
+  parallel_tc_kernel<DK><<<grid, kCW_Threads, plan.total, st>>>(mq, mk, mv, a, dec);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int retention_abi_version(void) { return 100; }
+
+const char* retention_status_str(ret_status st) {
+  switch (st) {
+    case RET_OK: return "RET_OK";
+    case RET_EINVAL: return "RET_EINVAL";
+    case RET_EUNSUPPORTED: return "RET_EUNSUPPORTED";
+    case RET_ECUDA: return "RET_ECUDA";
+    case RET_ETIMEOUT: return "RET_ETIMEOUT";
+  }
+  return "RET_UNKNOWN";
+}
+
+ret_status retention_get_device_status(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RET_ECUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_device_status, sizeof(int)) != cudaSuccess) return RET_ECUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return RET_ECUDA;
+    return RET_ETIMEOUT;
+  }
+  return RET_OK;
+}
+
+ret_status retention_recurrent_step(const void* q, const void* k, const void* v, const float* gamma,
+                                    void* y, float* state, ret_shape s, ret_dtype dt, void* stream) {
+  ret_status rc = check_shape(s, false);
+  if (rc != RET_OK) return rc;
+  if (!q || !k || !v || !y || !state) return RET_EINVAL;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
+  if (s.dk > kDecodeMaxDk) return RET_EUNSUPPORTED;
+  if (!aligned16(state)) return RET_EINVAL;
+  static HeadGamma hg;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int h = 0; h < s.H; ++h) hg.g[h] = gamma[h];
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dim3 grid((s.dv + kDecodeCols - 1) / kDecodeCols, s.B * s.H);
+  const bool vec = (s.dv % 4) == 0;
+  if (dt == RET_F32) {
+    auto* qf = static_cast<const float*>(q);
+    auto* kf = static_cast<const float*>(k);
+    auto* vf = static_cast<const float*>(v);
+    auto* yf = static_cast<float*>(y);
+    if (vec) recurrent_step_kernel<float, true><<<grid, kDecodeThreads, 0, st>>>(qf, kf, vf, yf, state, s.H, s.dk, s.dv, hg);
+    else recurrent_step_kernel<float, false><<<grid, kDecodeThreads, 0, st>>>(qf, kf, vf, yf, state, s.H, s.dk, s.dv, hg);
+  } else {
+    auto* qb = static_cast<const __nv_bfloat16*>(q);
+    auto* kb = static_cast<const __nv_bfloat16*>(k);
+    auto* vb = static_cast<const __nv_bfloat16*>(v);
+    auto* yb = static_cast<__nv_bfloat16*>(y);
+    if (vec) recurrent_step_kernel<__nv_bfloat16, true><<<grid, kDecodeThreads, 0, st>>>(qb, kb, vb, yb, state, s.H, s.dk, s.dv, hg);
+    else recurrent_step_kernel<__nv_bfloat16, false><<<grid, kDecodeThreads, 0, st>>>(qb, kb, vb, yb, state, s.H, s.dk, s.dv, hg);
+  }
+  return launch_status();
+}
+
+ret_status retention_parallel(const void* q, const void* k, const void* v, const float* gamma, void* y,
+                              ret_shape s, ret_dtype dt, void* stream) {
+  ret_status rc = check_shape(s, true);
+  if (rc != RET_OK) return rc;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (s.L == 0) return RET_OK;
+  if (!q || !k || !v || !y) return RET_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y)) return RET_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == RET_F32) {
+    if (s.dk > 256) return RET_EUNSUPPORTED;
+    static HeadLog2 hl;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int h = 0; h < s.H; ++h) hl.l2g[h] = log2_gamma(gamma[h]);
+    const int smem = (2 * kPF_Rows * (s.dk + 1) + kPF_Rows * kPF_Cols + kPF_Rows * 33) * 4;
+    if (cudaFuncSetAttribute(parallel_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return RET_ECUDA;
+    dim3 grid((s.dv + kPF_Cols - 1) / kPF_Cols, (s.L + kPF_Rows - 1) / kPF_Rows, s.B * s.H);
+    parallel_f32_kernel<<<grid, 256, smem, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
+                                                 static_cast<const float*>(v), static_cast<float*>(y), s.H, s.L,
+                                                 s.dk, s.dv, hl);
+    return launch_status();
+  }
+  if (dt != RET_BF16) return RET_EINVAL;
+  if (!tc_shape_ok(s) || !device_is_sm100()) return RET_EUNSUPPORTED;
+  switch (s.dk) {
+    case 64: return launch_parallel_tc<64>(q, k, v, gamma, y, s, st);
+    case 128: return launch_parallel_tc<128>(q, k, v, gamma, y, s, st);
+    default: return launch_parallel_tc<256>(q, k, v, gamma, y, s, st);
+  }
+}
+
+size_t retention_chunkwise_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
+  if (dt != RET_BF16 || chunk < 16 || chunk > 128 || chunk % 16 != 0) return 0;
+  if (check_shape(s, true) != RET_OK || s.L < 1 || !tc_shape_ok(s)) return 0;
+  int n_seg = 1, seg_chunks = 1;
+  plan_segments(s, chunk, &n_seg, &seg_chunks);
+  return seg_workspace_bytes(s, n_seg);
+}
+
+ret_status retention_chunkwise(const void* q, const void* k, const void* v, const float* gamma, void* y,
+                               const float* state_in, float* state_out, int chunk, ret_shape s,
+                               ret_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+  ret_status rc = check_shape(s, true);
+  if (rc != RET_OK) return rc;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (chunk < 1) return RET_EINVAL;
+  if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
+  if (s.L > 0 && (!q || !k || !v || !y)) return RET_EINVAL;
+  if (s.L > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y))) return RET_EINVAL;
+  if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out))) return RET_EINVAL;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RET_EINVAL;
+  if (dt == RET_F32) {
+    if (chunk > kCF_MaxC || s.dk > 256) return RET_EUNSUPPORTED;
+  } else {
+    if (chunk < 16 || chunk > 128 || chunk % 16 != 0) return RET_EUNSUPPORTED;
+    if (!tc_shape_ok(s)) return RET_EUNSUPPORTED;
+    if (s.L > 0 && !device_is_sm100()) return RET_EUNSUPPORTED;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t sbytes = (size_t)s.B * s.H * s.dk * s.dv * sizeof(float);
+  if (s.L == 0) {  // nothing to compute: the state passes through
+    if (!state_out) return RET_OK;
+    cudaError_t e = state_in ? (state_in == state_out ? cudaSuccess
+                                                      : cudaMemcpyAsync(state_out, state_in, sbytes,
+                                                                        cudaMemcpyDeviceToDevice, st))
+                             : cudaMemsetAsync(state_out, 0, sbytes, st);
+    return e == cudaSuccess ? RET_OK : RET_ECUDA;
+  }
+  if (dt == RET_F32) {
+    static HeadLog2 hl;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int h = 0; h < s.H; ++h) hl.l2g[h] = log2_gamma(gamma[h]);
+    const int smem = (s.dk * kCF_Cols + chunk * (chunk + 1) + chunk + 1) * 4;
+    if (cudaFuncSetAttribute(chunkwise_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return RET_ECUDA;
+    dim3 grid((s.dv + kCF_Cols - 1) / kCF_Cols, s.B * s.H);
+    chunkwise_f32_kernel<<<grid, 256, smem, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
+                                                  static_cast<const float*>(v), static_cast<float*>(y), state_in,
+                                                  state_out, s.H, s.L, s.dk, s.dv, chunk, hl);
+    return launch_status();
+  }
+  switch (s.dk) {
+    case 64: return launch_chunkwise_tc<64>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+    case 128: return launch_chunkwise_tc<128>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+    default: return launch_chunkwise_tc<256>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+  }
+}
+
+}  // extern "C"

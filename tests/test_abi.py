@@ -1,0 +1,131 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* the shared library loads and exports every function include/retention.h declares;
+* invalid arguments are rejected with the documented status before anything is
+  launched (these calls never reach the CUDA runtime, so they run on the CPU).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from retnet_retention_chunkwise_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "retention.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(retention_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _abi.load()
+
+
+def test_header_and_binding_agree():
+    assert _declared() == sorted(_abi.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_only_abi_symbols_are_exported():
+    # built with -fvisibility=hidden: the dynamic symbol table holds the C ABI
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    ours = sorted({ln.split()[-1] for ln in out.splitlines() if ln.split()[-1].startswith("retention_")})
+    assert ours == _declared()
+
+
+def test_status_strings_and_version(lib):
+    names = [lib.retention_status_str(i).decode() for i in range(5)]
+    assert names == ["RET_OK", "RET_EINVAL", "RET_EUNSUPPORTED", "RET_ECUDA", "RET_ETIMEOUT"]
+    assert lib.retention_status_str(99).decode() == "RET_UNKNOWN"
+    assert lib.retention_abi_version() == 100
+
+
+def _g(*vals):
+    return (ctypes.c_float * len(vals))(*vals)
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("gamma", [-0.01, 1.0001, float("nan"), float("inf")])
+def test_bad_gamma_is_einval(lib, gamma):
+    s = _abi.RetShape(1, 1, 8, 64, 128)
+    assert lib.retention_parallel(FAKE, FAKE, FAKE, _g(gamma), FAKE, s, _abi.RET_BF16, None) == _abi.RET_EINVAL
+    assert lib.retention_chunkwise(FAKE, FAKE, FAKE, _g(gamma), FAKE, None, None, 64, s, _abi.RET_BF16,
+                                   None, 0, None) == _abi.RET_EINVAL
+    assert lib.retention_recurrent_step(FAKE, FAKE, FAKE, _g(gamma), FAKE, FAKE, s, _abi.RET_BF16,
+                                        None) == _abi.RET_EINVAL
+
+
+def test_null_gamma_and_pointers_are_einval(lib):
+    s = _abi.RetShape(1, 1, 8, 64, 128)
+    assert lib.retention_parallel(FAKE, FAKE, FAKE, None, FAKE, s, _abi.RET_BF16, None) == _abi.RET_EINVAL
+    assert lib.retention_parallel(None, FAKE, FAKE, _g(0.5), FAKE, s, _abi.RET_BF16, None) == _abi.RET_EINVAL
+    assert lib.retention_chunkwise(FAKE, None, FAKE, _g(0.5), FAKE, None, None, 64, s, _abi.RET_BF16,
+                                   None, 0, None) == _abi.RET_EINVAL
+    assert lib.retention_recurrent_step(FAKE, FAKE, FAKE, _g(0.5), FAKE, None, s, _abi.RET_BF16,
+                                        None) == _abi.RET_EINVAL
+
+
+@pytest.mark.parametrize("shape", [(0, 1, 8, 64, 128), (1, 0, 8, 64, 128), (1, 1, -1, 64, 128),
+                                   (1, 1, 8, 0, 128), (1, 1, 8, 64, 0)])
+def test_bad_shapes_are_einval(lib, shape):
+    s = _abi.RetShape(*shape)
+    g = _g(*([0.5] * max(shape[1], 1)))
+    assert lib.retention_chunkwise(FAKE, FAKE, FAKE, g, FAKE, None, None, 64, s, _abi.RET_BF16,
+                                   None, 0, None) == _abi.RET_EINVAL
+
+
+def test_too_many_heads_is_unsupported(lib):
+    H = _abi.RET_MAX_HEADS + 1
+    s = _abi.RetShape(1, H, 8, 64, 128)
+    assert lib.retention_parallel(FAKE, FAKE, FAKE, _g(*([0.5] * H)), FAKE, s, _abi.RET_BF16,
+                                  None) == _abi.RET_EUNSUPPORTED
+
+
+def test_misaligned_pointers_are_einval(lib):
+    s = _abi.RetShape(1, 1, 8, 64, 128)
+    odd = ctypes.c_void_p(0x10008)
+    assert lib.retention_parallel(odd, FAKE, FAKE, _g(0.5), FAKE, s, _abi.RET_BF16, None) == _abi.RET_EINVAL
+    assert lib.retention_chunkwise(FAKE, FAKE, FAKE, _g(0.5), FAKE, None, None, 64, s, _abi.RET_BF16,
+                                   ctypes.c_void_p(0x10010), 1 << 20, None) == _abi.RET_EINVAL
+
+
+@pytest.mark.parametrize("chunk,dk,dv", [(8, 64, 128), (24, 64, 128), (256, 64, 128), (64, 96, 128),
+                                         (64, 64, 192), (64, 512, 128)])
+def test_unsupported_bf16_shapes(lib, chunk, dk, dv):
+    s = _abi.RetShape(1, 1, 256, dk, dv)
+    assert lib.retention_chunkwise(FAKE, FAKE, FAKE, _g(0.5), FAKE, None, None, chunk, s, _abi.RET_BF16,
+                                   None, 0, None) == _abi.RET_EUNSUPPORTED
+
+
+def test_zero_chunk_is_einval(lib):
+    s = _abi.RetShape(1, 1, 8, 64, 128)
+    assert lib.retention_chunkwise(FAKE, FAKE, FAKE, _g(0.5), FAKE, None, None, 0, s, _abi.RET_F32,
+                                   None, 0, None) == _abi.RET_EINVAL
+
+
+def test_empty_parallel_call_is_a_noop(lib):
+    s = _abi.RetShape(2, 2, 0, 64, 128)
+    assert lib.retention_parallel(None, None, None, _g(0.5, 0.9), None, s, _abi.RET_BF16, None) == _abi.RET_OK
+
+
+def test_workspace_query(lib):
+    few_heads = _abi.RetShape(1, 2, 8192, 64, 128)
+    many_heads = _abi.RetShape(4, 8, 8192, 256, 512)
+    assert lib.retention_chunkwise_workspace_bytes(64, many_heads, _abi.RET_BF16) == 0
+    n = lib.retention_chunkwise_workspace_bytes(64, few_heads, _abi.RET_BF16)
+    assert n > 0 and n % (2 * 64 * 128 * 4) == 0
+    assert lib.retention_chunkwise_workspace_bytes(64, few_heads, _abi.RET_F32) == 0

@@ -1,0 +1,185 @@
+"""GPU parity: every kernel, through the C ABI, against the fp64 oracle.
+
+Metric (per tensor): max |gpu - oracle| / max |oracle|.  Bounds: 1e-4 for fp32
+inputs, 2e-2 for bf16 inputs (fp32 accumulation and state).  Both sides read the
+same seeded bytes; the oracle widens them to fp64 exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import retnet_retention_chunkwise_b200 as ret
+from retnet_retention_chunkwise_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+
+
+def rel(gpu, ref):
+    g = gpu.detach().double().cpu().numpy() if isinstance(gpu, torch.Tensor) else np.asarray(gpu)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert np.all(np.isfinite(g)), "non-finite GPU output"
+    return float(np.max(np.abs(g - ref)) / max(np.max(np.abs(ref)), 1e-30))
+
+
+def dev(*ts):
+    return [None if t is None else t.cuda() for t in ts]
+
+
+@pytest.fixture(autouse=True)
+def _status_clean():
+    yield
+    assert ret.device_status() == 0
+
+
+# ------------------------------------------------------------ fp32 (1e-4)
+def test_single_head_f32_all_forms():
+    w = inputs.WORKLOADS["single_head_f32"]
+    q, k, v = inputs.qkv(w.B, w.H, w.L, w.dk, w.dv, w.dtype, w.seed)
+    gam = w.gammas()
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam)
+    qd, kd, vd = dev(q, k, v)
+    y = ret.parallel(qd, kd, vd, gam)
+    assert rel(y, y_ref) <= 1e-4
+    y, s = ret.chunkwise(qd, kd, vd, gam, w.chunk)
+    assert rel(y, y_ref) <= 1e-4 and rel(s, s_ref) <= 1e-4
+    state = torch.zeros(w.B, w.H, w.dk, w.dv, device="cuda")
+    ys = [ret.recurrent_step(qd[:, :, n:n + 1].contiguous(), kd[:, :, n:n + 1].contiguous(),
+                             vd[:, :, n:n + 1].contiguous(), gam, state) for n in range(w.L)]
+    assert rel(torch.cat(ys, dim=2), y_ref) <= 1e-4 and rel(state, s_ref) <= 1e-4
+
+
+@pytest.mark.parametrize("B,H,L,dk,dv,C", [(2, 3, 37, 16, 24, 16), (1, 2, 130, 64, 40, 32),
+                                           (1, 1, 5, 8, 8, 64), (1, 2, 64, 256, 33, 7)])
+def test_f32_ragged_with_state(B, H, L, dk, dv, C):
+    q, k, v = inputs.qkv(B, H, L, dk, dv, torch.float32, seed=3)
+    s_in = inputs.state(B, H, dk, dv, seed=4, scale=0.3)
+    gam = torch.tensor([0.5, 0.999, 0.0][:H] if H <= 3 else [0.9] * H)
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam, s_in)
+    qd, kd, vd, sd = dev(q, k, v, s_in)
+    y, s = ret.chunkwise(qd, kd, vd, gam, C, state_in=sd)
+    assert rel(y, y_ref) <= 1e-4 and rel(s, s_ref) <= 1e-4
+    y0_ref, _ = oracle.recurrent(q, k, v, gam)
+    assert rel(ret.parallel(qd, kd, vd, gam), y0_ref) <= 1e-4
+
+
+# ------------------------------------------------------ bf16 chunkwise (2e-2)
+def _chunk_case(B, H, L, dk, dv, C, gam=None, with_state=False, seed=0, ws="auto"):
+    q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed)
+    gam = inputs.multiscale_gammas(H) if gam is None else torch.tensor(gam, dtype=torch.float32)
+    s_in = inputs.state(B, H, dk, dv, seed=seed + 7, scale=0.5) if with_state else None
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam, s_in)
+    qd, kd, vd, sd = dev(q, k, v, s_in)
+    kw = {} if ws == "auto" else {"workspace": ws}
+    y, s = ret.chunkwise(qd, kd, vd, gam, C, state_in=sd, **kw)
+    return rel(y, y_ref), rel(s, s_ref)
+
+
+def test_msr_core_chunkwise():
+    w = inputs.WORKLOADS["msr_core_bf16"]
+    ey, es = _chunk_case(w.B, w.H, w.L, w.dk, w.dv, w.chunk)
+    assert ey <= 2e-2 and es <= 2e-2, (ey, es)
+
+
+@pytest.mark.parametrize("B,H,L,dk,dv,C", [
+    (1, 2, 200, 64, 128, 64),      # ragged tail
+    (1, 1, 50, 64, 128, 64),       # L < C
+    (1, 1, 1, 64, 128, 16),        # single token
+    (2, 2, 300, 128, 256, 128),    # dk 128, two dv slices
+    (1, 2, 260, 256, 128, 128),    # dk 256 (single P buffer)
+    (1, 1, 333, 64, 128, 48),      # C % 32 == 16
+    (1, 1, 160, 128, 128, 16),     # smallest block
+    (1, 2, 520, 256, 256, 32),
+])
+def test_chunkwise_shapes(B, H, L, dk, dv, C):
+    ey, es = _chunk_case(B, H, L, dk, dv, C, with_state=True, seed=L)
+    assert ey <= 2e-2 and es <= 2e-2, (ey, es)
+
+
+def test_chunkwise_special_gammas():
+    # gamma = 0 keeps only the diagonal; gamma = 1 is un-normalised linear attention
+    ey, es = _chunk_case(1, 3, 257, 64, 128, 64, gam=[0.0, 1.0, 0.5], with_state=True, seed=11)
+    assert ey <= 2e-2 and es <= 2e-2, (ey, es)
+
+
+def test_chunkwise_sequence_split_matches_single_pass():
+    B, H, L, dk, dv, C = 1, 2, 4096, 64, 128, 64
+    assert ret.workspace_bytes(C, B, H, L, dk, dv) > 0
+    ey, es = _chunk_case(B, H, L, dk, dv, C, with_state=True, seed=5)
+    assert ey <= 2e-2 and es <= 2e-2, (ey, es)
+    ey0, es0 = _chunk_case(B, H, L, dk, dv, C, with_state=True, seed=5, ws=None)
+    assert ey0 <= 2e-2 and es0 <= 2e-2, (ey0, es0)
+
+
+def test_chunkwise_state_in_place_and_split_calls():
+    B, H, L, dk, dv, C = 1, 4, 1024, 128, 256, 128
+    q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, 21)
+    gam = inputs.multiscale_gammas(H)
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam)
+    qd, kd, vd = dev(q, k, v)
+    state = torch.zeros(B, H, dk, dv, device="cuda")
+    ys = []
+    for c0 in (0, 256, 640):  # uneven calls, state carried in place
+        c1 = {0: 256, 256: 640, 640: L}[c0]
+        y, _ = ret.chunkwise(qd[:, :, c0:c1].contiguous(), kd[:, :, c0:c1].contiguous(),
+                             vd[:, :, c0:c1].contiguous(), gam, C, state_in=state, state_out=state)
+        ys.append(y)
+    assert rel(torch.cat(ys, dim=2), y_ref) <= 2e-2 and rel(state, s_ref) <= 2e-2
+
+
+def test_chunkwise_empty_sequence_passes_state():
+    s_in = inputs.state(1, 2, 64, 128, seed=1).cuda()
+    e = torch.empty(1, 2, 0, 64, dtype=torch.bfloat16, device="cuda")
+    ev = torch.empty(1, 2, 0, 128, dtype=torch.bfloat16, device="cuda")
+    _, s = ret.chunkwise(e, e, ev, [0.5, 0.9], 64, state_in=s_in)
+    assert torch.equal(s, s_in)
+
+
+# ------------------------------------------------------- bf16 parallel (2e-2)
+@pytest.mark.parametrize("B,H,L,dk,dv", [(2, 8, 2048, 64, 128), (1, 2, 1000, 128, 256),
+                                         (1, 1, 300, 256, 128), (1, 3, 77, 64, 128)])
+def test_parallel(B, H, L, dk, dv):
+    q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed=L)
+    gam = inputs.multiscale_gammas(H) if H != 3 else torch.tensor([0.0, 1.0, 0.7])
+    y_ref, _ = oracle.recurrent(q, k, v, gam)
+    qd, kd, vd = dev(q, k, v)
+    assert rel(ret.parallel(qd, kd, vd, gam), y_ref) <= 2e-2
+
+
+def test_parallel_and_chunkwise_agree_msr_core():
+    w = inputs.WORKLOADS["msr_core_bf16"]
+    q, k, v = dev(*inputs.qkv(w.B, w.H, w.L, w.dk, w.dv, w.dtype, w.seed))
+    gam = w.gammas()
+    yp = ret.parallel(q, k, v, gam).double()
+    yc, _ = ret.chunkwise(q, k, v, gam, w.chunk)
+    assert (yp - yc.double()).abs().max().item() / yp.abs().max().item() <= 2e-2
+
+
+# --------------------------------------------------------- decode (2e-2)
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32])
+def test_recurrent_steps(dt):
+    B, H, dk, dv, steps = 2, 4, 256, 512, 12
+    qs, ks, vs = inputs.decode_tokens(steps, B, H, dk, dv, dt, seed=1)
+    s0 = inputs.state(B, H, dk, dv, seed=9, scale=0.2)
+    gam = inputs.multiscale_gammas(H)
+    q = torch.cat(list(qs), dim=2)
+    k = torch.cat(list(ks), dim=2)
+    v = torch.cat(list(vs), dim=2)
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam, s0)
+    state = s0.cuda()
+    ys = [ret.recurrent_step(qs[n].cuda(), ks[n].cuda(), vs[n].cuda(), gam, state) for n in range(steps)]
+    tol = TOL[dt]
+    assert rel(torch.cat(ys, dim=2), y_ref) <= tol and rel(state, s_ref) <= tol
+
+
+def test_recurrent_step_odd_dv():
+    B, H, dk, dv = 1, 2, 20, 30
+    q, k, v = inputs.qkv(B, H, 1, dk, dv, torch.float32, seed=2)
+    s0 = inputs.state(B, H, dk, dv, seed=3)
+    gam = torch.tensor([0.25, 1.0])
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam, s0)
+    state = s0.cuda()
+    y = ret.recurrent_step(*dev(q, k, v), gam, state)
+    assert rel(y, y_ref) <= 1e-4 and rel(state, s_ref) <= 1e-4
