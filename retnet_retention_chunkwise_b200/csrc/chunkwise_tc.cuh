@@ -46,8 +46,14 @@
 
 namespace ret {
 
-constexpr int kCW_Threads = 192;
-constexpr int kCW_DVT = 128;       // dv columns per CTA
+constexpr int kCW_Threads = 192;      // helper kernels: 4 epilogue warps, TMA warp, MMA warp
+constexpr int kCW_DVT = 128;          // dv columns per CTA
+// Main chunkwise kernel warp roles (448 threads).
+constexpr int kWarpSBase = 4;         // warps 4-7: state group
+constexpr int kWarpZBase = 8;         // warps 8-11: (zeta V)^T builder
+constexpr int kWarpProducer = 12;     // TMA producer
+constexpr int kWarpMma = 13;          // TMEM allocator + MMA issuer
+constexpr int kCW_MainThreads = 14 * 32;
 constexpr int kCW_MaxStages = 4;
 constexpr uint32_t kSmemAlign = 1024;
 constexpr uint32_t kMiscBytes = 1024;
@@ -133,7 +139,7 @@ __device__ __forceinline__ void store_row32_sw128(uint8_t* tile, uint32_t box_by
 }
 
 template <int DK>
-__global__ void __launch_bounds__(kCW_Threads, 1)
+__global__ void __launch_bounds__(kCW_MainThreads, 1)
 chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                     const __grid_constant__ CUtensorMap mapV, const CwArgs a,
                     const __grid_constant__ CwDecay dec) {
@@ -151,57 +157,75 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   uint8_t* sV = base + sp.v;
   uint8_t* sSb = base + sp.sb;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + sp.misc);
-  uint64_t* full = bars;             // [4] TMA -> consumers
-  uint64_t* empty = bars + 4;        // [4] MMA5 done -> producer
-  uint64_t* pfull = bars + 8;        // [2] MMA1 done -> epilogue
-  uint64_t* pfree = bars + 10;       // [2] MMA3 done (P~ consumed) -> MMA1 of a later block
-  uint64_t* ocross = bars + 12;      // MMA4 done -> epilogue
-  uint64_t* e1done = bars + 13;      // epilogue (P~, zeta K, xi O ready) -> MMA3/MMA5
-  uint64_t* e2done = bars + 14;      // epilogue (Sb, rescaled S, O drained) -> MMA4 of next block
-  uint64_t* mma35 = bars + 15;       // MMA3+MMA5 done -> epilogue
-  uint64_t* fin = bars + 16;         // teardown drain of the MMA pipe
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17) + 1;
-  float* pw = reinterpret_cast<float*>(bars + 18);  // gamma^0..gamma^128
+  uint64_t* fullQ = bars;          // [4] TMA -> MMA
+  uint64_t* fullK = bars + 4;      // [4] TMA -> MMA
+  uint64_t* fullV = bars + 8;      // [4] TMA -> V group, MMA
+  uint64_t* emptyQ = bars + 12;    // [4] MMA4 done -> producer
+  uint64_t* emptyK = bars + 16;    // [4] MMA5 done -> producer
+  uint64_t* emptyV = bars + 20;    // [4] MMA3 done -> producer
+  uint64_t* zready = bars + 24;    // [4] V group: scaled V of stage s written -> MMA5 (and MMA3)
+  uint64_t* pfull = bars + 28;     // [2] MMA1 done -> P/O group
+  uint64_t* pfree = bars + 30;     // [2] MMA3 done -> MMA1 of block it+NP
+  uint64_t* ocross = bars + 32;    // MMA5 + MMA4 done -> P/O group, S group
+  uint64_t* pready = bars + 33;    // P/O group: P~ (and xi O) written -> MMA3
+  uint64_t* sready = bars + 35;    // S group: state copy + rescaled state written -> MMA5, MMA4
+  uint64_t* mma3done = bars + 36;  // MMA3 done -> P/O group (y)
+  uint64_t* ofree = bars + 37;     // P/O group: O read out -> V group, MMA4 of the next block
+  uint64_t* fin = bars + 38;       // teardown drain of the MMA pipe
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 39);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 39) + 1;
+  float* pw = reinterpret_cast<float*>(bars + 40);  // gamma^0 .. gamma^128
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int vt = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;
   const float l2g = dec.l2g[bh % a.H];
+  // Rescaled form (see the file header) when gamma^(C-1) >= 2^-64; else the
+  // direct form.  Uniform over the CTA (one head).
+  const bool rescaled = (float)(C - 1) * l2g >= -64.f;
   const int n_total = (a.L + C - 1) / C;
   const int c_begin = seg * a.seg_chunks;
   const int c_end = min(c_begin + a.seg_chunks, n_total);
   const int nck = max(c_end - c_begin, 0);
+  const int cta_id = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  (void)cta_id;
+  RET_TRACE_INIT();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&fullQ[i], 1);
+      mbar_init(&fullK[i], 1);
+      mbar_init(&fullV[i], 1);
+      mbar_init(&emptyQ[i], 1);
+      mbar_init(&emptyK[i], 1);
+      mbar_init(&emptyV[i], 1);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&zready[i], 128);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&pfull[i], 1);
       mbar_init(&pfree[i], 1);
     }
     mbar_init(ocross, 1);
-    mbar_init(e1done, 128);
-    mbar_init(e2done, 128);
-    mbar_init(mma35, 1);
+    mbar_init(pready, 128);
+    mbar_init(sready, 128);
+    mbar_init(mma3done, 1);
+    mbar_init(ofree, 128);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  for (int n = threadIdx.x; n <= 128; n += kCW_Threads) pw[n] = n == 0 ? 1.f : exp2f((float)n * l2g);
+  for (int n = threadIdx.x; n <= 128; n += kCW_MainThreads) pw[n] = n == 0 ? 1.f : exp2f((float)n * l2g);
   if (C < 128) {  // rows C..127 of every Q box are read by the M = 128 MMA: keep them zero
-    const uint32_t rows_bytes = (128u - (uint32_t)C) * 128u;
-    const uint32_t per_stage = (uint32_t)(DK / 64) * rows_bytes / 16u;
-    for (uint32_t e = threadIdx.x; e < (uint32_t)NS * per_stage; e += kCW_Threads) {
+    const uint32_t rows16 = (128u - (uint32_t)C) * 8u;  // 16-byte pieces per box
+    const uint32_t per_stage = (uint32_t)(DK / 64) * rows16;
+    for (uint32_t e = threadIdx.x; e < (uint32_t)NS * per_stage; e += kCW_MainThreads) {
       const uint32_t s = e / per_stage, rem = e % per_stage;
-      const uint32_t b = rem / (rows_bytes / 16u), o = rem % (rows_bytes / 16u);
+      const uint32_t b = rem / rows16, o = rem % rows16;
       *reinterpret_cast<uint4*>(sQ + s * sp.q_stage + b * 16384u + (uint32_t)C * 128u + o * 16u) =
           make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -210,42 +234,79 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
+    // Q, K, V of each block go to their own stage buffers with their own
+    // barriers, so each is reloaded as soon as its last reader is done:
+    // K after MMA5, Q after MMA4, V after MMA3 (the order they are issued in).
+    // The next block's tiles are prefetched into L2 as soon as this block's
+    // loads are issued, so a reload waits on L2 rather than on DRAM.
     if (lane == 0 && nck > 0) {
       tma_prefetch_desc(&mapQ);
       tma_prefetch_desc(&mapK);
       tma_prefetch_desc(&mapV);
-      const uint32_t bytes = (uint32_t)(2 * DK + kCW_DVT) * (uint32_t)C * 2u;
+      const uint32_t qk_bytes = (uint32_t)DK * (uint32_t)C * 2u;
+      const uint32_t v_bytes = (uint32_t)kCW_DVT * (uint32_t)C * 2u;
+      for (int it = 0; it < min(NS, nck); ++it) {
+        const int t0 = (c_begin + it) * C;
+        for (int b = 0; b < DK / 64; ++b) {
+          tma_prefetch_l2_3d(&mapK, b * 64, t0, bh);
+          tma_prefetch_l2_3d(&mapQ, b * 64, t0, bh);
+        }
+        for (int b = 0; b < 2; ++b) tma_prefetch_l2_3d(&mapV, vt * kCW_DVT + b * 64, t0, bh);
+      }
       int issued = 0;
       for (int it = 0; it < nck; ++it) {
         const int s = it % NS;
-        if (it >= NS && !mbar_wait(&empty[s], ((it / NS) - 1) & 1, abort_flag, a.lim)) break;
+        const uint32_t par = ((it / NS) - 1) & 1;
         const int t0 = (c_begin + it) * C;
-        mbar_arrive_expect_tx(&full[s], bytes);
+        if (it >= NS && !mbar_wait(&emptyK[s], par, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, it, 0);
+        mbar_arrive_expect_tx(&fullK[s], qk_bytes);
         for (int b = 0; b < DK / 64; ++b)
-          tma_load_3d(sQ + s * sp.q_stage + b * 16384, &mapQ, &full[s], b * 64, t0, bh);
+          tma_load_3d(sK + s * sp.k_stage + b * C * 128, &mapK, &fullK[s], b * 64, t0, bh);
+        if (it >= NS && !mbar_wait(&emptyQ[s], par, abort_flag, a.lim)) break;
+        mbar_arrive_expect_tx(&fullQ[s], qk_bytes);
         for (int b = 0; b < DK / 64; ++b)
-          tma_load_3d(sK + s * sp.k_stage + b * C * 128, &mapK, &full[s], b * 64, t0, bh);
+          tma_load_3d(sQ + s * sp.q_stage + b * 16384, &mapQ, &fullQ[s], b * 64, t0, bh);
+        if (it >= NS && !mbar_wait(&emptyV[s], par, abort_flag, a.lim)) break;
+        mbar_arrive_expect_tx(&fullV[s], v_bytes);
         for (int b = 0; b < 2; ++b)
-          tma_load_3d(sV + s * sp.v_stage + b * C * 128, &mapV, &full[s], vt * kCW_DVT + b * 64, t0, bh);
+          tma_load_3d(sV + s * sp.v_stage + b * C * 128, &mapV, &fullV[s], vt * kCW_DVT + b * 64, t0, bh);
         issued = it + 1;
+        if (it + NS < nck) {
+          const int tp = t0 + NS * C;
+          for (int b = 0; b < DK / 64; ++b) {
+            tma_prefetch_l2_3d(&mapK, b * 64, tp, bh);
+            tma_prefetch_l2_3d(&mapQ, b * 64, tp, bh);
+          }
+          for (int b = 0; b < 2; ++b) tma_prefetch_l2_3d(&mapV, vt * kCW_DVT + b * 64, tp, bh);
+        }
       }
       // every load issued must land before the CTA may exit
-      for (int it = max(0, issued - NS); it < issued; ++it) mbar_drain(&full[it % NS], (it / NS) & 1, a.lim);
+      for (int it = max(0, issued - NS); it < issued; ++it) {
+        mbar_drain(&fullQ[it % NS], (it / NS) & 1, a.lim);
+        mbar_drain(&fullK[it % NS], (it / NS) & 1, a.lim);
+        mbar_drain(&fullV[it % NS], (it / NS) & 1, a.lim);
+      }
     }
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ---------------------------------------------------------- MMA issuer
+    // Order per block: MMA1 (P = Q K^T), MMA5 (state update; frees K), MMA4
+    // (Q S; frees Q), MMA3 (P~ V; frees V and P).
     if (lane == 0 && nck > 0) {
       const uint32_t id1 = idesc_bf16(128, C, false, false);
       const uint32_t id4 = idesc_bf16(128, kCW_DVT, false, false);
       const uint32_t id3 = idesc_bf16(128, kCW_DVT, false, true);
-      const uint32_t id5 = idesc_bf16(128, DK, true, true);
+      const uint32_t id5 = idesc_bf16(128, DK, rescaled, true);  // A = V^T (smem, MN-major) or TMEM
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aSb = smem_u32(sSb);
       for (int it = 0; it < nck; ++it) {
         const int s = it % NS, pb = it % NP;
-        if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) break;
+        const uint32_t par = (it / NS) & 1;
+        if (!mbar_wait(&fullK[s], par, abort_flag, a.lim)) break;
+        if (!mbar_wait(&fullQ[s], par, abort_flag, a.lim)) break;
         if (it >= NP && !mbar_wait(&pfree[pb], ((it / NP) - 1) & 1, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, it, 1);
         tc_fence_after();
         const uint32_t q_s = aQ + s * sp.q_stage, k_s = aK + s * sp.k_stage, v_s = aV + s * sp.v_stage;
         // MMA1: P = Q K^T
@@ -256,8 +317,28 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           mma_ss(tm + TM_P + pb * 128, ad, bd, id1, kk > 0);
         }
         mma_commit(&pfull[pb]);
-        // MMA4: O = Q S_prev (bf16 copy of the state, written by the epilogue)
-        if (!mbar_wait(e2done, it & 1, abort_flag, a.lim)) break;
+        // MMA5: S^T += (zeta V)^T K, onto the state already rescaled by gamma^l.
+        // Rescaled form: zeta V is the V tile itself (scaled in place), read
+        // MN-major from shared memory.  Direct form: (zeta V)^T was built in the
+        // (free) O columns of TMEM.
+        // zready is per stage: in the rescaled form the V group runs ahead by up
+        // to NS blocks, so one barrier could complete two phases unobserved.
+        if (!mbar_wait(&zready[s], par, abort_flag, a.lim)) break;
+        if (!mbar_wait(sready, it & 1, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, it, 2);
+        tc_fence_after();
+        for (int kk = 0; kk < C / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(k_s + kk * 2048, C * 128, 1024);
+          if (rescaled)
+            mma_ss(tm + TM_S, sdesc_sw128(v_s + kk * 2048, C * 128, 1024), bd, id5, 1);
+          else
+            mma_ts(tm + TM_S, tm + TM_O + kk * 8, bd, id5, 1);
+        }
+        mma_commit(&emptyK[s]);
+        // MMA4: O = Q S_copy, once the previous block's O was drained.  It
+        // overwrites the O columns after MMA5 has read them (MMAs issued by one
+        // thread run in order).
+        if (!mbar_wait(ofree, it & 1, abort_flag, a.lim)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
@@ -266,89 +347,211 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           mma_ss(tm + TM_O, ad, bd, id4, kk > 0);
         }
         mma_commit(ocross);
-        // MMA3: O += P~ V ; MMA5: S^T += V^T (zeta K)
-        if (!mbar_wait(e1done, it & 1, abort_flag, a.lim)) break;
+        mma_commit(&emptyQ[s]);
+        // MMA3: O += P~ V
+        if (!mbar_wait(pready, it & 1, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, it, 4);
         tc_fence_after();
         for (int kk = 0; kk < C / 16; ++kk) {
           const uint64_t bd = sdesc_sw128(v_s + kk * 2048, C * 128, 1024);
           mma_ts(tm + TM_O, tm + TM_P + pb * 128 + kk * 8, bd, id3, 1);
         }
         mma_commit(&pfree[pb]);
-        for (int kk = 0; kk < C / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(v_s + kk * 2048, C * 128, 1024);
-          const uint64_t bd = sdesc_sw128(k_s + kk * 2048, C * 128, 1024);
-          mma_ss(tm + TM_S, ad, bd, id5, 1);
-        }
-        mma_commit(mma35);
-        mma_commit(&empty[s]);
+        mma_commit(mma3done);
+        mma_commit(&emptyV[s]);
       }
       mma_commit(fin);
       mbar_drain(fin, 0, a.lim);
     }
-  } else {
-    // ----------------------------------------------------------- epilogue
-    const uint32_t r = threadIdx.x;                 // TMEM lane == row of P / O, column of S
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const int v = vt * kCW_DVT + (int)r;            // this thread's dv column
+  } else if (warp >= kWarpZBase) {
+    // ---------------------------------------------------- V group (4 warps)
+    const uint32_t t = threadIdx.x - kWarpZBase * 32;
+    for (int it = 0; it < nck; ++it) {
+      const int s = it % NS;
+      if (!mbar_wait(&fullV[s], (it / NS) & 1, abort_flag, a.lim)) break;
+      // Direct form: (zeta V)^T goes into the O columns, free once the previous
+      // block's O was drained.
+      if (!rescaled && !mbar_wait(ofree, it & 1, abort_flag, a.lim)) break;
+      tc_fence_after();
+      const int l = min(C, a.L - (c_begin + it) * C);
+      uint8_t* vs = sV + s * sp.v_stage;
+      if (rescaled) {
+        // row j of the V tile scaled in place by zeta_j = gamma^(l-1-j) (0 past the end)
+        if ((int)t < C) {
+          const float zeta = ((int)t < l) ? pw[l - 1 - (int)t] : 0.f;
+          scale_row_sw128(vs, t, zeta);
+          scale_row_sw128(vs + C * 128, t, zeta);
+        }
+        fence_proxy_async_smem();
+      } else {
+        // (zeta V)^T into the O columns: lane v holds column v of V scaled
+        // row-wise by zeta_j, two rows per 32-bit column.  V is read from its
+        // swizzled tile as 32-bit pairs (v0, v0+1) of rows j and j+1 and
+        // re-paired by a byte permute.
+        const uint32_t lane_off = (uint32_t)((warp - kWarpZBase) * 32) << 16;
+        const uint32_t vb = t / 64, vv = t % 64;
+        const uint32_t vchunk = vv / 8;                // 16-byte chunk of the row
+        const uint32_t vbyte = ((vv % 8) & ~1u) * 2u;  // byte of the pair (v0, v0+1): 0, 4, 8, 12
+        const uint32_t sel = (t & 1) ? 0x7632u : 0x5410u;
+        const uint8_t* vt_s = vs + vb * C * 128;
+        for (int j0 = 0; j0 < C; j0 += 32) {
+          uint32_t w[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const uint32_t j = (uint32_t)j0 + 2u * u;
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vt_s + j * 128 + ((vchunk ^ (j & 7)) << 4) + vbyte);
+            const uint32_t w1 =
+                *reinterpret_cast<const uint32_t*>(vt_s + (j + 1) * 128 + ((vchunk ^ ((j + 1) & 7)) << 4) + vbyte);
+            const uint32_t pr = __byte_perm(w0, w1, sel);
+            const float z0 = ((int)j < l) ? pw[l - 1 - (int)j] : 0.f;
+            const float z1 = ((int)j + 1 < l) ? pw[l - 2 - (int)j] : 0.f;
+            w[u] = pack_bf16x2(bf16lo_to_f32(pr) * z0, bf16hi_to_f32(pr) * z1);
+          }
+          // When C % 32 == 16 the last piece covers 16 rows past C (zeta = 0
+          // there, read from the next, allocated, part of shared memory); the
+          // results land in columns MMA5 never reads.
+          tmem_st16(tm + lane_off + TM_O + j0 / 2, w);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+      }
+      mbar_arrive(&zready[s]);
+      if (t == 0) RET_TRACE_STAMP(cta_id, it, 3);
+    }
+  } else if (warp >= kWarpSBase) {
+    // ---------------------------------------------------- S group (4 warps)
+    // TMEM lane v = this thread's dv column of the state S^T.  Keeps the fp32
+    // state, its bf16 copy Sb for MMA4 and the gamma^l rescale for MMA5.  In the
+    // rescaled form the copy is of the rescaled state.
+    const uint32_t v_loc = threadIdx.x - kWarpSBase * 32;
+    const uint32_t lane_off = (uint32_t)((warp - kWarpSBase) * 32) << 16;
+    const int v = vt * kCW_DVT + (int)v_loc;
     const size_t dkdv = (size_t)DK * a.dv;
-    // initial state: S_prev (bf16 copy for MMA4) and gamma^l0 S_prev (accumulator for MMA5)
     {
       const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
                                        : (a.state_in ? a.state_in + (size_t)bh * dkdv : nullptr);
       const int l0 = min(C, a.L - c_begin * C);
       const float g0 = pw[max(l0, 0)];
+      const float gc = rescaled ? g0 : 1.f;
       for (int d0 = 0; d0 < DK; d0 += 32) {
         float x[32];
         uint32_t w[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          x[u] = src ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
-          w[u] = __float_as_uint(g0 * x[u]);
+          const float sv = src ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
+          x[u] = gc * sv;
+          w[u] = __float_as_uint(g0 * sv);
         }
-        store_row32_sw128(sSb, 16384, r, d0, x);
+        store_row32_sw128(sSb, 16384, v_loc, d0, x);
         tmem_st32(tm + lane_off + TM_S + d0, w);
       }
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(e2done);
+      mbar_arrive(sready);
     }
     for (int it = 0; it < nck; ++it) {
-      const int s = it % NS, pb = it % NP;
+      // MMA5 (state update) and MMA4 (last reader of Sb) are both done
+      if (!mbar_wait(ocross, it & 1, abort_flag, a.lim)) break;
+      if (v_loc == 0) RET_TRACE_STAMP(cta_id, it, 10);
+      tc_fence_after();
+      const int t0 = (c_begin + it) * C;
+      if (it < nck - 1) {
+        const float gn = pw[min(C, a.L - t0 - C)];
+        for (int d0 = 0; d0 < DK; d0 += 32) {
+          uint32_t sr[32];
+          tmem_ld32(tm + lane_off + TM_S + d0, sr);
+          tmem_ld_wait();
+          float x[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const float sv = __uint_as_float(sr[u]);
+            const float sg = gn * sv;
+            x[u] = rescaled ? sg : sv;
+            sr[u] = __float_as_uint(sg);
+          }
+          store_row32_sw128(sSb, 16384, v_loc, d0, x);
+          tmem_st32(tm + lane_off + TM_S + d0, sr);
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(sready);
+        if (v_loc == 0) RET_TRACE_STAMP(cta_id, it, 8);
+      } else if (a.state_out && seg == a.n_seg - 1) {
+        float* so = a.state_out + (size_t)bh * dkdv;
+        for (int d0 = 0; d0 < DK; d0 += 32) {
+          uint32_t sr[32];
+          tmem_ld32(tm + lane_off + TM_S + d0, sr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) so[(size_t)(d0 + u) * a.dv + v] = __uint_as_float(sr[u]);
+        }
+      }
+    }
+  } else {
+    // -------------------------------------------------- P/O group (4 warps)
+    // TMEM lane r = row r of P and O (token t0 + r of the block).
+    const int r = (int)threadIdx.x;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int row_lo = warp * 32;  // rows of this warp: [row_lo, row_lo + 32)
+    mbar_arrive(ofree);            // O starts free
+    for (int it = 0; it < nck; ++it) {
+      const int pb = it % NP;
       const int t0 = (c_begin + it) * C;
       const int l = min(C, a.L - t0);
       if (!mbar_wait(&pfull[pb], (it / NP) & 1, abort_flag, a.lim)) break;
-      if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) break;
       tc_fence_after();
-      // E1a: P -> P~ = bf16(P * gamma^(r-j)) for j <= r < l, else 0 (in place, two per column)
+      // P -> P~ in place (two bf16 per column).  Rows past the block end read
+      // zero Q rows and columns past it zero K rows, so P is already 0 there.
+      // Rescaled form: P~ = P on and below the diagonal (decay lives in zeta V
+      // and the row factor applied at the end).  Direct form: P~ = P gamma^(r-j).
       const uint32_t tp = tm + lane_off + TM_P + pb * 128;
       for (int j0 = 0; j0 < C; j0 += 32) {
         uint32_t pr[32];
         tmem_ld32(tp + j0, pr);
         tmem_ld_wait();
         uint32_t w[16];
+        if (j0 >= row_lo + 32) {
 #pragma unroll
-        for (int u = 0; u < 32; u += 2) {
-          const int j = j0 + u;
-          const float f0 = (j <= (int)r && (int)r < l) ? pw[r - j] : 0.f;
-          const float f1 = (j + 1 <= (int)r && (int)r < l) ? pw[r - j - 1] : 0.f;
-          w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * f0, __uint_as_float(pr[u + 1]) * f1);
+          for (int u = 0; u < 16; ++u) w[u] = 0u;
+        } else if (rescaled) {
+          if (j0 + 31 <= row_lo) {
+#pragma unroll
+            for (int u = 0; u < 32; u += 2) w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]), __uint_as_float(pr[u + 1]));
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; u += 2) {
+              const int j = j0 + u;
+              w[u / 2] = pack_bf16x2((j <= r) ? __uint_as_float(pr[u]) : 0.f,
+                                     (j + 1 <= r) ? __uint_as_float(pr[u + 1]) : 0.f);
+            }
+          }
+        } else if (j0 + 31 <= row_lo) {
+          // whole 32x32 block below the diagonal: gamma^(r-j) = gamma^(r-j0-31) * gamma^(31-u)
+          const float ar = pw[r - j0 - 31];
+#pragma unroll
+          for (int u = 0; u < 32; u += 2)
+            w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * ar * pw[31 - u],
+                                   __uint_as_float(pr[u + 1]) * ar * pw[30 - u]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; u += 2) {
+            const int j = j0 + u;
+            const float f0 = (j <= r) ? pw[r - j] : 0.f;
+            const float f1 = (j + 1 <= r) ? pw[r - j - 1] : 0.f;
+            w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * f0, __uint_as_float(pr[u + 1]) * f1);
+          }
         }
         // When C % 32 == 16 the last piece also covers 16 columns past C; their
         // packed results land at columns >= C/2, which MMA3 never reads.
         tmem_st16(tp + j0 / 2, w);
       }
-      // E1b: row j of K scaled by zeta_j = gamma^(l-1-j) (0 past the block end)
-      if ((int)r < C) {
-        const float zeta = ((int)r < l) ? pw[l - 1 - (int)r] : 0.f;
-        uint8_t* ks = sK + s * sp.k_stage;
-        for (int b = 0; b < DK / 64; ++b) scale_row_sw128(ks + b * C * 128, r, zeta);
-      }
-      fence_proxy_async_smem();
-      // E1c: O *= xi_r = gamma^(r+1)
-      if (!mbar_wait(ocross, it & 1, abort_flag, a.lim)) break;
-      tc_fence_after();
-      {
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 5);
+      if (!rescaled) {
+        // O *= xi_r = gamma^(r+1) once MMA4 wrote Q S_prev into O
+        if (!mbar_wait(ocross, it & 1, abort_flag, a.lim)) break;
+        tc_fence_after();
         const float xi = pw[r + 1];
         for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
           uint32_t o[32];
@@ -361,65 +564,41 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(e1done);
-      // E2: state -> bf16 copy + rescale (or state_out); O -> y
-      if (!mbar_wait(mma35, it & 1, abort_flag, a.lim)) break;
+      mbar_arrive(pready);
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 6);
+      // O -> y once MMA3 added P~ V.  Rescaled form: y_r = gamma^(r+1-l) O_r.
+      // O is read into registers (as bf16) and released before the global
+      // stores, so the next block's MMA4 need not wait for them.
+      if (!mbar_wait(mma3done, it & 1, abort_flag, a.lim)) break;
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 9);
       tc_fence_after();
-      const bool last = (it == nck - 1);
-      if (!last) {
-        const float gn = pw[min(C, a.L - t0 - C)];
-        for (int d0 = 0; d0 < DK; d0 += 32) {
-          uint32_t sr[32];
-          tmem_ld32(tm + lane_off + TM_S + d0, sr);
-          tmem_ld_wait();
-          float x[32];
-#pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            x[u] = __uint_as_float(sr[u]);
-            sr[u] = __float_as_uint(gn * x[u]);
-          }
-          store_row32_sw128(sSb, 16384, r, d0, x);
-          tmem_st32(tm + lane_off + TM_S + d0, sr);
-        }
-      } else if (a.state_out && seg == a.n_seg - 1) {
-        float* so = a.state_out + (size_t)bh * dkdv;
-        for (int d0 = 0; d0 < DK; d0 += 32) {
-          uint32_t sr[32];
-          tmem_ld32(tm + lane_off + TM_S + d0, sr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int u = 0; u < 32; ++u) so[(size_t)(d0 + u) * a.dv + v] = __uint_as_float(sr[u]);
-        }
-      }
       {
-        __nv_bfloat16* yrow = a.y + ((size_t)bh * a.L + t0 + r) * a.dv + vt * kCW_DVT;
+        const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) : 1.f;
+        uint32_t yw[kCW_DVT / 2];
+#pragma unroll
         for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(tm + lane_off + TM_O + c0, o);
           tmem_ld_wait();
-          if ((int)r < l) {
-            uint4* dst = reinterpret_cast<uint4*>(yrow + c0);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(o[8 * q4 + 0]), __uint_as_float(o[8 * q4 + 1]));
-              w.y = pack_bf16x2(__uint_as_float(o[8 * q4 + 2]), __uint_as_float(o[8 * q4 + 3]));
-              w.z = pack_bf16x2(__uint_as_float(o[8 * q4 + 4]), __uint_as_float(o[8 * q4 + 5]));
-              w.w = pack_bf16x2(__uint_as_float(o[8 * q4 + 6]), __uint_as_float(o[8 * q4 + 7]));
-              dst[q4] = w;
-            }
-          }
+          for (int u = 0; u < 16; ++u)
+            yw[c0 / 2 + u] = pack_bf16x2(yf * __uint_as_float(o[2 * u]), yf * __uint_as_float(o[2 * u + 1]));
+        }
+        tc_fence_before();
+        mbar_arrive(ofree);
+        if (r < l) {
+          uint4* dst = reinterpret_cast<uint4*>(a.y + ((size_t)bh * a.L + t0 + r) * a.dv + vt * kCW_DVT);
+#pragma unroll
+          for (int q4 = 0; q4 < kCW_DVT / 8; ++q4)
+            dst[q4] = make_uint4(yw[4 * q4], yw[4 * q4 + 1], yw[4 * q4 + 2], yw[4 * q4 + 3]);
         }
       }
-      tmem_st_wait();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(e2done);
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 7);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tm, kTmemCols);

@@ -26,7 +26,7 @@ using namespace ret;
 // Wall-clock budget of any single wait inside a kernel.  A healthy wait is
 // microseconds; this only bounds a kernel whose pipeline broke.
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
-constexpr uint32_t kWaitIter = 1u << 30;
+constexpr uint32_t kWaitIter = 1u << 24;      // polls (each parks for at most 100 us)
 
 WaitLimit wait_limit() {
   WaitLimit w{kWaitNs, kWaitIter};
@@ -219,7 +219,7 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
                            (int)plan.total) != cudaSuccess)
     return RET_ECUDA;
   dim3 grid(s.dv / kCW_DVT, BH, n_seg);
-  chunkwise_tc_kernel<DK><<<grid, kCW_Threads, plan.total, st>>>(mq, mk, mv, a, dec);
+  chunkwise_tc_kernel<DK><<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, a, dec);
   return launch_status();
 }
 
@@ -261,6 +261,18 @@ ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const
 }  // namespace
 
 extern "C" {
+
+#ifdef RET_TRACE
+// Trace builds only: route RET_TRACE_STAMP events to `buf` (device memory of
+// n_ctas * blocks * events u64), or switch tracing off with buf = NULL.
+RET_API int retention_debug_trace(void* buf, int blocks, int events) {
+  unsigned long long* p = static_cast<unsigned long long*>(buf);
+  if (cudaMemcpyToSymbol(g_trace_buf, &p, sizeof(p)) != cudaSuccess) return 1;
+  if (cudaMemcpyToSymbol(g_trace_blocks, &blocks, sizeof(int)) != cudaSuccess) return 1;
+  if (cudaMemcpyToSymbol(g_trace_events, &events, sizeof(int)) != cudaSuccess) return 1;
+  return 0;
+}
+#endif
 
 int retention_abi_version(void) { return 100; }
 

@@ -24,6 +24,35 @@ namespace ret {
 // this is the single definition.
 __device__ int g_device_status = 0;
 
+// Optional event trace (builds with -DRET_TRACE only): %globaltimer stamps per
+// (CTA, block, event) written to a caller-provided buffer.  RET_TRACE_INIT reads
+// the buffer description once into registers; the stamps are plain stores.
+// Both compile to nothing in the normal build.
+#ifdef RET_TRACE
+__device__ unsigned long long* g_trace_buf = nullptr;
+__device__ int g_trace_events = 0;   // events per (CTA, block)
+__device__ int g_trace_blocks = 0;   // block slots per CTA
+#define RET_TRACE_INIT()                                \
+  unsigned long long* trace_buf_ = g_trace_buf;         \
+  const int trace_ev_ = g_trace_events;                 \
+  const int trace_bl_ = g_trace_blocks
+#define RET_TRACE_STAMP(cta, it, ev)                                                       \
+  do {                                                                                     \
+    if (trace_buf_ && (it) < trace_bl_ && (ev) < trace_ev_) {                              \
+      unsigned long long t_;                                                               \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                             \
+      trace_buf_[((size_t)(cta) * trace_bl_ + (it)) * trace_ev_ + (ev)] = t_;              \
+    }                                                                                      \
+  } while (0)
+#else
+#define RET_TRACE_INIT() \
+  do {                   \
+  } while (0)
+#define RET_TRACE_STAMP(cta, it, ev) \
+  do {                               \
+  } while (0)
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -51,14 +80,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                "r"(bytes)
                : "memory");
 }
+// One poll of a phase.  The suspend-time hint lets the hardware park the
+// waiting thread (up to kSuspendNs) until the phase completes, so waiting warps
+// do not take issue slots from working warps on the same sub-partition.
+constexpr uint32_t kSuspendNs = 100000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -76,10 +109,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1; it < lim.max_iter; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > lim.ns) break;
-    }
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > lim.ns) break;
   }
   *abort = 1;
   atomicExch(&g_device_status, 4);
@@ -98,6 +129,13 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+// Prefetch one tile of a 3-D tensor map into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core, TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {

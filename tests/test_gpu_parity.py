@@ -104,6 +104,14 @@ def test_chunkwise_special_gammas():
     assert ey <= 2e-2 and es <= 2e-2, (ey, es)
 
 
+@pytest.mark.parametrize("C", [128, 64])
+def test_chunkwise_small_gammas_direct_form(C):
+    # gamma^(C-1) < 2^-64 takes the direct form (decay applied to P and O);
+    # the other heads take the rescaled form.
+    ey, es = _chunk_case(1, 4, 300, 128, 128, C, gam=[0.5, 0.25, 0.6, 0.97], with_state=True, seed=13)
+    assert ey <= 2e-2 and es <= 2e-2, (ey, es)
+
+
 def test_chunkwise_sequence_split_matches_single_pass():
     B, H, L, dk, dv, C = 1, 2, 4096, 64, 128, 64
     assert ret.workspace_bytes(C, B, H, L, dk, dv) > 0
