@@ -119,6 +119,33 @@ RET_API ret_status retention_recurrent_step(const void* q, const void* k, const 
                                     const float* gamma, void* y, float* state, ret_shape s,
                                     ret_dtype dt, void* stream);
 
+/*
+ * Chunkwise form for callers that cannot allocate device memory -- for
+ * example code that must not touch the allocator while a CUDA graph is being
+ * captured, runtimes that fix every device buffer at start-up, or plugin hosts
+ * that own all device memory.  Same arguments and results as
+ * retention_chunkwise, without the workspace pair: the scratch for the
+ * sequence split comes from a fixed 16 MiB array inside this library's device
+ * memory, held on every GPU that loads the library until the process exits.  The pages have no counterpart; this
+ * is a property of the library, not of the method.
+ *   - Shapes whose split needs more scratch than the array holds
+ *     (retention_chunkwise_workspace_bytes() > 16 MiB) return
+ *     RET_EUNSUPPORTED before anything is launched; shapes that need no split
+ *     never touch the array.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call uses the same array and leaves its contents behind.  Nothing
+ *     in it has to start at zero (each call writes every slot it reads), but
+ *     calls that can run at the same time on the GPU -- different streams, or
+ *     different host threads -- race on it: serialise them.
+ *   - No cudaMalloc, cudaFree or other allocating call is made.
+ */
+RET_API ret_status retention_chunkwise_static_ws(const void* q, const void* k, const void* v,
+                                                 const float* gamma, void* y, const float* state_in,
+                                                 float* state_out, int chunk, ret_shape s,
+                                                 ret_dtype dt, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word:
  * RET_OK, RET_ETIMEOUT if a kernel's bounded wait expired since the last
  * query, or RET_ECUDA if the stream reported an error. */

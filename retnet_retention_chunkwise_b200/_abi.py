@@ -25,7 +25,9 @@ EXPORTS = (
     "retention_get_device_status",
     "retention_status_str",
     "retention_abi_version",
+    "retention_chunkwise_static_ws",
 )
+STATIC_WS_BYTES = 16 << 20  # scratch array behind retention_chunkwise_static_ws
 
 
 class RetShape(ctypes.Structure):
@@ -49,6 +51,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.retention_status_str.argtypes = [i]
     lib.retention_status_str.restype = ctypes.c_char_p
     lib.retention_abi_version.argtypes = []
+    lib.retention_chunkwise_static_ws.argtypes = [vp, vp, vp, fp, vp, vp, vp, i, RetShape, i, vp]
+    lib.retention_chunkwise_static_ws.restype = ctypes.c_int
     for name in ("retention_parallel", "retention_chunkwise", "retention_recurrent_step",
                  "retention_get_device_status", "retention_abi_version"):
         getattr(lib, name).restype = ctypes.c_int

@@ -258,6 +258,39 @@ ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const
   return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for retention_chunkwise_static_ws: a fixed array in this library's
+// device memory, for callers that cannot allocate.  Its size is the most
+// sequence-split scratch that entry point accepts.  Every GPU that loads the
+// library holds it until the process exits.
+constexpr size_t kStaticWsBytes = (size_t)16 << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
+
+// Device address of g_static_ws for the current device.  The host-side name of
+// a __device__ array is only a stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+void* static_ws_address(ret_status* rc) {
+  constexpr int kMaxDevices = 64;
+  static void* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *rc = RET_ECUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || p == nullptr) {
+      *rc = RET_ECUDA;
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  *rc = RET_OK;
+  return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -423,6 +456,26 @@ ret_status retention_chunkwise(const void* q, const void* k, const void* v, cons
     case 128: return launch_chunkwise_tc<128>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
     default: return launch_chunkwise_tc<256>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
   }
+}
+
+// Chunkwise form with the sequence-split scratch taken from g_static_ws
+// instead of a caller buffer (see the header for who needs this).
+ret_status retention_chunkwise_static_ws(const void* q, const void* k, const void* v, const float* gamma,
+                                         void* y, const float* state_in, float* state_out, int chunk,
+                                         ret_shape s, ret_dtype dt, void* stream) {
+  ret_status rc = check_shape(s, true);
+  if (rc != RET_OK) return rc;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (chunk < 1) return RET_EINVAL;
+  const size_t need = retention_chunkwise_workspace_bytes(chunk, s, dt);
+  if (need > kStaticWsBytes) return RET_EUNSUPPORTED;  // beyond the fixed scratch
+  void* ws = nullptr;
+  if (need > 0) {
+    ws = static_ws_address(&rc);
+    if (rc != RET_OK) return rc;
+  }
+  return retention_chunkwise(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, ws,
+                             need > 0 ? kStaticWsBytes : 0, stream);
 }
 
 }  // extern "C"
