@@ -138,11 +138,50 @@ __device__ __forceinline__ void store_row32_sw128(uint8_t* tile, uint32_t box_by
   }
 }
 
+// Store 32 columns of 32 rows (one row per lane, 32 fp32 each, scaled by f)
+// as bf16 with fewer memory transactions: a 4x4 transpose of 16-byte pieces
+// inside each lane quad (two shuffle stages) makes every store instruction
+// write 8 rows x 64 contiguous bytes instead of 32 rows x 16 bytes.
+// `row0` points at column c0 of the warp's first row; rows with
+// (lane-row >= nrows) are not written.
+__device__ __forceinline__ void store_rows_bf16_quad(__nv_bfloat16* row0, size_t row_stride, int lane,
+                                                     const uint32_t (&o)[32], float f, int nrows) {
+  uint32_t c[4][4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      c[k][e] = pack_bf16x2(f * __uint_as_float(o[8 * k + 2 * e]), f * __uint_as_float(o[8 * k + 2 * e + 1]));
+  const bool b0 = lane & 1, b1 = lane & 2;
+#pragma unroll
+  for (int k = 0; k < 4; k += 2)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, b0 ? c[k][e] : c[k + 1][e], 1);
+      if (b0) c[k][e] = recv; else c[k + 1][e] = recv;
+    }
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, b1 ? c[k][e] : c[k + 2][e], 2);
+      if (b1) c[k][e] = recv; else c[k + 2][e] = recv;
+    }
+  // lane = 4m + p now holds piece p (columns 8p..8p+7) of rows 4m .. 4m+3
+  const int m = lane >> 2, p = lane & 3;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int row = 4 * m + k;
+    if (row < nrows)
+      *reinterpret_cast<uint4*>(row0 + (size_t)row * row_stride + 8 * p) = make_uint4(c[k][0], c[k][1], c[k][2], c[k][3]);
+  }
+}
+
 template <int DK>
 __global__ void __launch_bounds__(kCW_MainThreads, 1)
 chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-                    const __grid_constant__ CUtensorMap mapV, const CwArgs a,
-                    const __grid_constant__ CwDecay dec) {
+                    const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapY,
+                    const CwArgs a, const __grid_constant__ CwDecay dec) {
   static_assert(DK == 64 || DK == 128 || DK == 256, "dk must be 64, 128 or 256");
   constexpr int NP = (DK <= 128) ? 2 : 1;
   constexpr uint32_t TM_S = 0, TM_P = DK, TM_O = DK + 128 * NP;
@@ -162,7 +201,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   uint64_t* fullV = bars + 8;      // [4] TMA -> V group, MMA
   uint64_t* emptyQ = bars + 12;    // [4] MMA4 done -> producer
   uint64_t* emptyK = bars + 16;    // [4] MMA5 done -> producer
-  uint64_t* emptyV = bars + 20;    // [4] MMA3 done -> producer
+  uint64_t* emptyV = bars + 20;    // [4] y of the block stored out of the V buffer -> producer
   uint64_t* zready = bars + 24;    // [4] V group: scaled V of stage s written -> MMA5 (and MMA3)
   uint64_t* pfull = bars + 28;     // [2] MMA1 done -> P/O group
   uint64_t* pfree = bars + 30;     // [2] MMA3 done -> MMA1 of block it+NP
@@ -172,6 +211,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   uint64_t* mma3done = bars + 36;  // MMA3 done -> P/O group (y)
   uint64_t* ofree = bars + 37;     // P/O group: O read out -> V group, MMA4 of the next block
   uint64_t* fin = bars + 38;       // teardown drain of the MMA pipe
+  uint64_t* ystaged = bars + 34;   // P/O group: y of the block staged in shared memory -> TMA store
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 39);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 39) + 1;
   float* pw = reinterpret_cast<float*>(bars + 40);  // gamma^0 .. gamma^128
@@ -209,6 +249,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     mbar_init(sready, 128);
     mbar_init(mma3done, 1);
     mbar_init(ofree, 128);
+    mbar_init(ystaged, 128);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -358,7 +399,6 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         }
         mma_commit(&pfree[pb]);
         mma_commit(mma3done);
-        mma_commit(&emptyV[s]);
       }
       mma_commit(fin);
       mbar_drain(fin, 0, a.lim);
@@ -567,35 +607,60 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       mbar_arrive(pready);
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 6);
       // O -> y once MMA3 added P~ V.  Rescaled form: y_r = gamma^(r+1-l) O_r.
-      // O is read into registers (as bf16) and released before the global
-      // stores, so the next block's MMA4 need not wait for them.
       if (!mbar_wait(mma3done, it & 1, abort_flag, a.lim)) break;
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 9);
       tc_fence_after();
-      {
-        const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) : 1.f;
-        uint32_t yw[kCW_DVT / 2];
+      const int s = it % NS;
+      const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) : 1.f;
+      if (NS >= 2) {
+        // The V tile is dead after MMA3 and its buffer is not needed again for
+        // NS-1 blocks: stage y there (bf16, 128B-swizzled) for two TMA tensor
+        // stores; the producer reloads the buffer once the stores have read it.
+        uint8_t* ystage = sV + s * sp.v_stage;
 #pragma unroll
         for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(tm + lane_off + TM_O + c0, o);
           tmem_ld_wait();
+          float x[32];
 #pragma unroll
-          for (int u = 0; u < 16; ++u)
-            yw[c0 / 2 + u] = pack_bf16x2(yf * __uint_as_float(o[2 * u]), yf * __uint_as_float(o[2 * u + 1]));
+          for (int u = 0; u < 32; ++u) x[u] = yf * __uint_as_float(o[u]);
+          if (r < C) store_row32_sw128(ystage, (uint32_t)C * 128u, (uint32_t)r, (uint32_t)c0, x);
         }
         tc_fence_before();
         mbar_arrive(ofree);
-        if (r < l) {
-          uint4* dst = reinterpret_cast<uint4*>(a.y + ((size_t)bh * a.L + t0 + r) * a.dv + vt * kCW_DVT);
-#pragma unroll
-          for (int q4 = 0; q4 < kCW_DVT / 8; ++q4)
-            dst[q4] = make_uint4(yw[4 * q4], yw[4 * q4 + 1], yw[4 * q4 + 2], yw[4 * q4 + 3]);
+        fence_proxy_async_smem();
+        mbar_arrive(ystaged);
+        if (r == 0) {
+          if (!mbar_wait(ystaged, it & 1, abort_flag, a.lim)) break;
+          tma_store_3d(&mapY, ystage, vt * kCW_DVT, t0, bh);
+          tma_store_3d(&mapY, ystage + C * 128, vt * kCW_DVT + 64, t0, bh);
+          bulk_commit_group();
+          bulk_wait_read_all();
+          mbar_arrive(&emptyV[s]);
         }
+      } else {
+        // Single stage: the V buffer is reloaded at once, so y goes straight
+        // from registers to global memory (quad-transposed stores).
+        if (r == 0) mbar_arrive(&emptyV[s]);
+        __nv_bfloat16* wrow0 = a.y + ((size_t)bh * a.L + t0 + row_lo) * a.dv + vt * kCW_DVT;
+#pragma unroll
+        for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tm + lane_off + TM_O + c0, o);
+          tmem_ld_wait();
+          // the factor differs per row: scale before the transpose
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(yf * __uint_as_float(o[u]));
+          store_rows_bf16_quad(wrow0 + c0, (size_t)a.dv, lane, o, 1.f, l - row_lo);
+        }
+        tc_fence_before();
+        mbar_arrive(ofree);
       }
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 7);
     }
   }
+  if (threadIdx.x == 0) bulk_wait_all();  // y stores issued by this thread are complete
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma) {

@@ -149,9 +149,9 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
                                void* y, const float* state_in, float* state_out, int C,
                                const ret_shape& s, void* ws, size_t ws_bytes, cudaStream_t st) {
   const int BH = s.B * s.H;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, my;
   if (!make_map(&mq, q, DK, s.L, BH, C) || !make_map(&mk, k, DK, s.L, BH, C) ||
-      !make_map(&mv, v, s.dv, s.L, BH, C))
+      !make_map(&mv, v, s.dv, s.L, BH, C) || !make_map(&my, y, s.dv, s.L, BH, C))
     return RET_ECUDA;
   static CwDecay dec;  // staged on the host; copied into the launch's parameters
   static std::mutex mu;
@@ -219,7 +219,7 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
                            (int)plan.total) != cudaSuccess)
     return RET_ECUDA;
   dim3 grid(s.dv / kCW_DVT, BH, n_seg);
-  chunkwise_tc_kernel<DK><<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, a, dec);
+  chunkwise_tc_kernel<DK><<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, my, a, dec);
   return launch_status();
 }
 
