@@ -671,6 +671,389 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
 }
 
 // ------------------------------------------------------------------------
+// dk = 256: one stage, with the scores and the cross-block term fused into a
+// single N = C + 128 MMA per K step:  [P | X] = Q [K ; Sb]^T, where the bf16
+// state copy Sb sits in shared memory right after the K rows of each 64-column
+// box and X (the cross-block term, then the whole output O) sits in TMEM right
+// after P.  Q is read once per block and the wide instruction keeps the tensor
+// core near its peak rate; TMEM holds S^T [0, 256) and [P | X] [256, 512).
+// Order per block: MMA14 ([P | X]; frees Q), MMA5 (state update; frees K),
+// MMA3 (X += P~ V; frees V).
+struct Cw256Smem {
+  uint32_t q, ks, v, misc, total, ks_box;
+};
+
+__host__ __device__ inline Cw256Smem cw256_smem_plan(int C) {
+  Cw256Smem s;
+  s.ks_box = (uint32_t)(C + 128) * 128u;  // K rows 0..C-1, then Sb rows (dv columns 0..127)
+  s.q = 0;
+  s.ks = 4u * 16384u;
+  s.v = s.ks + 4u * s.ks_box;
+  s.misc = s.v + 2u * (uint32_t)C * 128u;
+  s.total = s.misc + kMiscBytes + kSmemAlign;
+  return s;
+}
+
+__global__ void __launch_bounds__(kCW_MainThreads, 1)
+chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                       const __grid_constant__ CUtensorMap mapV, const CwArgs a,
+                       const __grid_constant__ CwDecay dec) {
+  constexpr int DK = 256;
+  constexpr uint32_t kTmemCols = 512, TM_S = 0, TM_P = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align_smem(smem_raw);
+  const int C = a.C;
+  const uint32_t TM_X = TM_P + (uint32_t)C;
+  const Cw256Smem sp = cw256_smem_plan(C);
+  uint8_t* sQ = base + sp.q;
+  uint8_t* sKS = base + sp.ks;
+  uint8_t* sV = base + sp.v;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + sp.misc);
+  uint64_t* fullQ = bars + 0;
+  uint64_t* fullK = bars + 1;
+  uint64_t* fullV = bars + 2;
+  uint64_t* emptyQ = bars + 3;     // MMA14 done
+  uint64_t* emptyK = bars + 4;     // MMA5 done
+  uint64_t* emptyV = bars + 5;     // MMA3 done
+  uint64_t* zready = bars + 6;     // V group: zeta applied (to V, or to K in the direct form)
+  uint64_t* pxfull = bars + 7;     // MMA14 done -> P/O group, V group (direct form)
+  uint64_t* pready = bars + 8;     // P/O group: P~ (and xi X) written -> MMA3
+  uint64_t* mma5done = bars + 9;   // MMA5 done -> S group
+  uint64_t* sready = bars + 10;    // S group: Sb + rescaled state written -> MMA14, MMA5
+  uint64_t* mma3done = bars + 11;  // MMA3 done -> P/O group (y)
+  uint64_t* ofree = bars + 12;     // P/O group: X read out -> MMA14 of the next block
+  uint64_t* fin = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14) + 1;
+  float* pw = reinterpret_cast<float*>(bars + 16);  // gamma^0 .. gamma^128
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int vt = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;
+  const float l2g = dec.l2g[bh % a.H];
+  const bool rescaled = (float)(C - 1) * l2g >= -64.f;
+  const int n_total = (a.L + C - 1) / C;
+  const int c_begin = seg * a.seg_chunks;
+  const int c_end = min(c_begin + a.seg_chunks, n_total);
+  const int nck = max(c_end - c_begin, 0);
+  const int cta_id = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  (void)cta_id;
+  RET_TRACE_INIT();
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+    mbar_init(zready, 128);
+    mbar_init(pxfull, 1);
+    mbar_init(pready, 128);
+    mbar_init(mma5done, 1);
+    mbar_init(sready, 128);
+    mbar_init(mma3done, 1);
+    mbar_init(ofree, 128);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int n = threadIdx.x; n <= 128; n += kCW_MainThreads) pw[n] = n == 0 ? 1.f : exp2f((float)n * l2g);
+  if (C < 128) {  // rows C..127 of every Q box are read by the M = 128 MMA: keep them zero
+    const uint32_t rows16 = (128u - (uint32_t)C) * 8u;
+    for (uint32_t e = threadIdx.x; e < 4u * rows16; e += kCW_MainThreads) {
+      const uint32_t b = e / rows16, o = e % rows16;
+      *reinterpret_cast<uint4*>(sQ + b * 16384u + (uint32_t)C * 128u + o * 16u) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tmem_slot;
+
+  if (warp == kWarpProducer) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nck > 0) {
+      tma_prefetch_desc(&mapQ);
+      tma_prefetch_desc(&mapK);
+      tma_prefetch_desc(&mapV);
+      const uint32_t qk_bytes = (uint32_t)DK * (uint32_t)C * 2u;
+      const uint32_t v_bytes = (uint32_t)kCW_DVT * (uint32_t)C * 2u;
+      int issued = 0;
+      for (int it = 0; it < nck; ++it) {
+        const uint32_t par = (it - 1) & 1;
+        const int t0 = (c_begin + it) * C;
+        if (it >= 1 && !mbar_wait(emptyQ, par, abort_flag, a.lim)) break;
+        mbar_arrive_expect_tx(fullQ, qk_bytes);
+        for (int b = 0; b < 4; ++b) tma_load_3d(sQ + b * 16384, &mapQ, fullQ, b * 64, t0, bh);
+        if (it >= 1 && !mbar_wait(emptyK, par, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, it, 0);
+        mbar_arrive_expect_tx(fullK, qk_bytes);
+        for (int b = 0; b < 4; ++b) tma_load_3d(sKS + b * sp.ks_box, &mapK, fullK, b * 64, t0, bh);
+        if (it >= 1 && !mbar_wait(emptyV, par, abort_flag, a.lim)) break;
+        mbar_arrive_expect_tx(fullV, v_bytes);
+        for (int b = 0; b < 2; ++b) tma_load_3d(sV + b * C * 128, &mapV, fullV, vt * kCW_DVT + b * 64, t0, bh);
+        issued = it + 1;
+        if (it + 1 < nck) {  // next block's tiles into L2 while this one runs
+          const int tp = t0 + C;
+          for (int b = 0; b < 4; ++b) {
+            tma_prefetch_l2_3d(&mapQ, b * 64, tp, bh);
+            tma_prefetch_l2_3d(&mapK, b * 64, tp, bh);
+          }
+          for (int b = 0; b < 2; ++b) tma_prefetch_l2_3d(&mapV, vt * kCW_DVT + b * 64, tp, bh);
+        }
+      }
+      if (issued > 0) {
+        mbar_drain(fullQ, (issued - 1) & 1, a.lim);
+        mbar_drain(fullK, (issued - 1) & 1, a.lim);
+        mbar_drain(fullV, (issued - 1) & 1, a.lim);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0 && nck > 0) {
+      const uint32_t id14 = idesc_bf16(128, C + 128, false, false);
+      const uint32_t id5 = idesc_bf16(128, DK, true, true);
+      const uint32_t id3 = idesc_bf16(128, kCW_DVT, false, true);
+      const uint32_t aQ = smem_u32(sQ), aKS = smem_u32(sKS), aV = smem_u32(sV);
+      for (int it = 0; it < nck; ++it) {
+        const uint32_t par = it & 1;
+        if (!mbar_wait(fullQ, par, abort_flag, a.lim)) break;
+        if (!mbar_wait(fullK, par, abort_flag, a.lim)) break;
+        if (!mbar_wait(sready, par, abort_flag, a.lim)) break;
+        if (!mbar_wait(ofree, par, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, it, 1);
+        tc_fence_after();
+        // MMA14: [P | X] = Q [K ; Sb]^T
+#pragma unroll
+        for (int kk = 0; kk < DK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(aQ + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(aKS + (kk / 4) * sp.ks_box + (kk % 4) * 32, 16, 1024);
+          mma_ss(tm + TM_P, ad, bd, id14, kk > 0);
+        }
+        mma_commit(pxfull);
+        mma_commit(emptyQ);
+        // MMA5: S^T += (zeta V)^T K  (rescaled: zeta on V; direct: zeta on K)
+        if (!mbar_wait(zready, par, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, it, 2);
+        tc_fence_after();
+        for (int kk = 0; kk < C / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(aV + kk * 2048, C * 128, 1024);
+          const uint64_t bd = sdesc_sw128(aKS + kk * 2048, sp.ks_box, 1024);
+          mma_ss(tm + TM_S, ad, bd, id5, 1);
+        }
+        mma_commit(mma5done);
+        mma_commit(emptyK);
+        // MMA3: X += P~ V
+        if (!mbar_wait(pready, par, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, it, 4);
+        tc_fence_after();
+        for (int kk = 0; kk < C / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(aV + kk * 2048, C * 128, 1024);
+          mma_ts(tm + TM_X, tm + TM_P + kk * 8, bd, id3, 1);
+        }
+        mma_commit(mma3done);
+        mma_commit(emptyV);
+      }
+      mma_commit(fin);
+      mbar_drain(fin, 0, a.lim);
+    }
+  } else if (warp >= kWarpZBase) {
+    // ---------------------------------------------------- V group (4 warps)
+    // zeta_j = gamma^(l-1-j) (0 past the block end) applied to row j of V
+    // (rescaled form, any time after V lands) or of K (direct form, after
+    // MMA14 has read the unscaled K).
+    const uint32_t t = threadIdx.x - kWarpZBase * 32;
+    for (int it = 0; it < nck; ++it) {
+      const uint32_t par = it & 1;
+      if (!mbar_wait(fullV, par, abort_flag, a.lim)) break;
+      if (!rescaled) {
+        if (!mbar_wait(fullK, par, abort_flag, a.lim)) break;
+        if (!mbar_wait(pxfull, par, abort_flag, a.lim)) break;
+      }
+      const int l = min(C, a.L - (c_begin + it) * C);
+      if ((int)t < C) {
+        const float zeta = ((int)t < l) ? pw[l - 1 - (int)t] : 0.f;
+        if (rescaled) {
+          scale_row_sw128(sV, t, zeta);
+          scale_row_sw128(sV + C * 128, t, zeta);
+        } else {
+          for (int b = 0; b < 4; ++b) scale_row_sw128(sKS + b * sp.ks_box, t, zeta);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(zready);
+      if (t == 0) RET_TRACE_STAMP(cta_id, it, 3);
+    }
+  } else if (warp >= kWarpSBase) {
+    // ---------------------------------------------------- S group (4 warps)
+    // lane v: dv column v of S^T; writes Sb (rows C..C+127 of each KS box).
+    const uint32_t v_loc = threadIdx.x - kWarpSBase * 32;
+    const uint32_t lane_off = (uint32_t)((warp - kWarpSBase) * 32) << 16;
+    const int v = vt * kCW_DVT + (int)v_loc;
+    const size_t dkdv = (size_t)DK * a.dv;
+    uint8_t* sSb = sKS + (uint32_t)C * 128u;  // first Sb row of box 0; box stride ks_box
+    {
+      const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
+                                       : (a.state_in ? a.state_in + (size_t)bh * dkdv : nullptr);
+      const int l0 = min(C, a.L - c_begin * C);
+      const float g0 = pw[max(l0, 0)];
+      const float gc = rescaled ? g0 : 1.f;
+      for (int d0 = 0; d0 < DK; d0 += 32) {
+        float x[32];
+        uint32_t w[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) {
+          const float sv = src ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
+          x[u] = gc * sv;
+          w[u] = __float_as_uint(g0 * sv);
+        }
+        store_row32_sw128(sSb, sp.ks_box, v_loc, d0, x);
+        tmem_st32(tm + lane_off + TM_S + d0, w);
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(sready);
+    }
+    for (int it = 0; it < nck; ++it) {
+      // MMA5 done; MMA14 (the reader of the old Sb) ran before it
+      if (!mbar_wait(mma5done, it & 1, abort_flag, a.lim)) break;
+      tc_fence_after();
+      const int t0 = (c_begin + it) * C;
+      if (it < nck - 1) {
+        const float gn = pw[min(C, a.L - t0 - C)];
+        for (int d0 = 0; d0 < DK; d0 += 32) {
+          uint32_t sr[32];
+          tmem_ld32(tm + lane_off + TM_S + d0, sr);
+          tmem_ld_wait();
+          float x[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const float sv = __uint_as_float(sr[u]);
+            const float sg = gn * sv;
+            x[u] = rescaled ? sg : sv;
+            sr[u] = __float_as_uint(sg);
+          }
+          store_row32_sw128(sSb, sp.ks_box, v_loc, d0, x);
+          tmem_st32(tm + lane_off + TM_S + d0, sr);
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(sready);
+        if (v_loc == 0) RET_TRACE_STAMP(cta_id, it, 8);
+      } else if (a.state_out && seg == a.n_seg - 1) {
+        float* so = a.state_out + (size_t)bh * dkdv;
+        for (int d0 = 0; d0 < DK; d0 += 32) {
+          uint32_t sr[32];
+          tmem_ld32(tm + lane_off + TM_S + d0, sr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) so[(size_t)(d0 + u) * a.dv + v] = __uint_as_float(sr[u]);
+        }
+      }
+    }
+  } else {
+    // -------------------------------------------------- P/O group (4 warps)
+    const int r = (int)threadIdx.x;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int row_lo = warp * 32;
+    mbar_arrive(ofree);  // X starts free
+    for (int it = 0; it < nck; ++it) {
+      const uint32_t par = it & 1;
+      const int t0 = (c_begin + it) * C;
+      const int l = min(C, a.L - t0);
+      if (!mbar_wait(pxfull, par, abort_flag, a.lim)) break;
+      tc_fence_after();
+      // P -> P~ in place (see the main kernel for the two forms)
+      const uint32_t tp = tm + lane_off + TM_P;
+      for (int j0 = 0; j0 < C; j0 += 32) {
+        uint32_t pr[32];
+        tmem_ld32(tp + j0, pr);
+        tmem_ld_wait();
+        uint32_t w[16];
+        if (j0 >= row_lo + 32) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) w[u] = 0u;
+        } else if (rescaled) {
+          if (j0 + 31 <= row_lo) {
+#pragma unroll
+            for (int u = 0; u < 32; u += 2) w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]), __uint_as_float(pr[u + 1]));
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; u += 2) {
+              const int j = j0 + u;
+              w[u / 2] = pack_bf16x2((j <= r) ? __uint_as_float(pr[u]) : 0.f,
+                                     (j + 1 <= r) ? __uint_as_float(pr[u + 1]) : 0.f);
+            }
+          }
+        } else if (j0 + 31 <= row_lo) {
+          const float ar = pw[r - j0 - 31];
+#pragma unroll
+          for (int u = 0; u < 32; u += 2)
+            w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * ar * pw[31 - u],
+                                   __uint_as_float(pr[u + 1]) * ar * pw[30 - u]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; u += 2) {
+            const int j = j0 + u;
+            const float f0 = (j <= r) ? pw[r - j] : 0.f;
+            const float f1 = (j + 1 <= r) ? pw[r - j - 1] : 0.f;
+            w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * f0, __uint_as_float(pr[u + 1]) * f1);
+          }
+        }
+        // For C % 32 == 16 the last piece reads 16 columns past P (the start of
+        // X) and writes packed results below column C/2 + 8 < C: never into X,
+        // never read by MMA3.
+        tmem_st16(tp + j0 / 2, w);
+      }
+      if (!rescaled) {
+        // X *= xi_r = gamma^(r+1): X holds Q S_prev from MMA14
+        const float xi = pw[r + 1];
+        for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tm + lane_off + TM_X + c0, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * xi);
+          tmem_st32(tm + lane_off + TM_X + c0, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(pready);
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 6);
+      // y = (gamma^(r+1-l) in the rescaled form) X, once MMA3 is done
+      if (!mbar_wait(mma3done, par, abort_flag, a.lim)) break;
+      tc_fence_after();
+      {
+        const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) : 1.f;
+        __nv_bfloat16* wrow0 = a.y + ((size_t)bh * a.L + t0 + row_lo) * a.dv + vt * kCW_DVT;
+#pragma unroll
+        for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tm + lane_off + TM_X + c0, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(yf * __uint_as_float(o[u]));
+          store_rows_bf16_quad(wrow0 + c0, (size_t)a.dv, lane, o, 1.f, l - row_lo);
+        }
+        tc_fence_before();
+        mbar_arrive(ofree);
+      }
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 7);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tm, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------
 // Segment sums for the sequence split: for segment g of one (b, h) and one
 // 128-column dv slice,  D_g^T = sum_{t in g} gamma^(e_g - t) v_t^T k_t  with e_g
 // the segment's last token, written (as [dk][dv], like a state) to slot g+1 of

@@ -215,12 +215,24 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
                                               n_seg, seg_chunks * C, dec);
     if (launch_status() != RET_OK) return RET_ECUDA;
   }
-  if (cudaFuncSetAttribute(chunkwise_tc_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)plan.total) != cudaSuccess)
-    return RET_ECUDA;
   dim3 grid(s.dv / kCW_DVT, BH, n_seg);
-  chunkwise_tc_kernel<DK><<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, my, a, dec);
-  return launch_status();
+  if constexpr (DK == 256) {
+    // one stage; scores and cross-block term fused into one wide MMA
+    const Cw256Smem p256 = cw256_smem_plan(C);
+    if ((int)p256.total > smax) return RET_EUNSUPPORTED;
+    a.nstages = 1;
+    if (cudaFuncSetAttribute(chunkwise_tc256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)p256.total) != cudaSuccess)
+      return RET_ECUDA;
+    chunkwise_tc256_kernel<<<grid, kCW_MainThreads, p256.total, st>>>(mq, mk, mv, a, dec);
+    return launch_status();
+  } else {
+    if (cudaFuncSetAttribute(chunkwise_tc_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)plan.total) != cudaSuccess)
+      return RET_ECUDA;
+    chunkwise_tc_kernel<DK><<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, my, a, dec);
+    return launch_status();
+  }
 }
 
 template <int DK>
