@@ -745,7 +745,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
     mbar_init(pxfull, 1);
     mbar_init(pready, 128);
     mbar_init(mma5done, 1);
-    mbar_init(sready, 128);
+    mbar_init(sready, 256);  // S group and V group each rescale half of dk
     mbar_init(mma3done, 1);
     mbar_init(ofree, 128);
     mbar_init(fin, 1);
@@ -857,38 +857,18 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       mma_commit(fin);
       mbar_drain(fin, 0, a.lim);
     }
-  } else if (warp >= kWarpZBase) {
-    // ---------------------------------------------------- V group (4 warps)
-    // zeta_j = gamma^(l-1-j) (0 past the block end) applied to row j of V
-    // (rescaled form, any time after V lands) or of K (direct form, after
-    // MMA14 has read the unscaled K).
-    const uint32_t t = threadIdx.x - kWarpZBase * 32;
-    for (int it = 0; it < nck; ++it) {
-      const uint32_t par = it & 1;
-      if (!mbar_wait(fullV, par, abort_flag, a.lim)) break;
-      if (!rescaled) {
-        if (!mbar_wait(fullK, par, abort_flag, a.lim)) break;
-        if (!mbar_wait(pxfull, par, abort_flag, a.lim)) break;
-      }
-      const int l = min(C, a.L - (c_begin + it) * C);
-      if ((int)t < C) {
-        const float zeta = ((int)t < l) ? pw[l - 1 - (int)t] : 0.f;
-        if (rescaled) {
-          scale_row_sw128(sV, t, zeta);
-          scale_row_sw128(sV + C * 128, t, zeta);
-        } else {
-          for (int b = 0; b < 4; ++b) scale_row_sw128(sKS + b * sp.ks_box, t, zeta);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(zready);
-      if (t == 0) RET_TRACE_STAMP(cta_id, it, 3);
-    }
   } else if (warp >= kWarpSBase) {
-    // ---------------------------------------------------- S group (4 warps)
-    // lane v: dv column v of S^T; writes Sb (rows C..C+127 of each KS box).
-    const uint32_t v_loc = threadIdx.x - kWarpSBase * 32;
-    const uint32_t lane_off = (uint32_t)((warp - kWarpSBase) * 32) << 16;
+    // ------------------------------------------ S group and V group (8 warps)
+    // Both keep the state: lane v owns dv column v of S^T; the S group the dk
+    // columns [0, 128), the V group [128, 256).  The state copy Sb sits in rows
+    // C..C+127 of each KS box.  The V group also applies zeta_j = gamma^(l-1-j)
+    // (0 past the block end) to row j of V (rescaled form, as soon as V lands)
+    // or of K (direct form, once MMA14 has read the unscaled K).
+    const bool vgrp = warp >= kWarpZBase;
+    const int gbase = vgrp ? kWarpZBase : kWarpSBase;
+    const uint32_t v_loc = threadIdx.x - gbase * 32;
+    const uint32_t lane_off = (uint32_t)((warp - gbase) * 32) << 16;
+    const int d_lo = vgrp ? 128 : 0;
     const int v = vt * kCW_DVT + (int)v_loc;
     const size_t dkdv = (size_t)DK * a.dv;
     uint8_t* sSb = sKS + (uint32_t)C * 128u;  // first Sb row of box 0; box stride ks_box
@@ -898,7 +878,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       const int l0 = min(C, a.L - c_begin * C);
       const float g0 = pw[max(l0, 0)];
       const float gc = rescaled ? g0 : 1.f;
-      for (int d0 = 0; d0 < DK; d0 += 32) {
+      for (int d0 = d_lo; d0 < d_lo + 128; d0 += 32) {
         float x[32];
         uint32_t w[32];
 #pragma unroll
@@ -916,13 +896,34 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       mbar_arrive(sready);
     }
     for (int it = 0; it < nck; ++it) {
-      // MMA5 done; MMA14 (the reader of the old Sb) ran before it
-      if (!mbar_wait(mma5done, it & 1, abort_flag, a.lim)) break;
-      tc_fence_after();
+      const uint32_t par = it & 1;
       const int t0 = (c_begin + it) * C;
+      if (vgrp) {
+        if (!mbar_wait(fullV, par, abort_flag, a.lim)) break;
+        if (!rescaled) {
+          if (!mbar_wait(fullK, par, abort_flag, a.lim)) break;
+          if (!mbar_wait(pxfull, par, abort_flag, a.lim)) break;
+        }
+        const int l = min(C, a.L - t0);
+        if ((int)v_loc < C) {
+          const float zeta = ((int)v_loc < l) ? pw[l - 1 - (int)v_loc] : 0.f;
+          if (rescaled) {
+            scale_row_sw128(sV, v_loc, zeta);
+            scale_row_sw128(sV + C * 128, v_loc, zeta);
+          } else {
+            for (int b = 0; b < 4; ++b) scale_row_sw128(sKS + b * sp.ks_box, v_loc, zeta);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(zready);
+        if (v_loc == 0) RET_TRACE_STAMP(cta_id, it, 3);
+      }
+      // MMA5 done; MMA14 (the reader of the old Sb) ran before it
+      if (!mbar_wait(mma5done, par, abort_flag, a.lim)) break;
+      tc_fence_after();
       if (it < nck - 1) {
         const float gn = pw[min(C, a.L - t0 - C)];
-        for (int d0 = 0; d0 < DK; d0 += 32) {
+        for (int d0 = d_lo; d0 < d_lo + 128; d0 += 32) {
           uint32_t sr[32];
           tmem_ld32(tm + lane_off + TM_S + d0, sr);
           tmem_ld_wait();
@@ -941,10 +942,10 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(sready);
-        if (v_loc == 0) RET_TRACE_STAMP(cta_id, it, 8);
+        if (v_loc == 0 && !vgrp) RET_TRACE_STAMP(cta_id, it, 8);
       } else if (a.state_out && seg == a.n_seg - 1) {
         float* so = a.state_out + (size_t)bh * dkdv;
-        for (int d0 = 0; d0 < DK; d0 += 32) {
+        for (int d0 = d_lo; d0 < d_lo + 128; d0 += 32) {
           uint32_t sr[32];
           tmem_ld32(tm + lane_off + TM_S + d0, sr);
           tmem_ld_wait();
