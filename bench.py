@@ -39,13 +39,13 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from retnet_retention_chunkwise_b200 import inputs  # noqa: E402
+from retnet_retention_chunkwise_b200 import inputs, replicas  # noqa: E402
 
 METRIC = "retention tokens/sec (chunkwise fwd, decode) and % of tensor/HBM roofline"
 HEADLINE = inputs.WORKLOADS["retnet1p3b_layer_bf16"]
 L2_BYTES = 126 * 1024 * 1024
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "chunkwise_tc_retnet1p3b_layer.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "chunkwise_tc256_retnet1p3b_layer.md")
 
 
 # --------------------------------------------------------------- accounting
@@ -186,18 +186,10 @@ class Dist:
             torch.cuda.synchronize()
 
     def max(self, x: float) -> float:
-        if not self.pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x, device="cuda")
 
     def sum(self, x: float) -> float:
-        if not self.pg:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t)
-        return float(t.item())
+        return replicas.sum_over_ranks(x, device="cuda")
 
     def close(self):
         if self.pg:
@@ -206,16 +198,8 @@ class Dist:
 
 # ------------------------------------------------------------------ helpers
 def gpu_qkv(B, H, L, dk, dv, seed):
-    """Seeded N(0,1)/sqrt(dk) bf16 q, k, v drawn on the device (same recipe as
-    inputs.qkv, device generator; values are not compared with the oracle here)."""
-    g = torch.Generator(device="cuda").manual_seed(seed)
-    s = 1.0 / math.sqrt(dk)
-    out = []
-    for d in (dk, dk, dv):
-        t = torch.empty((B, H, L, d), dtype=torch.bfloat16, device="cuda")
-        t.copy_(torch.randn((B, H, L, d), generator=g, device="cuda") * s)
-        out.append(t)
-    return out
+    """Seeded N(0,1)/sqrt(dk) bf16 q, k, v drawn on the device."""
+    return list(inputs.qkv_cuda(B, H, L, dk, dv, torch.bfloat16, seed))
 
 
 _FLUSH = None
@@ -287,7 +271,7 @@ def bench_headline(ret, args, dist, peaks):
             "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
             "frac": round((ach_gbs / peaks["hbm_gbs"]) if bound == "hbm" else (ach_tf / peaks["bf16_tflops"]), 4),
             "traffic": measured_traffic(),
-            "kernel": "chunkwise_tc_kernel<256>",
+            "kernel": "chunkwise_tc256_kernel",
             "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
             "kernel_ms": round(kern_ms, 4),
             "tensor": {"achieved_tflops": round(ach_tf, 1), "peak": peaks["bf16_tflops"],
@@ -324,7 +308,7 @@ def bench_e2e(ret, args, dist):
         ret.chunkwise(qd, kd, vd, gam, w.chunk, state_out=sd, out=yd)
         yh.copy_(yd, non_blocking=True)
 
-    steps = max(3, min(args.steps, 20))
+    steps = 10
     _, total = time_calls(step, steps, max(args.warmup, 3), dist)
     t_ms = dist.max(total / steps)
     value = dist.sum(w.B * w.L * steps) / (t_ms * 1e-3 * steps)
@@ -381,7 +365,7 @@ def bench_small(ret, args, dist, peaks):
     q, k, v = gpu_qkv(w.B, w.H, w.L, w.dk, w.dv, seed=0)
     gam = w.gammas()
     y = torch.empty_like(v)
-    n = max(args.steps, 10)
+    n = 50
     per, _ = time_calls(lambda: ret.parallel(q, k, v, gam, out=y), n, max(args.warmup, 3), dist, flush=True)
     t = dist.max(statistics.median(per))
     fl = parallel_flops(w.B, w.H, w.L, w.dk, w.dv)
@@ -413,7 +397,7 @@ def bench_small(ret, args, dist, peaks):
             state.zero_()
             for qq, kk, vv in parts:
                 ret.chunkwise(qq, kk, vv, gam, C, state_in=state, state_out=state, out=y)
-        per, _ = time_calls(four_calls, max(args.steps // 2, 5), max(args.warmup, 3), dist)
+        per, _ = time_calls(four_calls, 10, max(args.warmup, 3), dist)
         t = dist.max(statistics.median(per))
         fl = w.B * w.H * w.L * chunk_flops_per_head_token(C, w.dk, w.dv)
         nb = chunk_bytes(w.B, w.H, w.L, w.dk, w.dv) + 2 * inputs.LONG_CONTEXT_CALLS * w.B * w.H * w.dk * w.dv * 4

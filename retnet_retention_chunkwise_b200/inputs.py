@@ -56,6 +56,19 @@ def qkv(B: int, H: int, L: int, dk: int, dv: int, dtype=torch.bfloat16, seed: in
     return q.to(dtype), k.to(dtype), v.to(dtype)
 
 
+def qkv_cuda(B: int, H: int, L: int, dk: int, dv: int, dtype=torch.bfloat16, seed: int = 0,
+             device="cuda"):
+    """Seeded q, k, v drawn on the device (torch CUDA generator), same recipe as
+    :func:`qkv`.  For workloads too large to draw on the host; the oracle reads
+    these exact bytes after a copy to the host."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    s = 1.0 / math.sqrt(dk)
+    out = []
+    for d in (dk, dk, dv):
+        out.append((torch.randn((B, H, L, d), generator=g, device=device, dtype=torch.float32) * s).to(dtype))
+    return tuple(out)
+
+
 def decode_tokens(steps: int, B: int, H: int, dk: int, dv: int, dtype=torch.bfloat16,
                   seed: int = 1):
     """Seeded single-token q, k [steps,B,H,1,dk] and v [steps,B,H,1,dv] for decode."""
