@@ -72,6 +72,7 @@ struct CwArgs {
   float* state_out;         // may be null
   const float* seg_state;   // [BH][n_seg][dk][dv] initial states when n_seg > 1
   WaitLimit lim;
+  int debug_drop_block;     // fault injection: block whose K load is never issued (-1 = none)
 };
 
 struct CwSmem {
@@ -303,9 +304,11 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         const int t0 = (c_begin + it) * C;
         if (it >= NS && !mbar_wait(&emptyK[s], par, abort_flag, a.lim)) break;
         RET_TRACE_STAMP(cta_id, it, 0);
-        mbar_arrive_expect_tx(&fullK[s], qk_bytes);
-        for (int b = 0; b < DK / 64; ++b)
-          tma_load_3d(sK + s * sp.k_stage + b * C * 128, &mapK, &fullK[s], b * 64, t0, bh);
+        if (c_begin + it != a.debug_drop_block) {  // fault injection: a load that never lands
+          mbar_arrive_expect_tx(&fullK[s], qk_bytes);
+          for (int b = 0; b < DK / 64; ++b)
+            tma_load_3d(sK + s * sp.k_stage + b * C * 128, &mapK, &fullK[s], b * 64, t0, bh);
+        }
         if (it >= NS && !mbar_wait(&emptyQ[s], par, abort_flag, a.lim)) break;
         mbar_arrive_expect_tx(&fullQ[s], qk_bytes);
         for (int b = 0; b < DK / 64; ++b)
@@ -787,8 +790,10 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         for (int b = 0; b < 4; ++b) tma_load_3d(sQ + b * 16384, &mapQ, fullQ, b * 64, t0, bh);
         if (it >= 1 && !mbar_wait(emptyK, par, abort_flag, a.lim)) break;
         RET_TRACE_STAMP(cta_id, it, 0);
-        mbar_arrive_expect_tx(fullK, qk_bytes);
-        for (int b = 0; b < 4; ++b) tma_load_3d(sKS + b * sp.ks_box, &mapK, fullK, b * 64, t0, bh);
+        if (c_begin + it != a.debug_drop_block) {  // fault injection: a load that never lands
+          mbar_arrive_expect_tx(fullK, qk_bytes);
+          for (int b = 0; b < 4; ++b) tma_load_3d(sKS + b * sp.ks_box, &mapK, fullK, b * 64, t0, bh);
+        }
         if (it >= 1 && !mbar_wait(emptyV, par, abort_flag, a.lim)) break;
         mbar_arrive_expect_tx(fullV, v_bytes);
         for (int b = 0; b < 2; ++b) tma_load_3d(sV + b * C * 128, &mapV, fullV, vt * kCW_DVT + b * 64, t0, bh);

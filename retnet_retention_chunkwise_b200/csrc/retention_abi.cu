@@ -28,16 +28,22 @@ using namespace ret;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 constexpr uint32_t kWaitIter = 1u << 24;      // polls (each parks for at most 100 us)
 
+// RETENTION_WAIT_LIMIT_MS (read at every launch) shortens or lengthens it.
 WaitLimit wait_limit() {
   WaitLimit w{kWaitNs, kWaitIter};
-  static int env_ms = -1;
-  if (env_ms < 0) {
-    const char* e = getenv("RETENTION_WAIT_LIMIT_MS");
-    env_ms = e ? atoi(e) : 0;
-    if (env_ms < 0) env_ms = 0;
-  }
-  if (env_ms > 0) w.ns = (uint64_t)env_ms * 1000000ull;
+  const char* e = getenv("RETENTION_WAIT_LIMIT_MS");
+  const int ms = e ? atoi(e) : 0;
+  if (ms > 0) w.ns = (uint64_t)ms * 1000000ull;
   return w;
+}
+
+// Fault injection for tests of the bounded-wait path: with
+// RETENTION_DEBUG_DROP_BLOCK=n (read at every launch) the chunkwise kernels
+// never issue the K load of block n, so the wait for it expires, the kernel
+// tears down and the device status reads RET_ETIMEOUT.  Unset: -1, no effect.
+int debug_drop_block() {
+  const char* e = getenv("RETENTION_DEBUG_DROP_BLOCK");
+  return e ? atoi(e) : -1;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -193,6 +199,7 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
   a.state_out = state_out;
   a.seg_state = static_cast<const float*>(ws);
   a.lim = wait_limit();
+  a.debug_drop_block = debug_drop_block();
 
   if (n_seg > 1) {
     // segment sums -> workspace slots 1..n_seg-1, then the scan fills every slot
@@ -202,6 +209,7 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
       if ((int)(n * per + kMiscBytes + kSmemAlign) <= smax) { ns2 = n; break; }
     CwArgs a2 = a;
     a2.nstages = ns2;
+    a2.debug_drop_block = -1;
     const int smem2 = (int)(ns2 * per + kMiscBytes + kSmemAlign);
     if (cudaFuncSetAttribute(chunk_state_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) !=
         cudaSuccess)
