@@ -273,8 +273,9 @@ ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const
   if (cudaFuncSetAttribute(parallel_tc_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)plan.total) != cudaSuccess)
     return RET_ECUDA;
-  dim3 grid(s.dv / 128, a.n_qt, BH);
-  parallel_tc_kernel<DK><<<grid, kCW_Threads, plan.total, st>>>(mq, mk, mv, a, dec);
+  // blockIdx.y = y pairs query tiles n_qt-1-y and y (one tile when they meet)
+  dim3 grid(s.dv / 128, (a.n_qt + 1) / 2, BH);
+  parallel_tc_kernel<DK><<<grid, kPA_Threads, plan.total, st>>>(mq, mk, mv, a, dec);
   return launch_status();
 }
 

@@ -147,7 +147,8 @@ def test_chunkwise_empty_sequence_passes_state():
 
 # ------------------------------------------------------- bf16 parallel (2e-2)
 @pytest.mark.parametrize("B,H,L,dk,dv", [(2, 8, 2048, 64, 128), (1, 2, 1000, 128, 256),
-                                         (1, 1, 300, 256, 128), (1, 3, 77, 64, 128)])
+                                         (1, 1, 300, 256, 128), (1, 3, 77, 64, 128),
+                                         (1, 2, 129, 256, 256), (3, 1, 512, 128, 384)])
 def test_parallel(B, H, L, dk, dv):
     q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed=L)
     gam = inputs.multiscale_gammas(H) if H != 3 else torch.tensor([0.0, 1.0, 0.7])
