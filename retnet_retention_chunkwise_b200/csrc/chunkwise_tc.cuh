@@ -145,14 +145,8 @@ __device__ __forceinline__ void store_row32_sw128(uint8_t* tile, uint32_t box_by
 // write 8 rows x 64 contiguous bytes instead of 32 rows x 16 bytes.
 // `row0` points at column c0 of the warp's first row; rows with
 // (lane-row >= nrows) are not written.
-__device__ __forceinline__ void store_rows_bf16_quad(__nv_bfloat16* row0, size_t row_stride, int lane,
-                                                     const uint32_t (&o)[32], float f, int nrows) {
-  uint32_t c[4][4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      c[k][e] = pack_bf16x2(f * __uint_as_float(o[8 * k + 2 * e]), f * __uint_as_float(o[8 * k + 2 * e + 1]));
+__device__ __forceinline__ void store_rows_quad_core(__nv_bfloat16* row0, size_t row_stride, int lane,
+                                                     uint32_t (&c)[4][4], int nrows) {
   const bool b0 = lane & 1, b1 = lane & 2;
 #pragma unroll
   for (int k = 0; k < 4; k += 2)
@@ -176,6 +170,28 @@ __device__ __forceinline__ void store_rows_bf16_quad(__nv_bfloat16* row0, size_t
     if (row < nrows)
       *reinterpret_cast<uint4*>(row0 + (size_t)row * row_stride + 8 * p) = make_uint4(c[k][0], c[k][1], c[k][2], c[k][3]);
   }
+}
+
+__device__ __forceinline__ void store_rows_bf16_quad(__nv_bfloat16* row0, size_t row_stride, int lane,
+                                                     const uint32_t (&o)[32], float f, int nrows) {
+  uint32_t c[4][4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      c[k][e] = pack_bf16x2(f * __uint_as_float(o[8 * k + 2 * e]), f * __uint_as_float(o[8 * k + 2 * e + 1]));
+  store_rows_quad_core(row0, row_stride, lane, c, nrows);
+}
+
+// Same, from 32 columns already packed as bf16 pairs (w[u] = columns 2u, 2u+1).
+__device__ __forceinline__ void store_rows_packed_quad(__nv_bfloat16* row0, size_t row_stride, int lane,
+                                                       const uint32_t (&w)[16], int nrows) {
+  uint32_t c[4][4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[k][e] = w[4 * k + e];
+  store_rows_quad_core(row0, row_stride, lane, c, nrows);
 }
 
 template <int DK>
@@ -682,6 +698,21 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
 // core near its peak rate; TMEM holds S^T [0, 256) and [P | X] [256, 512).
 // Order per block: MMA14 ([P | X]; frees Q), MMA5 (state update; frees K),
 // MMA3 (X += P~ V; frees V).
+// Scaled state (rescaled form): TMEM holds U, and the state decayed for the
+// coming block is rho * U.  After a block rho takes on gamma^l of the next
+// block instead of the state being multiplied in TMEM; only when rho would
+// drop below 2^-64 is U multiplied through (and rho reset to 1), so the
+// scaled operands (zeta V / rho, U) stay below 2^64 in magnitude.
+__device__ __forceinline__ float cw_rho_next(float rho, float gl) {
+  const float r = gl * rho;
+  return r < 0x1p-64f ? 1.f : r;
+}
+
+// rho for the first block of a segment (g0 = gamma^l0): 1 in the direct form.
+__device__ __forceinline__ float cw_rho_first(bool rescaled, float g0) {
+  return (rescaled && g0 >= 0x1p-64f) ? g0 : 1.f;
+}
+
 struct Cw256Smem {
   uint32_t q, ks, v, misc, total, ks_box;
 };
@@ -877,12 +908,16 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
     const int v = vt * kCW_DVT + (int)v_loc;
     const size_t dkdv = (size_t)DK * a.dv;
     uint8_t* sSb = sKS + (uint32_t)C * 128u;  // first Sb row of box 0; box stride ks_box
+    const float g0 = pw[max(min(C, a.L - c_begin * C), 0)];
+    float rho = cw_rho_first(rescaled, g0);
     {
       const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
                                        : (a.state_in ? a.state_in + (size_t)bh * dkdv : nullptr);
-      const int l0 = min(C, a.L - c_begin * C);
-      const float g0 = pw[max(l0, 0)];
-      const float gc = rescaled ? g0 : 1.f;
+      // TMEM starts as gu S_in: rescaled, U = S_in (or gamma^l0 S_in when rho
+      // was reset); direct, the decayed state gamma^l0 S_in.  Sb = bf16(U) in
+      // the rescaled form, S_in in the direct form.
+      const float gu = (rho == 1.f) ? g0 : 1.f;
+      const float gc = rescaled ? gu : 1.f;
       for (int d0 = d_lo; d0 < d_lo + 128; d0 += 32) {
         float x[32];
         uint32_t w[32];
@@ -890,7 +925,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         for (int u = 0; u < 32; ++u) {
           const float sv = src ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
           x[u] = gc * sv;
-          w[u] = __float_as_uint(g0 * sv);
+          w[u] = __float_as_uint(gu * sv);
         }
         store_row32_sw128(sSb, sp.ks_box, v_loc, d0, x);
         tmem_st32(tm + lane_off + TM_S + d0, w);
@@ -905,6 +940,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       const int t0 = (c_begin + it) * C;
       if (vgrp) {
         if (!mbar_wait(fullV, par, abort_flag, a.lim)) break;
+        if (v_loc == 0) RET_TRACE_STAMP(cta_id, it, 9);
         if (!rescaled) {
           if (!mbar_wait(fullK, par, abort_flag, a.lim)) break;
           if (!mbar_wait(pxfull, par, abort_flag, a.lim)) break;
@@ -913,8 +949,9 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         if ((int)v_loc < C) {
           const float zeta = ((int)v_loc < l) ? pw[l - 1 - (int)v_loc] : 0.f;
           if (rescaled) {
-            scale_row_sw128(sV, v_loc, zeta);
-            scale_row_sw128(sV + C * 128, v_loc, zeta);
+            const float zs = zeta * __frcp_rn(rho);  // zeta / rho
+            scale_row_sw128(sV, v_loc, zs);
+            scale_row_sw128(sV + C * 128, v_loc, zs);
           } else {
             for (int b = 0; b < 4; ++b) scale_row_sw128(sKS + b * sp.ks_box, v_loc, zeta);
           }
@@ -925,25 +962,37 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       }
       // MMA5 done; MMA14 (the reader of the old Sb) ran before it
       if (!mbar_wait(mma5done, par, abort_flag, a.lim)) break;
+      if (v_loc == 0 && !vgrp) RET_TRACE_STAMP(cta_id, it, 5);
       tc_fence_after();
       if (it < nck - 1) {
         const float gn = pw[min(C, a.L - t0 - C)];
+        // direct form: decay the state in TMEM, Sb = S.  Rescaled form: Sb = U,
+        // and U is multiplied through only when rho is reset.
+        const float rho_n = rescaled ? cw_rho_next(rho, gn) : 1.f;
+        const bool write_back = !rescaled || rho_n == 1.f;
+        const float mult = rescaled ? gn * rho : gn;
         for (int d0 = d_lo; d0 < d_lo + 128; d0 += 32) {
           uint32_t sr[32];
           tmem_ld32(tm + lane_off + TM_S + d0, sr);
           tmem_ld_wait();
           float x[32];
+          if (write_back) {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const float sv = __uint_as_float(sr[u]);
-            const float sg = gn * sv;
-            x[u] = rescaled ? sg : sv;
-            sr[u] = __float_as_uint(sg);
+            for (int u = 0; u < 32; ++u) {
+              const float sv = __uint_as_float(sr[u]);
+              const float sg = mult * sv;
+              x[u] = rescaled ? sg : sv;
+              sr[u] = __float_as_uint(sg);
+            }
+            tmem_st32(tm + lane_off + TM_S + d0, sr);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) x[u] = __uint_as_float(sr[u]);
           }
           store_row32_sw128(sSb, sp.ks_box, v_loc, d0, x);
-          tmem_st32(tm + lane_off + TM_S + d0, sr);
         }
-        tmem_st_wait();
+        rho = rho_n;
+        if (write_back) tmem_st_wait();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(sready);
@@ -955,7 +1004,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
           tmem_ld32(tm + lane_off + TM_S + d0, sr);
           tmem_ld_wait();
 #pragma unroll
-          for (int u = 0; u < 32; ++u) so[(size_t)(d0 + u) * a.dv + v] = __uint_as_float(sr[u]);
+          for (int u = 0; u < 32; ++u) so[(size_t)(d0 + u) * a.dv + v] = rho * __uint_as_float(sr[u]);
         }
       }
     }
@@ -964,12 +1013,14 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
     const int r = (int)threadIdx.x;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int row_lo = warp * 32;
+    float rho = cw_rho_first(rescaled, pw[max(min(C, a.L - c_begin * C), 0)]);
     mbar_arrive(ofree);  // X starts free
     for (int it = 0; it < nck; ++it) {
       const uint32_t par = it & 1;
       const int t0 = (c_begin + it) * C;
       const int l = min(C, a.L - t0);
       if (!mbar_wait(pxfull, par, abort_flag, a.lim)) break;
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 10);
       tc_fence_after();
       // P -> P~ in place (see the main kernel for the two forms)
       const uint32_t tp = tm + lane_off + TM_P;
@@ -1031,23 +1082,30 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 6);
       // y = (gamma^(r+1-l) in the rescaled form) X, once MMA3 is done
       if (!mbar_wait(mma3done, par, abort_flag, a.lim)) break;
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 11);
       tc_fence_after();
       {
-        const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) : 1.f;
+        // X -> registers as bf16 pairs, release X to the next block's MMA14,
+        // then the global stores.
+        const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) * rho : 1.f;
         __nv_bfloat16* wrow0 = a.y + ((size_t)bh * a.L + t0 + row_lo) * a.dv + vt * kCW_DVT;
+        uint32_t yb[4][16];
 #pragma unroll
-        for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          tmem_ld32(tm + lane_off + TM_X + c0, o);
+          tmem_ld32(tm + lane_off + TM_X + 32 * c, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(yf * __uint_as_float(o[u]));
-          store_rows_bf16_quad(wrow0 + c0, (size_t)a.dv, lane, o, 1.f, l - row_lo);
+          for (int u = 0; u < 16; ++u)
+            yb[c][u] = pack_bf16x2(yf * __uint_as_float(o[2 * u]), yf * __uint_as_float(o[2 * u + 1]));
         }
         tc_fence_before();
         mbar_arrive(ofree);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) store_rows_packed_quad(wrow0 + 32 * c, (size_t)a.dv, lane, yb[c], l - row_lo);
       }
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 7);
+      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[min(C, a.L - t0 - C)]);
     }
   }
   tc_fence_before();

@@ -92,6 +92,7 @@ def test_msr_core_chunkwise():
     (1, 1, 333, 64, 128, 48),      # C % 32 == 16
     (1, 1, 160, 128, 128, 16),     # smallest block
     (1, 2, 520, 256, 256, 32),
+    (2, 3, 700, 256, 384, 64),     # dk 256, ragged, three dv slices
 ])
 def test_chunkwise_shapes(B, H, L, dk, dv, C):
     ey, es = _chunk_case(B, H, L, dk, dv, C, with_state=True, seed=L)
@@ -104,12 +105,29 @@ def test_chunkwise_special_gammas():
     assert ey <= 2e-2 and es <= 2e-2, (ey, es)
 
 
-@pytest.mark.parametrize("C", [128, 64])
-def test_chunkwise_small_gammas_direct_form(C):
+@pytest.mark.parametrize("dk,C", [(128, 128), (128, 64), (256, 128), (256, 64)])
+def test_chunkwise_small_gammas_direct_form(dk, C):
     # gamma^(C-1) < 2^-64 takes the direct form (decay applied to P and O);
     # the other heads take the rescaled form.
-    ey, es = _chunk_case(1, 4, 300, 128, 128, C, gam=[0.5, 0.25, 0.6, 0.97], with_state=True, seed=13)
+    ey, es = _chunk_case(1, 4, 300, dk, 128, C, gam=[0.5, 0.25, 0.6, 0.97], with_state=True, seed=13)
     assert ey <= 2e-2 and es <= 2e-2, (ey, es)
+
+
+@pytest.mark.parametrize("dk,C", [(256, 128), (256, 64), (128, 128)])
+def test_chunkwise_rescaled_state_renormalisation(dk, C):
+    # gamma^(C-1) >= 2^-64 keeps these heads in the rescaled form, and the
+    # decay of the stored state runs below 2^-64 after one to a few blocks
+    # (every other block for 0.75 at C = 128), so the scaled state is
+    # multiplied through several times in one call.
+    B, H, L, dv = 1, 4, 1100, 256
+    q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed=17)
+    gam = torch.tensor([0.75, 0.9, 0.97, 1.0])
+    s_in = inputs.state(B, H, dk, dv, seed=3, scale=0.5)
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam, s_in)
+    qd, kd, vd, sd = dev(q, k, v, s_in)
+    y, s = ret.chunkwise(qd, kd, vd, gam, C, state_in=sd)
+    for h in range(H):  # per head: the gamma = 1 head would dominate a joint bound
+        assert rel(y[:, h], y_ref[:, h]) <= 2e-2 and rel(s[:, h], s_ref[:, h]) <= 2e-2, h
 
 
 def test_chunkwise_sequence_split_matches_single_pass():
