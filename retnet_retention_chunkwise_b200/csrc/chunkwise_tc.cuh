@@ -1211,10 +1211,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
     for (int it = 0; it < nck; ++it) {
       const int s = it % NS;
       if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) { ok = false; break; }
-      if ((int)r < C) {
-        const int t = (c_begin + it) * C + (int)r;
+      for (uint32_t j = r; j < (uint32_t)C; j += 128) {  // rows j and j + 128 (blocks up to 256)
+        const int t = (c_begin + it) * C + (int)j;
         const float f = (t <= seg_last) ? (t == seg_last ? 1.f : exp2f((float)(seg_last - t) * l2g)) : 0.f;
-        for (int b = 0; b < DK / 64; ++b) scale_row_sw128(sK + s * k_stage + b * C * 128, r, f);
+        for (int b = 0; b < DK / 64; ++b) scale_row_sw128(sK + s * k_stage + b * C * 128, j, f);
       }
       fence_proxy_async_smem();
       mbar_arrive(&kready[s]);

@@ -14,6 +14,7 @@
 
 #include "../../include/retention.h"
 #include "chunkwise_tc.cuh"
+#include "chunkwise_wide.cuh"
 #include "decode.cuh"
 #include "parallel_tc.cuh"
 #include "simt_f32.cuh"
@@ -125,6 +126,12 @@ bool tc_shape_ok(const ret_shape& s) {
   return (s.dk == 64 || s.dk == 128 || s.dk == 256) && (s.dv % kCW_DVT) == 0;
 }
 
+// Block lengths of the bf16 chunkwise path: multiples of 16 up to 128 for
+// every dk; up to 256 for dk <= 128 (two row halves per block).
+bool tc_chunk_ok(int chunk, int dk) {
+  return chunk >= 16 && chunk % 16 == 0 && (chunk <= 128 || (chunk <= 256 && dk <= 128));
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -166,8 +173,12 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
 
   const int smax = max_smem_optin();
   int ns = 0;
-  for (int n = kCW_MaxStages; n >= 1; --n)
-    if ((int)cw_smem_plan(DK, C, n).total <= smax) { ns = n; break; }
+  if (C <= 128) {
+    for (int n = kCW_MaxStages; n >= 1; --n)
+      if ((int)cw_smem_plan(DK, C, n).total <= smax) { ns = n; break; }
+  } else if (DK <= 128 && (int)cw_wide_smem_plan(DK, C).total <= smax) {
+    ns = 1;  // blocks of 129..256 rows: one stage, two row halves
+  }
   if (ns == 0) return RET_EUNSUPPORTED;
   CwSmem plan = cw_smem_plan(DK, C, ns);
 
@@ -235,6 +246,14 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
     chunkwise_tc256_kernel<<<grid, kCW_MainThreads, p256.total, st>>>(mq, mk, mv, a, dec);
     return launch_status();
   } else {
+    if (C > 128) {
+      const CwWideSmem pw = cw_wide_smem_plan(DK, C);
+      if (cudaFuncSetAttribute(chunkwise_wide_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)pw.total) != cudaSuccess)
+        return RET_ECUDA;
+      chunkwise_wide_kernel<DK><<<grid, kCW_MainThreads, pw.total, st>>>(mq, mk, mv, a, dec);
+      return launch_status();
+    }
     if (cudaFuncSetAttribute(chunkwise_tc_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)plan.total) != cudaSuccess)
       return RET_ECUDA;
@@ -422,7 +441,7 @@ ret_status retention_parallel(const void* q, const void* k, const void* v, const
 }
 
 size_t retention_chunkwise_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
-  if (dt != RET_BF16 || chunk < 16 || chunk > 128 || chunk % 16 != 0) return 0;
+  if (dt != RET_BF16 || !tc_chunk_ok(chunk, s.dk)) return 0;
   if (check_shape(s, true) != RET_OK || s.L < 1 || !tc_shape_ok(s)) return 0;
   int n_seg = 1, seg_chunks = 1;
   plan_segments(s, chunk, &n_seg, &seg_chunks);
@@ -444,7 +463,7 @@ ret_status retention_chunkwise(const void* q, const void* k, const void* v, cons
   if (dt == RET_F32) {
     if (chunk > kCF_MaxC || s.dk > 256) return RET_EUNSUPPORTED;
   } else {
-    if (chunk < 16 || chunk > 128 || chunk % 16 != 0) return RET_EUNSUPPORTED;
+    if (!tc_chunk_ok(chunk, s.dk)) return RET_EUNSUPPORTED;
     if (!tc_shape_ok(s)) return RET_EUNSUPPORTED;
     if (s.L > 0 && !device_is_sm100()) return RET_EUNSUPPORTED;
   }

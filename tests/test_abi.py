@@ -103,8 +103,8 @@ def test_misaligned_pointers_are_einval(lib):
                                    ctypes.c_void_p(0x10010), 1 << 20, None) == _abi.RET_EINVAL
 
 
-@pytest.mark.parametrize("chunk,dk,dv", [(8, 64, 128), (24, 64, 128), (256, 64, 128), (64, 96, 128),
-                                         (64, 64, 192), (64, 512, 128)])
+@pytest.mark.parametrize("chunk,dk,dv", [(8, 64, 128), (24, 64, 128), (272, 64, 128), (144, 256, 128),
+                                         (256, 256, 512), (64, 96, 128), (64, 64, 192), (64, 512, 128)])
 def test_unsupported_bf16_shapes(lib, chunk, dk, dv):
     s = _abi.RetShape(1, 1, 256, dk, dv)
     assert lib.retention_chunkwise(FAKE, FAKE, FAKE, _g(0.5), FAKE, None, None, chunk, s, _abi.RET_BF16,
@@ -129,3 +129,6 @@ def test_workspace_query(lib):
     n = lib.retention_chunkwise_workspace_bytes(64, few_heads, _abi.RET_BF16)
     assert n > 0 and n % (2 * 64 * 128 * 4) == 0
     assert lib.retention_chunkwise_workspace_bytes(64, few_heads, _abi.RET_F32) == 0
+    # blocks of up to 256 rows for dk <= 128; none beyond 128 for dk = 256
+    assert lib.retention_chunkwise_workspace_bytes(256, few_heads, _abi.RET_BF16) > 0
+    assert lib.retention_chunkwise_workspace_bytes(256, _abi.RetShape(1, 2, 8192, 256, 128), _abi.RET_BF16) == 0

@@ -71,7 +71,7 @@ def test_decode_6p7b_sampled_heads():
         assert rel(state[b, h], s_ref[0, 0]) <= TOL
 
 
-@pytest.mark.parametrize("C", [64, 128])
+@pytest.mark.parametrize("C", [64, 128, 256])
 def test_long_context_four_calls_match_one_call_and_oracle(C):
     w = inputs.WORKLOADS["long_context_bf16"]  # B1 H16 L65536 dk128 dv256
     q, k, v = inputs.qkv_cuda(w.B, w.H, w.L, w.dk, w.dv, w.dtype, w.seed)

@@ -93,6 +93,11 @@ def test_msr_core_chunkwise():
     (1, 1, 160, 128, 128, 16),     # smallest block
     (1, 2, 520, 256, 256, 32),
     (2, 3, 700, 256, 384, 64),     # dk 256, ragged, three dv slices
+    (1, 2, 700, 128, 256, 256),    # blocks of 256 rows (two row halves), ragged tail
+    (1, 1, 200, 64, 128, 256),     # L < C = 256: half b partly past the end
+    (1, 1, 1, 64, 128, 256),       # single token in a 256 block
+    (1, 2, 520, 128, 128, 144),    # C = 144: half b of 16 rows, C % 32 == 16
+    (2, 1, 1000, 64, 256, 240),    # C = 240
 ])
 def test_chunkwise_shapes(B, H, L, dk, dv, C):
     ey, es = _chunk_case(B, H, L, dk, dv, C, with_state=True, seed=L)
@@ -105,7 +110,7 @@ def test_chunkwise_special_gammas():
     assert ey <= 2e-2 and es <= 2e-2, (ey, es)
 
 
-@pytest.mark.parametrize("dk,C", [(128, 128), (128, 64), (256, 128), (256, 64)])
+@pytest.mark.parametrize("dk,C", [(128, 128), (128, 64), (256, 128), (256, 64), (128, 256), (64, 176)])
 def test_chunkwise_small_gammas_direct_form(dk, C):
     # gamma^(C-1) < 2^-64 takes the direct form (decay applied to P and O);
     # the other heads take the rescaled form.
@@ -113,7 +118,7 @@ def test_chunkwise_small_gammas_direct_form(dk, C):
     assert ey <= 2e-2 and es <= 2e-2, (ey, es)
 
 
-@pytest.mark.parametrize("dk,C", [(256, 128), (256, 64), (128, 128)])
+@pytest.mark.parametrize("dk,C", [(256, 128), (256, 64), (128, 128), (128, 256)])
 def test_chunkwise_rescaled_state_renormalisation(dk, C):
     # gamma^(C-1) >= 2^-64 keeps these heads in the rescaled form, and the
     # decay of the stored state runs below 2^-64 after one to a few blocks
@@ -130,8 +135,9 @@ def test_chunkwise_rescaled_state_renormalisation(dk, C):
         assert rel(y[:, h], y_ref[:, h]) <= 2e-2 and rel(s[:, h], s_ref[:, h]) <= 2e-2, h
 
 
-def test_chunkwise_sequence_split_matches_single_pass():
-    B, H, L, dk, dv, C = 1, 2, 4096, 64, 128, 64
+@pytest.mark.parametrize("dk,C", [(64, 64), (128, 256)])
+def test_chunkwise_sequence_split_matches_single_pass(dk, C):
+    B, H, L, dv = 1, 2, 4096, 128
     assert ret.workspace_bytes(C, B, H, L, dk, dv) > 0
     ey, es = _chunk_case(B, H, L, dk, dv, C, with_state=True, seed=5)
     assert ey <= 2e-2 and es <= 2e-2, (ey, es)

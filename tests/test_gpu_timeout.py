@@ -18,9 +18,9 @@ def _rel(a, b):
     return float(np.max(np.abs(a - b)) / np.max(np.abs(b)))
 
 
-@pytest.mark.parametrize("dk,dv", [(128, 128), (256, 256)])
-def test_dropped_load_times_out_then_recovers(monkeypatch, dk, dv):
-    B, H, L, C = 1, 2, 640, 128
+@pytest.mark.parametrize("dk,dv,C", [(128, 128, 128), (256, 256, 128), (128, 128, 256)])
+def test_dropped_load_times_out_then_recovers(monkeypatch, dk, dv, C):
+    B, H, L = 1, 2, 640
     q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed=31)
     gam = inputs.multiscale_gammas(H)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
