@@ -10,7 +10,7 @@ Also measured in the same run (same timing rules, reported under "forms"):
                 after a 512-token chunkwise prefill (6.7B-shaped heads);
   parallel   -- parallel form, B=2, H=8, L=2048, dk=64, dv=128 (MSR core);
   chunkwise_msr_core -- chunkwise C=64 on the same MSR-core shape;
-  long_context_C{64,128} -- B=1, H=16, L=65536, dk=128, dv=256 as four
+  long_context_C{64,128,256} -- B=1, H=16, L=65536, dk=128, dv=256 as four
                 16384-token calls with the state carried in place.
 
 Timing: CUDA events on the launching stream, >= 3 warm-up steps, barrier +
@@ -392,7 +392,7 @@ def bench_small(ret, args, dist, peaks):
     del q, k, v
     y = torch.empty_like(parts[0][2])
     state = torch.zeros((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device="cuda")
-    for C in (64, 128):
+    for C in (64, 128, 256):
         def four_calls():
             state.zero_()
             for qq, kk, vv in parts:

@@ -194,6 +194,21 @@ __device__ __forceinline__ void store_rows_packed_quad(__nv_bfloat16* row0, size
   store_rows_quad_core(row0, row_stride, lane, c, nrows);
 }
 
+// Scaled state (rescaled form): TMEM holds U, and the state decayed for the
+// coming block is rho * U.  After a block rho takes on gamma^l of the next
+// block instead of the state being multiplied in TMEM; only when rho would
+// drop below 2^-64 is U multiplied through (and rho reset to 1), so the
+// scaled operands (zeta V / rho, U) stay below 2^64 in magnitude.
+__device__ __forceinline__ float cw_rho_next(float rho, float gl) {
+  const float r = gl * rho;
+  return r < 0x1p-64f ? 1.f : r;
+}
+
+// rho for the first block of a segment (g0 = gamma^l0): 1 in the direct form.
+__device__ __forceinline__ float cw_rho_first(bool rescaled, float g0) {
+  return (rescaled && g0 >= 0x1p-64f) ? g0 : 1.f;
+}
+
 template <int DK>
 __global__ void __launch_bounds__(kCW_MainThreads, 1)
 chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
@@ -425,6 +440,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   } else if (warp >= kWarpZBase) {
     // ---------------------------------------------------- V group (4 warps)
     const uint32_t t = threadIdx.x - kWarpZBase * 32;
+    float rho = cw_rho_first(rescaled, pw[max(min(C, a.L - c_begin * C), 0)]);
     for (int it = 0; it < nck; ++it) {
       const int s = it % NS;
       if (!mbar_wait(&fullV[s], (it / NS) & 1, abort_flag, a.lim)) break;
@@ -437,9 +453,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       if (rescaled) {
         // row j of the V tile scaled in place by zeta_j = gamma^(l-1-j) (0 past the end)
         if ((int)t < C) {
-          const float zeta = ((int)t < l) ? pw[l - 1 - (int)t] : 0.f;
-          scale_row_sw128(vs, t, zeta);
-          scale_row_sw128(vs + C * 128, t, zeta);
+          const float zs = (((int)t < l) ? pw[l - 1 - (int)t] : 0.f) * __frcp_rn(rho);  // zeta / rho
+          scale_row_sw128(vs, t, zs);
+          scale_row_sw128(vs + C * 128, t, zs);
         }
         fence_proxy_async_smem();
       } else {
@@ -476,6 +492,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       }
       mbar_arrive(&zready[s]);
       if (t == 0) RET_TRACE_STAMP(cta_id, it, 3);
+      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[min(C, a.L - (c_begin + it) * C - C)]);
     }
   } else if (warp >= kWarpSBase) {
     // ---------------------------------------------------- S group (4 warps)
@@ -486,12 +503,15 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     const uint32_t lane_off = (uint32_t)((warp - kWarpSBase) * 32) << 16;
     const int v = vt * kCW_DVT + (int)v_loc;
     const size_t dkdv = (size_t)DK * a.dv;
+    const float g0 = pw[max(min(C, a.L - c_begin * C), 0)];
+    float rho = cw_rho_first(rescaled, g0);
     {
       const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
                                        : (a.state_in ? a.state_in + (size_t)bh * dkdv : nullptr);
-      const int l0 = min(C, a.L - c_begin * C);
-      const float g0 = pw[max(l0, 0)];
-      const float gc = rescaled ? g0 : 1.f;
+      // rescaled: U = S_in (or gamma^l0 S_in when rho was reset), Sb = bf16(U);
+      // direct: TMEM holds gamma^l0 S_in, Sb = S_in
+      const float gu = (rho == 1.f) ? g0 : 1.f;
+      const float gc = rescaled ? gu : 1.f;
       for (int d0 = 0; d0 < DK; d0 += 32) {
         float x[32];
         uint32_t w[32];
@@ -499,7 +519,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         for (int u = 0; u < 32; ++u) {
           const float sv = src ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
           x[u] = gc * sv;
-          w[u] = __float_as_uint(g0 * sv);
+          w[u] = __float_as_uint(gu * sv);
         }
         store_row32_sw128(sSb, 16384, v_loc, d0, x);
         tmem_st32(tm + lane_off + TM_S + d0, w);
@@ -517,22 +537,31 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       const int t0 = (c_begin + it) * C;
       if (it < nck - 1) {
         const float gn = pw[min(C, a.L - t0 - C)];
+        const float rho_n = rescaled ? cw_rho_next(rho, gn) : 1.f;
+        const bool write_back = !rescaled || rho_n == 1.f;
+        const float mult = rescaled ? gn * rho : gn;
         for (int d0 = 0; d0 < DK; d0 += 32) {
           uint32_t sr[32];
           tmem_ld32(tm + lane_off + TM_S + d0, sr);
           tmem_ld_wait();
           float x[32];
+          if (write_back) {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const float sv = __uint_as_float(sr[u]);
-            const float sg = gn * sv;
-            x[u] = rescaled ? sg : sv;
-            sr[u] = __float_as_uint(sg);
+            for (int u = 0; u < 32; ++u) {
+              const float sv = __uint_as_float(sr[u]);
+              const float sg = mult * sv;
+              x[u] = rescaled ? sg : sv;
+              sr[u] = __float_as_uint(sg);
+            }
+            tmem_st32(tm + lane_off + TM_S + d0, sr);
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) x[u] = __uint_as_float(sr[u]);
           }
           store_row32_sw128(sSb, 16384, v_loc, d0, x);
-          tmem_st32(tm + lane_off + TM_S + d0, sr);
         }
-        tmem_st_wait();
+        rho = rho_n;
+        if (write_back) tmem_st_wait();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(sready);
@@ -544,7 +573,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           tmem_ld32(tm + lane_off + TM_S + d0, sr);
           tmem_ld_wait();
 #pragma unroll
-          for (int u = 0; u < 32; ++u) so[(size_t)(d0 + u) * a.dv + v] = __uint_as_float(sr[u]);
+          for (int u = 0; u < 32; ++u) so[(size_t)(d0 + u) * a.dv + v] = rho * __uint_as_float(sr[u]);
         }
       }
     }
@@ -554,6 +583,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     const int r = (int)threadIdx.x;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int row_lo = warp * 32;  // rows of this warp: [row_lo, row_lo + 32)
+    float rho = cw_rho_first(rescaled, pw[max(min(C, a.L - c_begin * C), 0)]);
     mbar_arrive(ofree);            // O starts free
     for (int it = 0; it < nck; ++it) {
       const int pb = it % NP;
@@ -630,7 +660,8 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 9);
       tc_fence_after();
       const int s = it % NS;
-      const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) : 1.f;
+      const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) * rho : 1.f;
+      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[min(C, a.L - t0 - C)]);
       if (NS >= 2) {
         // The V tile is dead after MMA3 and its buffer is not needed again for
         // NS-1 blocks: stage y there (bf16, 128B-swizzled) for two TMA tensor
@@ -698,21 +729,6 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
 // core near its peak rate; TMEM holds S^T [0, 256) and [P | X] [256, 512).
 // Order per block: MMA14 ([P | X]; frees Q), MMA5 (state update; frees K),
 // MMA3 (X += P~ V; frees V).
-// Scaled state (rescaled form): TMEM holds U, and the state decayed for the
-// coming block is rho * U.  After a block rho takes on gamma^l of the next
-// block instead of the state being multiplied in TMEM; only when rho would
-// drop below 2^-64 is U multiplied through (and rho reset to 1), so the
-// scaled operands (zeta V / rho, U) stay below 2^64 in magnitude.
-__device__ __forceinline__ float cw_rho_next(float rho, float gl) {
-  const float r = gl * rho;
-  return r < 0x1p-64f ? 1.f : r;
-}
-
-// rho for the first block of a segment (g0 = gamma^l0): 1 in the direct form.
-__device__ __forceinline__ float cw_rho_first(bool rescaled, float g0) {
-  return (rescaled && g0 >= 0x1p-64f) ? g0 : 1.f;
-}
-
 struct Cw256Smem {
   uint32_t q, ks, v, misc, total, ks_box;
 };
