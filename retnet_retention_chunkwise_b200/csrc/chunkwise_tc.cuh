@@ -791,7 +791,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
-    mbar_init(zready, 128);
+    mbar_init(zready, 256);  // S and V groups each scale half of the tile
     mbar_init(pxfull, 1);
     mbar_init(pready, 128);
     mbar_init(mma5done, 1);
@@ -920,7 +920,8 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
     const int gbase = vgrp ? kWarpZBase : kWarpSBase;
     const uint32_t v_loc = threadIdx.x - gbase * 32;
     const uint32_t lane_off = (uint32_t)((warp - gbase) * 32) << 16;
-    const int d_lo = vgrp ? 128 : 0;
+    const int half = vgrp ? 1 : 0;
+    const int d_lo = 128 * half;
     const int v = vt * kCW_DVT + (int)v_loc;
     const size_t dkdv = (size_t)DK * a.dv;
     uint8_t* sSb = sKS + (uint32_t)C * 128u;  // first Sb row of box 0; box stride ks_box
@@ -954,9 +955,12 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
     for (int it = 0; it < nck; ++it) {
       const uint32_t par = it & 1;
       const int t0 = (c_begin + it) * C;
-      if (vgrp) {
+      {
+        // zeta (rescaled: zeta / rho) on row v_loc of V (rescaled form, as soon
+        // as V lands) or of K (direct form, once MMA14 has read it); the S group
+        // takes the first half of the row's 64-column boxes, the V group the rest.
         if (!mbar_wait(fullV, par, abort_flag, a.lim)) break;
-        if (v_loc == 0) RET_TRACE_STAMP(cta_id, it, 9);
+        if (v_loc == 0 && vgrp) RET_TRACE_STAMP(cta_id, it, 9);
         if (!rescaled) {
           if (!mbar_wait(fullK, par, abort_flag, a.lim)) break;
           if (!mbar_wait(pxfull, par, abort_flag, a.lim)) break;
@@ -965,16 +969,14 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         if ((int)v_loc < C) {
           const float zeta = ((int)v_loc < l) ? pw[l - 1 - (int)v_loc] : 0.f;
           if (rescaled) {
-            const float zs = zeta * __frcp_rn(rho);  // zeta / rho
-            scale_row_sw128(sV, v_loc, zs);
-            scale_row_sw128(sV + C * 128, v_loc, zs);
+            scale_row_sw128(sV + half * C * 128, v_loc, zeta * __frcp_rn(rho));
           } else {
-            for (int b = 0; b < 4; ++b) scale_row_sw128(sKS + b * sp.ks_box, v_loc, zeta);
+            for (int b = 2 * half; b < 2 * half + 2; ++b) scale_row_sw128(sKS + b * sp.ks_box, v_loc, zeta);
           }
         }
         fence_proxy_async_smem();
         mbar_arrive(zready);
-        if (v_loc == 0) RET_TRACE_STAMP(cta_id, it, 3);
+        if (v_loc == 0 && vgrp) RET_TRACE_STAMP(cta_id, it, 3);
       }
       // MMA5 done; MMA14 (the reader of the old Sb) ran before it
       if (!mbar_wait(mma5done, par, abort_flag, a.lim)) break;
