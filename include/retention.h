@@ -96,8 +96,9 @@ RET_API ret_status retention_parallel(const void* q, const void* k, const void* 
  *             also split across CTAs for parallelism; with less, or NULL, the
  *             call still runs, with fewer CTAs.  Results do not depend on it
  *             beyond fp32 rounding.
- * Supported: RET_F32 with 1 <= chunk <= 128, dk <= 256; RET_BF16 with chunk a
- * multiple of 16 in [16, 128], dk in {64, 128, 256}, dv a multiple of 128.
+ * Supported: RET_F32 with 1 <= chunk <= 128, dk <= 256; RET_BF16 with dk in
+ * {64, 128, 256}, dv a multiple of 128 and chunk a multiple of 16 in
+ * [16, 128], or in [16, 256] when dk <= 128.
  */
 RET_API ret_status retention_chunkwise(const void* q, const void* k, const void* v, const float* gamma,
                                void* y, const float* state_in, float* state_out, int chunk,
@@ -145,6 +146,40 @@ RET_API ret_status retention_chunkwise_static_ws(const void* q, const void* k, c
                                                  const float* gamma, void* y, const float* state_in,
                                                  float* state_out, int chunk, ret_shape s,
                                                  ret_dtype dt, void* stream);
+
+/*
+ * Chunkwise form on host buffers: q, k, v are copied from host memory, the
+ * chunkwise form runs on the device, and y is copied back to host memory, all
+ * inside this call's work on `stream` (the same results as
+ * retention_chunkwise on device copies of the inputs).  The (b, h) rows are
+ * processed in groups of consecutive heads of one batch row.  Each group's
+ * host-to-device copy, its kernels and its device-to-host copy run on
+ * separate streams, ordered by events, so the two copy directions and the
+ * kernels of different groups overlap.  This is a property of the library, not
+ * of the method.
+ * q_host, k_host, v_host, y_host : host buffers, [B][H][L][d] in the call's
+ *             dtype; page-locked memory lets the copies run asynchronously.
+ *             They must stay valid, and y_host unread, until `stream` completes.
+ * q_dev, k_dev, v_dev, y_dev : device buffers of the same sizes, owned by the
+ *             caller (the library allocates no device memory).
+ * state_in, state_out, chunk, workspace : as for retention_chunkwise (device
+ *             pointers; the workspace serves one group at a time, see the query
+ *             below).
+ * n_groups  : requested number of groups (<= 0: 8).  Groups never span batch
+ *             rows, so the call may use more.
+ * The copy streams and events are created on first use on each device and
+ * kept until the process exits.  Returns before the work completes; errors in
+ * the arguments are reported before anything is enqueued.
+ */
+RET_API ret_status retention_chunkwise_host(const void* q_host, const void* k_host, const void* v_host,
+                                            const float* gamma, void* y_host, void* q_dev, void* k_dev,
+                                            void* v_dev, void* y_dev, const float* state_in, float* state_out,
+                                            int chunk, ret_shape s, ret_dtype dt, void* workspace,
+                                            size_t workspace_bytes, int n_groups, void* stream);
+
+/* Workspace size that lets every group of retention_chunkwise_host use its full
+ * sequence split. */
+RET_API size_t retention_chunkwise_host_workspace_bytes(int chunk, ret_shape s, ret_dtype dt, int n_groups);
 
 /* Synchronises `stream`, then returns and clears the device status word:
  * RET_OK, RET_ETIMEOUT if a kernel's bounded wait expired since the last

@@ -168,6 +168,55 @@ def chunkwise(q, k, v, gamma, chunk: int, *, state_in=None, state_out=None, retu
     return y, state_out
 
 
+def chunkwise_host(q, k, v, gamma, chunk: int, *, dev=None, out=None, state_in=None, state_out=None,
+                   workspace="auto", n_groups: int = 0):
+    """Chunkwise form on host tensors: q, k, v are copied to the device, the form
+    runs there and y comes back to ``out`` (a host tensor, page-locked if it is
+    allocated here), with the copies of the two directions and the kernels of
+    successive (b, h) groups overlapped by the library (retention_chunkwise_host).
+
+    ``dev`` = (q_dev, k_dev, v_dev, y_dev) CUDA tensors of the same shapes, or
+    None to allocate them.  ``state_in`` / ``state_out`` are CUDA fp32 tensors as
+    for :func:`chunkwise`.  Returns (y_host, state_out).  The call is
+    asynchronous on the current stream: synchronise before reading y_host.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"retention: {n} must be a contiguous host tensor")
+    if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
+        raise ValueError("retention: expected q, k [B,H,L,dk] and v [B,H,L,dv]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("retention: q, k, v must share a dtype")
+    dt = _dtype(q)
+    s = _shape(q, v)
+    device = torch.device("cuda", torch.cuda.current_device())
+    if out is None:
+        out = torch.empty(v.shape, dtype=v.dtype).pin_memory()
+    if out.is_cuda or tuple(out.shape) != tuple(v.shape) or out.dtype != v.dtype or not out.is_contiguous():
+        raise ValueError("retention: out must be a contiguous host tensor shaped like v")
+    if dev is None:
+        dev = tuple(torch.empty(t.shape, dtype=t.dtype, device=device) for t in (q, k, v, v))
+    for t, h, n in zip(dev, (q, k, v, v), ("q_dev", "k_dev", "v_dev", "y_dev")):
+        _cuda(t, n)
+        if tuple(t.shape) != tuple(h.shape) or t.dtype != h.dtype:
+            raise ValueError(f"retention: {n} must match its host tensor")
+    sshape = (s.B, s.H, s.dk, s.dv)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        if t is not None:
+            _cuda(t, n)
+            if t.dtype != torch.float32 or tuple(t.shape) != sshape:
+                raise ValueError(f"retention: {n} must be fp32 {sshape}")
+    if isinstance(workspace, str):
+        workspace = _workspace(int(library().retention_chunkwise_host_workspace_bytes(chunk, s, dt, n_groups)),
+                               device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(library().retention_chunkwise_host(_ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(out),
+                                              *(_ptr(t) for t in dev), _ptr(state_in), _ptr(state_out),
+                                              int(chunk), s, dt, _ptr(workspace), wbytes, int(n_groups),
+                                              _stream()), "retention_chunkwise_host")
+    return out, state_out
+
+
 def recurrent_step(q, k, v, gamma, state, *, out=None):
     """One decode step in place on ``state``: S <- gamma S + k^T v, y = q S.
 

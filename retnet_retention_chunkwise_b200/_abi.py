@@ -26,6 +26,8 @@ EXPORTS = (
     "retention_status_str",
     "retention_abi_version",
     "retention_chunkwise_static_ws",
+    "retention_chunkwise_host",
+    "retention_chunkwise_host_workspace_bytes",
 )
 STATIC_WS_BYTES = 16 << 20  # scratch array behind retention_chunkwise_static_ws
 
@@ -53,6 +55,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.retention_abi_version.argtypes = []
     lib.retention_chunkwise_static_ws.argtypes = [vp, vp, vp, fp, vp, vp, vp, i, RetShape, i, vp]
     lib.retention_chunkwise_static_ws.restype = ctypes.c_int
+    lib.retention_chunkwise_host.argtypes = [vp, vp, vp, fp, vp, vp, vp, vp, vp, vp, vp, i, RetShape, i,
+                                             vp, sz, i, vp]
+    lib.retention_chunkwise_host.restype = ctypes.c_int
+    lib.retention_chunkwise_host_workspace_bytes.argtypes = [i, RetShape, i, i]
+    lib.retention_chunkwise_host_workspace_bytes.restype = sz
     for name in ("retention_parallel", "retention_chunkwise", "retention_recurrent_step",
                  "retention_get_device_status", "retention_abi_version"):
         getattr(lib, name).restype = ctypes.c_int

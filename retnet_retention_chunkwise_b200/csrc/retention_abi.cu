@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/retention.h"
 #include "chunkwise_tc.cuh"
@@ -299,6 +300,58 @@ ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const
 }
 
 // ---------------------------------------------------------------------------
+// Host-buffer chunkwise (retention_chunkwise_host): the (b, h) rows are cut
+// into groups of consecutive heads of one batch row; each group's copies in,
+// kernels and copy out go to three streams ordered by events.
+
+struct HostGroups {
+  int heads;    // heads per group (the last group of a batch row may have fewer)
+  int per_row;  // groups per batch row
+};
+
+HostGroups plan_host_groups(const ret_shape& s, int n_groups) {
+  if (n_groups <= 0) n_groups = 8;
+  const long long rows = (long long)s.B * s.H;
+  int hpg = (int)std::min<long long>(s.H, std::max<long long>(1, (rows + n_groups - 1) / n_groups));
+  HostGroups g;
+  g.heads = hpg;
+  g.per_row = (s.H + hpg - 1) / hpg;
+  return g;
+}
+
+// Copy streams of one device, created on first use and kept for the process.
+struct CopyStreams {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+};
+
+ret_status copy_streams(CopyStreams* out) {
+  static std::mutex mu;
+  static CopyStreams per_dev[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RET_ECUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  CopyStreams& cs = per_dev[dev];
+  if (!cs.h2d && cudaStreamCreateWithFlags(&cs.h2d, cudaStreamNonBlocking) != cudaSuccess) return RET_ECUDA;
+  if (!cs.d2h && cudaStreamCreateWithFlags(&cs.d2h, cudaStreamNonBlocking) != cudaSuccess) return RET_ECUDA;
+  *out = cs;
+  return RET_OK;
+}
+
+// A pool of timing-free events per device, grown on demand and reused.  Calls
+// on one device are serialised by the pool's lock while they enqueue, so the
+// events of one call are not re-recorded by another before this call's waits
+// are enqueued (a wait captures the event's state when it is enqueued).
+struct EventPool {
+  std::mutex mu;
+  std::vector<cudaEvent_t> ev[64];
+};
+
+EventPool& event_pool() {
+  static EventPool p;
+  return p;
+}
+
+// ---------------------------------------------------------------------------
 // Scratch for retention_chunkwise_static_ws: a fixed array in this library's
 // device memory, for callers that cannot allocate.  Its size is the most
 // sequence-split scratch that entry point accepts.  Every GPU that loads the
@@ -347,7 +400,7 @@ RET_API int retention_debug_trace(void* buf, int blocks, int events) {
 }
 #endif
 
-int retention_abi_version(void) { return 100; }
+int retention_abi_version(void) { return 101; }
 
 const char* retention_status_str(ret_status st) {
   switch (st) {
@@ -516,6 +569,105 @@ ret_status retention_chunkwise_static_ws(const void* q, const void* k, const voi
   }
   return retention_chunkwise(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, ws,
                              need > 0 ? kStaticWsBytes : 0, stream);
+}
+
+size_t retention_chunkwise_host_workspace_bytes(int chunk, ret_shape s, ret_dtype dt, int n_groups) {
+  if (check_shape(s, true) != RET_OK) return 0;
+  const HostGroups g = plan_host_groups(s, n_groups);
+  ret_shape gs = s;
+  gs.B = 1;
+  gs.H = g.heads;
+  return retention_chunkwise_workspace_bytes(chunk, gs, dt);
+}
+
+ret_status retention_chunkwise_host(const void* q_host, const void* k_host, const void* v_host,
+                                    const float* gamma, void* y_host, void* q_dev, void* k_dev, void* v_dev,
+                                    void* y_dev, const float* state_in, float* state_out, int chunk,
+                                    ret_shape s, ret_dtype dt, void* workspace, size_t workspace_bytes,
+                                    int n_groups, void* stream) {
+  ret_status rc = check_shape(s, true);
+  if (rc != RET_OK) return rc;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
+  if (chunk < 1) return RET_EINVAL;
+  if (s.L > 0 && (!q_host || !k_host || !v_host || !y_host || !q_dev || !k_dev || !v_dev || !y_dev))
+    return RET_EINVAL;
+  if (s.L == 0)  // nothing to copy: the state passes through as in retention_chunkwise
+    return retention_chunkwise(q_dev, k_dev, v_dev, gamma, y_dev, state_in, state_out, chunk, s, dt,
+                               workspace, workspace_bytes, stream);
+  // Shape support and alignment are checked once for the whole call (every
+  // group's pointers are the bases plus whole rows), so no group fails on them.
+  if (dt == RET_F32 ? (chunk > kCF_MaxC || s.dk > 256)
+                    : (!tc_chunk_ok(chunk, s.dk) || !tc_shape_ok(s) || !device_is_sm100()))
+    return RET_EUNSUPPORTED;
+  if (!aligned16(q_dev) || !aligned16(k_dev) || !aligned16(v_dev) || !aligned16(y_dev) ||
+      (state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)) ||
+      (((size_t)s.L * s.dk * (dt == RET_BF16 ? 2 : 4)) & 15u) || (((size_t)s.L * s.dv * (dt == RET_BF16 ? 2 : 4)) & 15u) ||
+      (((size_t)s.dk * s.dv * 4) & 15u))
+    return RET_EINVAL;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RET_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CopyStreams cs;
+  if ((rc = copy_streams(&cs)) != RET_OK) return rc;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RET_ECUDA;
+
+  const HostGroups g = plan_host_groups(s, n_groups);
+  const int n_total = s.B * g.per_row;
+  const size_t es = dt == RET_BF16 ? 2 : 4;
+  const size_t qk_row = (size_t)s.L * s.dk * es, v_row = (size_t)s.L * s.dv * es;
+  const size_t st_row = (size_t)s.dk * s.dv;
+
+  EventPool& pool = event_pool();
+  std::lock_guard<std::mutex> lock(pool.mu);
+  std::vector<cudaEvent_t>& ev = pool.ev[dev];
+  const size_t need = 2 * (size_t)n_total + 2;
+  while (ev.size() < need) {
+    cudaEvent_t e;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return RET_ECUDA;
+    ev.push_back(e);
+  }
+  cudaEvent_t e_start = ev[0], e_done = ev[1];
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // everything after the work already on `stream`
+  if (!ok(cudaEventRecord(e_start, st)) || !ok(cudaStreamWaitEvent(cs.h2d, e_start, 0)) ||
+      !ok(cudaStreamWaitEvent(cs.d2h, e_start, 0)))
+    return RET_ECUDA;
+  const char* qh = static_cast<const char*>(q_host);
+  const char* kh = static_cast<const char*>(k_host);
+  const char* vh = static_cast<const char*>(v_host);
+  char* yh = static_cast<char*>(y_host);
+  char* qd = static_cast<char*>(q_dev);
+  char* kd = static_cast<char*>(k_dev);
+  char* vd = static_cast<char*>(v_dev);
+  char* yd = static_cast<char*>(y_dev);
+  int gi = 0;
+  for (int b = 0; b < s.B; ++b) {
+    for (int h0 = 0; h0 < s.H; h0 += g.heads, ++gi) {
+      const int nh = std::min(g.heads, s.H - h0);
+      const size_t r0 = (size_t)b * s.H + h0;  // first (b, h) row of the group
+      cudaEvent_t e_in = ev[2 + 2 * gi], e_out = ev[3 + 2 * gi];
+      if (!ok(cudaMemcpyAsync(qd + r0 * qk_row, qh + r0 * qk_row, nh * qk_row, cudaMemcpyHostToDevice, cs.h2d)) ||
+          !ok(cudaMemcpyAsync(kd + r0 * qk_row, kh + r0 * qk_row, nh * qk_row, cudaMemcpyHostToDevice, cs.h2d)) ||
+          !ok(cudaMemcpyAsync(vd + r0 * v_row, vh + r0 * v_row, nh * v_row, cudaMemcpyHostToDevice, cs.h2d)) ||
+          !ok(cudaEventRecord(e_in, cs.h2d)) || !ok(cudaStreamWaitEvent(st, e_in, 0)))
+        return RET_ECUDA;
+      ret_shape gs = s;
+      gs.B = 1;
+      gs.H = nh;
+      rc = retention_chunkwise(qd + r0 * qk_row, kd + r0 * qk_row, vd + r0 * v_row, gamma + h0,
+                               yd + r0 * v_row, state_in ? state_in + r0 * st_row : nullptr,
+                               state_out ? state_out + r0 * st_row : nullptr, chunk, gs, dt, workspace,
+                               workspace_bytes, stream);
+      if (rc != RET_OK) return rc;
+      if (!ok(cudaEventRecord(e_out, st)) || !ok(cudaStreamWaitEvent(cs.d2h, e_out, 0)) ||
+          !ok(cudaMemcpyAsync(yh + r0 * v_row, yd + r0 * v_row, nh * v_row, cudaMemcpyDeviceToHost, cs.d2h)))
+        return RET_ECUDA;
+    }
+  }
+  // the call's work ends on `stream` once the last copy out is done
+  if (!ok(cudaEventRecord(e_done, cs.d2h)) || !ok(cudaStreamWaitEvent(st, e_done, 0))) return RET_ECUDA;
+  return RET_OK;
 }
 
 }  // extern "C"

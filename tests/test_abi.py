@@ -49,7 +49,7 @@ def test_status_strings_and_version(lib):
     names = [lib.retention_status_str(i).decode() for i in range(5)]
     assert names == ["RET_OK", "RET_EINVAL", "RET_EUNSUPPORTED", "RET_ECUDA", "RET_ETIMEOUT"]
     assert lib.retention_status_str(99).decode() == "RET_UNKNOWN"
-    assert lib.retention_abi_version() == 100
+    assert lib.retention_abi_version() == 101
 
 
 def _g(*vals):
@@ -132,3 +132,25 @@ def test_workspace_query(lib):
     # blocks of up to 256 rows for dk <= 128; none beyond 128 for dk = 256
     assert lib.retention_chunkwise_workspace_bytes(256, few_heads, _abi.RET_BF16) > 0
     assert lib.retention_chunkwise_workspace_bytes(256, _abi.RetShape(1, 2, 8192, 256, 128), _abi.RET_BF16) == 0
+
+
+def test_host_entry_validation(lib):
+    s = _abi.RetShape(1, 2, 256, 64, 128)
+    g = _g(0.5, 0.9)
+    args = lambda qh, dev: (qh, FAKE, FAKE, g, FAKE, dev, FAKE, FAKE, FAKE, None, None, 64, s,  # noqa: E731
+                            _abi.RET_BF16, None, 0, 0, None)
+    assert lib.retention_chunkwise_host(*args(None, FAKE)) == _abi.RET_EINVAL      # host q missing
+    assert lib.retention_chunkwise_host(*args(FAKE, None)) == _abi.RET_EINVAL      # device q missing
+    bad = _abi.RetShape(1, 2, 256, 96, 128)
+    assert lib.retention_chunkwise_host(FAKE, FAKE, FAKE, g, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 64, bad,
+                                        _abi.RET_BF16, None, 0, 0, None) == _abi.RET_EUNSUPPORTED
+    assert lib.retention_chunkwise_host(FAKE, FAKE, FAKE, _g(0.5, 1.5), FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+                                        64, s, _abi.RET_BF16, None, 0, 0, None) == _abi.RET_EINVAL
+
+
+def test_host_entry_workspace_query(lib):
+    # groups are 4 heads of one batch row here (8 groups over B*H = 32 rows)
+    s = _abi.RetShape(4, 8, 8192, 128, 256)
+    n = lib.retention_chunkwise_host_workspace_bytes(128, s, _abi.RET_BF16, 8)
+    assert n == lib.retention_chunkwise_workspace_bytes(128, _abi.RetShape(1, 4, 8192, 128, 256), _abi.RET_BF16)
+    assert n > 0
