@@ -12,7 +12,8 @@
 //         taking 64 of the 128 key columns)
 //   MMA3  O += P~ V_kt        (A from TMEM)
 // MMA1 of the next key tile is issued before MMA3 of this one, so the tensor
-// core works while the epilogue applies the decay.  At the end of a query
+// core works while the epilogue applies the decay; the MMA warp never waits
+// for its own MMAs to finish (they run in issue order), only for the epilogue.  At the end of a query
 // tile the epilogue reads O out to y; the second query tile's first MMA3
 // waits for that.
 //
@@ -81,7 +82,6 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
   uint64_t* full = bars;          // [4] K, V tile of a stage landed
   uint64_t* empty = bars + 4;     // [4] MMA3 done with the stage
   uint64_t* pfull = bars + 8;     // [2] MMA1 done
-  uint64_t* pfree = bars + 10;    // [2] MMA3 done with the P buffer
   uint64_t* e1done = bars + 12;   // [2] epilogue wrote P~
   uint64_t* qfull = bars + 14;    // [2] Q tile of query tile 0 / 1 landed
   uint64_t* ofull = bars + 16;    // phase t: O of query tile t complete
@@ -106,7 +106,6 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&pfull[i], 1);
-      mbar_init(&pfree[i], 1);
       mbar_init(&e1done[i], 32 * kPA_EpiWarps);
       mbar_init(&qfull[i], 1);
     }
@@ -181,7 +180,6 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
           mma_ts(tm + TM_O + t * 128, tm + TM_P + pb * 128 + (kk / 4) * 64 + (kk % 4) * 8, bd, id3,
                  (kt > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&pfree[pb]);
         mma_commit(&empty[s]);
         if (kt == qt) mma_commit(ofull);  // last key tile of this query tile
         return true;
@@ -192,7 +190,9 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         const int s = i % NS, pb = i & 1;
         if (kt == 0 && !mbar_wait(&qfull[t], 0, abort_flag, a.lim)) { ok = false; break; }
         if (!mbar_wait(&full[s], (i / NS) & 1, abort_flag, a.lim)) { ok = false; break; }
-        if (i >= 2 && !mbar_wait(&pfree[pb], ((i >> 1) - 1) & 1, abort_flag, a.lim)) { ok = false; break; }
+        // P buffer pb was last read by MMA3(i-2), issued before this MMA1 by
+        // this thread (MMAs of one thread run in order), and written by the
+        // epilogue for item i-2 before that MMA3 was issued: no wait needed.
         tc_fence_after();
         const uint32_t q_s = aQ + t * sp.q_buf, k_s = aK + s * sp.k_stage;
 #pragma unroll
