@@ -17,6 +17,9 @@ arrays.  Each C function cites the passage it follows:
   (same section), plus gamma^(n+1) q_n S_in for a carried-in state.
 * ``chunkwise``  -- the block form of the same section, derived by splitting
   the sum at each block start.
+* ``groupnorm``  -- one normalisation group per head over its dv values (author
+  responses on paperhub.cn, reply on GroupNorm vs LayerNorm), mean and biased
+  variance per (b, h, n), optional per-channel affine.
 
 Inputs are float64 numpy arrays (bf16 or fp32 values widen to fp64 exactly).
 """
@@ -64,7 +67,8 @@ def load(path: str | None = None):
     lib.oracle_recurrent.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
     lib.oracle_parallel.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
     lib.oracle_chunkwise.argtypes = [i, i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
-    for f in (lib.oracle_recurrent, lib.oracle_parallel, lib.oracle_chunkwise):
+    lib.oracle_groupnorm.argtypes = [i, i, i, i, dp, ctypes.c_double, dp, dp, dp]
+    for f in (lib.oracle_recurrent, lib.oracle_parallel, lib.oracle_chunkwise, lib.oracle_groupnorm):
         f.restype = ctypes.c_int
     if path == _LIB:
         _lib = lib
@@ -131,3 +135,19 @@ def chunkwise(q, k, v, gamma, chunk: int, state_in=None, nthreads: int = 0, lib=
 def recurrent_step(q, k, v, gamma, state, nthreads: int = 0, lib=None):
     """One decode step (q, k, v of shape [B,H,1,d]) from ``state``; returns (y, new_state)."""
     return _run("recurrent", q, k, v, gamma, state, 0, nthreads, lib)
+
+
+def groupnorm(y, eps: float = 1e-5, weight=None, bias=None, lib=None):
+    """Per-head group normalisation of y [B,H,L,dv] in fp64 (weight, bias: [H*dv] or None)."""
+    lib = lib or load()
+    y = _f64(y)
+    B, H, L, dv = y.shape
+    w = None if weight is None else _f64(weight).reshape(-1)
+    b = None if bias is None else _f64(bias).reshape(-1)
+    for t in (w, b):
+        if t is not None and t.shape[0] != H * dv:
+            raise ValueError("oracle: weight and bias must have H*dv values")
+    out = np.zeros_like(y)
+    if lib.oracle_groupnorm(B, H, L, dv, _ptr(y), float(eps), _ptr(w), _ptr(b), _ptr(out)) != 0:
+        raise ValueError("oracle_groupnorm: invalid arguments")
+    return out

@@ -238,3 +238,37 @@ int oracle_chunkwise(int B, int H, int L, int dk, int dv, int C, const double* q
                      int nthreads) {
     return run(2, B, H, L, dk, dv, C, q, k, v, gamma, state_in, y, state_out, nthreads);
 }
+
+/*
+ * Group normalisation of the retention output, one group per head.  Source:
+ * the author responses on paperhub.cn ("Retentive Network: A Successor to
+ * Transformer for Large Language Models", reply comparing GroupNorm with
+ * LayerNorm): heads carry different statistics, so each head is normalised on
+ * its own.  Readings (the page gives no formula, eps or affine): for every
+ * (b, h, n) the dv values of y_n of head h are taken as one group,
+ *     mean = (1/dv) sum_c y_c ,   var = (1/dv) sum_c (y_c - mean)^2
+ *     out_c = (y_c - mean) / sqrt(var + eps) * w[h*dv + c] + bias[h*dv + c]
+ * with w and bias optional (NULL: 1 and 0).  Two passes in fp64.
+ * Layout: y, out [B][H][L][dv]; w, bias [H*dv].  out may alias y.
+ */
+int oracle_groupnorm(int B, int H, int L, int dv, const double* y, double eps,
+                     const double* w, const double* bias, double* out) {
+    if (B < 0 || H < 1 || L < 0 || dv < 1 || !y || !out || !(eps >= 0.0)) return -1;
+    for (long r = 0; r < (long)B * H * L; ++r) {
+        const int h = (int)((r / L) % H);
+        const double* yr = y + r * dv;
+        double* o = out + r * dv;
+        double mean = 0.0;
+        for (int c = 0; c < dv; ++c) mean += yr[c];
+        mean /= dv;
+        double var = 0.0;
+        for (int c = 0; c < dv; ++c) var += (yr[c] - mean) * (yr[c] - mean);
+        var /= dv;
+        const double inv = 1.0 / sqrt(var + eps);
+        for (int c = 0; c < dv; ++c) {
+            const double z = (yr[c] - mean) * inv;
+            o[c] = z * (w ? w[(size_t)h * dv + c] : 1.0) + (bias ? bias[(size_t)h * dv + c] : 0.0);
+        }
+    }
+    return 0;
+}

@@ -183,9 +183,48 @@ def pin_linearity(lib):
     assert rel_err(y4, 3.0 * y1) <= RTOL
 
 
+def pin_groupnorm_golden(lib):
+    inp, cases = golden_io.load("groupnorm_rows.txt")
+    y = inp["y"][None, None]  # [1, 1, 2 tokens, dv 4]
+    for eps, exp in cases:
+        out = oracle.groupnorm(y, eps=eps, lib=lib)
+        assert np.allclose(out[0, 0], exp["out"], rtol=0, atol=1e-9), (eps, out[0, 0])
+
+
+def pin_groupnorm_invariants(lib):
+    rng = np.random.default_rng(5)
+    y = rng.standard_normal((2, 3, 5, 8)) * 3.0 + 1.5
+    z = oracle.groupnorm(y, eps=0.0, lib=lib)
+    # every (b, h, n) group: zero mean, unit mean square
+    assert np.allclose(z.mean(-1), 0.0, atol=1e-12)
+    assert np.allclose((z * z).mean(-1), 1.0, atol=1e-12)
+    # invariant to a positive scale and a shift of the group
+    assert np.allclose(oracle.groupnorm(2.5 * y - 7.0, eps=0.0, lib=lib), z, atol=1e-12)
+    # eps only shrinks: the mean square is var / (var + eps) < 1
+    ze = oracle.groupnorm(y, eps=0.5, lib=lib)
+    assert np.all((ze * ze).mean(-1) < 1.0) and np.allclose(ze.mean(-1), 0.0, atol=1e-12)
+
+
+def pin_groupnorm_heads(lib):
+    rng = np.random.default_rng(6)
+    y = rng.standard_normal((1, 2, 4, 6))
+    base = oracle.groupnorm(y, lib=lib)
+    y2 = y.copy()
+    y2[0, 1] *= 3.0
+    y2[0, 1, :, 0] += 1.0
+    assert np.array_equal(oracle.groupnorm(y2, lib=lib)[0, 0], base[0, 0])  # head 0 untouched
+    # per-head affine: head h uses weight[h*dv:(h+1)*dv], bias likewise
+    w = np.concatenate([np.full(6, 1.0), np.full(6, 2.0)])
+    b = np.concatenate([np.zeros(6), np.full(6, 0.25)])
+    out = oracle.groupnorm(y, weight=w, bias=b, lib=lib)
+    assert np.allclose(out[0, 0], base[0, 0], atol=1e-12)
+    assert np.allclose(out[0, 1], 2.0 * base[0, 1] + 0.25, atol=1e-12)
+
+
 ALL_PINS = [pin_three_token, pin_one_token_with_state, pin_multihead_gamma_indexing,
             pin_exact_rational, pin_gamma_one_is_unnormalised_linear_attention,
-            pin_gamma_zero_is_diagonal, pin_forms_agree, pin_split_call, pin_linearity]
+            pin_gamma_zero_is_diagonal, pin_forms_agree, pin_split_call, pin_linearity,
+            pin_groupnorm_golden, pin_groupnorm_invariants, pin_groupnorm_heads]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -242,6 +281,10 @@ MUTATIONS = [
     ("0^0 taken as 0", "if (n == 0) return 1.0;", "if (n == 0) return g;"),
     ("wrong head's gamma", "J->gamma[h]", "J->gamma[(h + 1) % J->H]"),
     ("state_out not written", "if (s_out) memcpy(s_out, S,", "if (0) memcpy(s_out, S,"),
+    ("groupnorm unbiased variance", "var /= dv;", "var /= (dv - 1);"),
+    ("groupnorm drops eps", "sqrt(var + eps)", "sqrt(var)"),
+    ("groupnorm wrong head's weight", "w[(size_t)h * dv + c]", "w[(size_t)((h + 1) % H) * dv + c]"),
+    ("groupnorm mean off by one element", "mean /= dv;", "mean /= (dv + 1);"),
 ]
 
 
