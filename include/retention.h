@@ -181,6 +181,43 @@ RET_API ret_status retention_chunkwise_host(const void* q_host, const void* k_ho
  * sequence split. */
 RET_API size_t retention_chunkwise_host_workspace_bytes(int chunk, ret_shape s, ret_dtype dt, int n_groups);
 
+/*
+ * Per-head group normalisation of a retention output (the layer that follows
+ * the contraction; author responses on paperhub.cn, "Retentive Network: A
+ * Successor to Transformer for Large Language Models", reply on GroupNorm vs
+ * LayerNorm: one group per head, since heads carry different statistics).
+ * For each (b, h, n) the dv values of y_n form one group:
+ *     out_c = (y_c - mean) / sqrt(var + eps) * weight[h*dv + c] + bias[h*dv + c]
+ * with the biased variance (the page gives no formula, eps or affine; these
+ * are the readings taken).
+ * y, out   : device [B][H][L][dv] in the call's dtype (s.dk is ignored); out may
+ *            be y.  16-byte aligned when dv % 128 == 0.
+ * weight, bias : device fp32 [H*dv], or NULL for 1 and 0.
+ * eps      : finite, >= 0.  Supported: dv <= 1024.
+ */
+RET_API ret_status retention_groupnorm(const void* y, void* out, float eps, const float* weight,
+                                       const float* bias, ret_shape s, ret_dtype dt, void* stream);
+
+/*
+ * Chunkwise form followed by retention_groupnorm on its output: y receives the
+ * normalised output.  The other arguments are as for retention_chunkwise.
+ * For bf16 with dk = 256, chunk <= 128 and dv <= 1024, the normalisation is
+ * fused into the chunkwise kernel's output epilogue.  The CTAs holding the dv
+ * slices of one head then form a thread-block cluster, and they exchange
+ * per-row statistics through a part of the workspace.  This needs
+ * retention_chunkwise_gn_workspace_bytes() of workspace; with less, or for
+ * other shapes, the normalisation runs as a second kernel on y.
+ */
+RET_API ret_status retention_chunkwise_gn(const void* q, const void* k, const void* v, const float* gamma,
+                                          void* y, const float* state_in, float* state_out, int chunk,
+                                          ret_shape s, ret_dtype dt, float eps, const float* weight,
+                                          const float* bias, void* workspace, size_t workspace_bytes,
+                                          void* stream);
+
+/* Workspace size for retention_chunkwise_gn (the sequence split plus, when the
+ * normalisation is fused, its statistics exchange). */
+RET_API size_t retention_chunkwise_gn_workspace_bytes(int chunk, ret_shape s, ret_dtype dt);
+
 /* Synchronises `stream`, then returns and clears the device status word:
  * RET_OK, RET_ETIMEOUT if a kernel's bounded wait expired since the last
  * query, or RET_ECUDA if the stream reported an error. */

@@ -217,6 +217,61 @@ def chunkwise_host(q, k, v, gamma, chunk: int, *, dev=None, out=None, state_in=N
     return out, state_out
 
 
+def _gn_params(weight, bias, H: int, dv: int, device):
+    for t, n in ((weight, "weight"), (bias, "bias")):
+        if t is not None:
+            _cuda(t, n)
+            if t.dtype != torch.float32 or t.numel() != H * dv or t.device != device:
+                raise ValueError(f"retention: {n} must be fp32 with H*dv values on the device of y")
+
+
+def groupnorm(y, eps: float = 1e-5, *, weight=None, bias=None, out=None):
+    """Per-head group normalisation of y [B,H,L,dv]: each (b, h, n) row of dv
+    values by its own mean and biased variance, then ``* weight + bias`` per
+    channel (fp32 [H*dv] CUDA tensors, optional).  ``out`` may be ``y``."""
+    _cuda(y, "y")
+    dt = _dtype(y)
+    if y.dim() != 4:
+        raise ValueError("retention: y must be [B,H,L,dv]")
+    B, H, L, dv = y.shape
+    out = out if out is not None else torch.empty_like(y)
+    _cuda(out, "out")
+    if out.shape != y.shape or out.dtype != y.dtype:
+        raise ValueError("retention: out must match y")
+    _gn_params(weight, bias, H, dv, y.device)
+    _check(library().retention_groupnorm(_ptr(y), _ptr(out), float(eps), _ptr(weight), _ptr(bias),
+                                         _abi.RetShape(B, H, L, 1, dv), dt, _stream()), "retention_groupnorm")
+    return out
+
+
+def chunkwise_groupnorm(q, k, v, gamma, chunk: int, eps: float = 1e-5, *, weight=None, bias=None,
+                        state_in=None, state_out=None, return_state=True, out=None, workspace="auto"):
+    """Chunkwise form followed by the per-head group normalisation of its output
+    (see :func:`groupnorm`), fused into the output epilogue of the dk = 256 bf16
+    kernel and run as a second kernel otherwise.  Returns (normalised y, state_out)."""
+    dt = _qkv(q, k, v)
+    s = _shape(q, v)
+    y = out if out is not None else torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    _cuda(y, "out")
+    sshape = (s.B, s.H, s.dk, s.dv)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        if t is not None:
+            _cuda(t, n)
+            if t.dtype != torch.float32 or tuple(t.shape) != sshape:
+                raise ValueError(f"retention: {n} must be fp32 {sshape}")
+    if state_out is None and return_state:
+        state_out = torch.empty(sshape, dtype=torch.float32, device=q.device)
+    _gn_params(weight, bias, s.H, s.dv, q.device)
+    if isinstance(workspace, str):
+        workspace = _workspace(int(library().retention_chunkwise_gn_workspace_bytes(chunk, s, dt)), q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(library().retention_chunkwise_gn(_ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(y),
+                                            _ptr(state_in), _ptr(state_out), int(chunk), s, dt, float(eps),
+                                            _ptr(weight), _ptr(bias), _ptr(workspace), wbytes, _stream()),
+           "retention_chunkwise_gn")
+    return y, state_out
+
+
 def recurrent_step(q, k, v, gamma, state, *, out=None):
     """One decode step in place on ``state``: S <- gamma S + k^T v, y = q S.
 

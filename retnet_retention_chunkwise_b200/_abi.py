@@ -28,6 +28,9 @@ EXPORTS = (
     "retention_chunkwise_static_ws",
     "retention_chunkwise_host",
     "retention_chunkwise_host_workspace_bytes",
+    "retention_groupnorm",
+    "retention_chunkwise_gn",
+    "retention_chunkwise_gn_workspace_bytes",
 )
 STATIC_WS_BYTES = 16 << 20  # scratch array behind retention_chunkwise_static_ws
 
@@ -60,6 +63,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.retention_chunkwise_host.restype = ctypes.c_int
     lib.retention_chunkwise_host_workspace_bytes.argtypes = [i, RetShape, i, i]
     lib.retention_chunkwise_host_workspace_bytes.restype = sz
+    f32 = ctypes.c_float
+    lib.retention_groupnorm.argtypes = [vp, vp, f32, vp, vp, RetShape, i, vp]
+    lib.retention_groupnorm.restype = ctypes.c_int
+    lib.retention_chunkwise_gn.argtypes = [vp, vp, vp, fp, vp, vp, vp, i, RetShape, i, f32, vp, vp, vp, sz, vp]
+    lib.retention_chunkwise_gn.restype = ctypes.c_int
+    lib.retention_chunkwise_gn_workspace_bytes.argtypes = [i, RetShape, i]
+    lib.retention_chunkwise_gn_workspace_bytes.restype = sz
     for name in ("retention_parallel", "retention_chunkwise", "retention_recurrent_step",
                  "retention_get_device_status", "retention_abi_version"):
         getattr(lib, name).restype = ctypes.c_int

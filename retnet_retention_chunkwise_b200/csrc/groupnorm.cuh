@@ -1,0 +1,121 @@
+// groupnorm.cuh -- per-head group normalisation of the retention output.
+//
+// One normalisation group per head (author responses on paperhub.cn,
+// "Retentive Network: A Successor to Transformer for Large Language Models",
+// reply comparing GroupNorm with LayerNorm: heads carry different statistics).
+// For each (b, h, n) the dv values of y_n are one group:
+//     out_c = (y_c - mean) / sqrt(var + eps) * w[h*dv + c] + bias[h*dv + c]
+// with the biased variance, and w, bias optional (null: 1 and 0).
+//
+// This kernel runs on a finished y (one warp per row, fp32 statistics in two
+// passes over registers).  The dk = 256 chunkwise kernel can instead fuse the
+// same normalisation into its output epilogue.
+#pragma once
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace ret {
+
+constexpr int kGN_MaxDv = 1024;
+constexpr int kGN_RowsPerBlock = 8;
+
+template <typename T>
+__device__ __forceinline__ void gn_load4(const T* p, float (&x)[4]);
+template <>
+__device__ __forceinline__ void gn_load4<float>(const float* p, float (&x)[4]) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  x[0] = v.x, x[1] = v.y, x[2] = v.z, x[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void gn_load4<__nv_bfloat16>(const __nv_bfloat16* p, float (&x)[4]) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  x[0] = __uint_as_float(v.x << 16), x[1] = __uint_as_float(v.x & 0xffff0000u);
+  x[2] = __uint_as_float(v.y << 16), x[3] = __uint_as_float(v.y & 0xffff0000u);
+}
+template <typename T>
+__device__ __forceinline__ void gn_store4(T* p, const float (&x)[4]);
+template <>
+__device__ __forceinline__ void gn_store4<float>(float* p, const float (&x)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+}
+template <>
+__device__ __forceinline__ void gn_store4<__nv_bfloat16>(__nv_bfloat16* p, const float (&x)[4]) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]), b = __floats2bfloat162_rn(x[2], x[3]);
+  uint2 v;
+  v.x = *reinterpret_cast<const uint32_t*>(&a);
+  v.y = *reinterpret_cast<const uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// One warp per (b, h, n) row.  Vectorised (4 values per lane per step) when
+// dv % 128 == 0, else one value per lane per step; dv <= 1024.  out may alias y.
+template <typename T, int VEC>
+__global__ void __launch_bounds__(32 * kGN_RowsPerBlock)
+groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, float eps,
+                      const float* __restrict__ w, const float* __restrict__ bias) {
+  constexpr int kSteps = kGN_MaxDv / (32 * VEC);
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kGN_RowsPerBlock + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int h = (int)((row / L) % H);
+  const T* yr = y + row * dv;
+  T* orow = out + row * dv;
+  float x[kSteps][VEC];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kSteps; ++i) {
+    const int c = (i * 32 + lane) * VEC;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) x[i][e] = 0.f;
+    if (c < dv) {
+      if constexpr (VEC == 4) {
+        gn_load4<T>(yr + c, x[i]);
+      } else {
+        x[i][0] = (float)yr[c];
+      }
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) s += x[i][e];
+    }
+  }
+  const float mean = warp_sum(s) / (float)dv;
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < kSteps; ++i) {
+    if ((i * 32 + lane) * VEC < dv) {
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        const float d = x[i][e] - mean;
+        q += d * d;
+      }
+    }
+  }
+  const float rstd = rsqrtf(warp_sum(q) / (float)dv + eps);
+  const float* wr = w ? w + (size_t)h * dv : nullptr;
+  const float* br = bias ? bias + (size_t)h * dv : nullptr;
+#pragma unroll
+  for (int i = 0; i < kSteps; ++i) {
+    const int c = (i * 32 + lane) * VEC;
+    if (c < dv) {
+      float z[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        z[e] = (x[i][e] - mean) * rstd;
+        if (wr) z[e] *= wr[c + e];
+        if (br) z[e] += br[c + e];
+      }
+      if constexpr (VEC == 4) {
+        gn_store4<T>(orow + c, z);
+      } else {
+        orow[c] = (T)z[0];
+      }
+    }
+  }
+}
+
+}  // namespace ret
