@@ -199,14 +199,9 @@ RET_API ret_status retention_groupnorm(const void* y, void* out, float eps, cons
                                        const float* bias, ret_shape s, ret_dtype dt, void* stream);
 
 /*
- * Chunkwise form followed by retention_groupnorm on its output: y receives the
- * normalised output.  The other arguments are as for retention_chunkwise.
- * For bf16 with dk = 256, chunk <= 128 and dv <= 1024, the normalisation is
- * fused into the chunkwise kernel's output epilogue.  The CTAs holding the dv
- * slices of one head then form a thread-block cluster, and they exchange
- * per-row statistics through a part of the workspace.  This needs
- * retention_chunkwise_gn_workspace_bytes() of workspace; with less, or for
- * other shapes, the normalisation runs as a second kernel on y.
+ * Chunkwise form followed by retention_groupnorm on its output, in place: y
+ * receives the normalised output.  The other arguments are as for
+ * retention_chunkwise; the normalisation runs as a second kernel on the stream.
  */
 RET_API ret_status retention_chunkwise_gn(const void* q, const void* k, const void* v, const float* gamma,
                                           void* y, const float* state_in, float* state_out, int chunk,
@@ -214,8 +209,7 @@ RET_API ret_status retention_chunkwise_gn(const void* q, const void* k, const vo
                                           const float* bias, void* workspace, size_t workspace_bytes,
                                           void* stream);
 
-/* Workspace size for retention_chunkwise_gn (the sequence split plus, when the
- * normalisation is fused, its statistics exchange). */
+/* Workspace size for retention_chunkwise_gn (that of the chunkwise call). */
 RET_API size_t retention_chunkwise_gn_workspace_bytes(int chunk, ret_shape s, ret_dtype dt);
 
 /* Synchronises `stream`, then returns and clears the device status word:

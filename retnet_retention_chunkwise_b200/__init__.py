@@ -247,8 +247,8 @@ def groupnorm(y, eps: float = 1e-5, *, weight=None, bias=None, out=None):
 def chunkwise_groupnorm(q, k, v, gamma, chunk: int, eps: float = 1e-5, *, weight=None, bias=None,
                         state_in=None, state_out=None, return_state=True, out=None, workspace="auto"):
     """Chunkwise form followed by the per-head group normalisation of its output
-    (see :func:`groupnorm`), fused into the output epilogue of the dk = 256 bf16
-    kernel and run as a second kernel otherwise.  Returns (normalised y, state_out)."""
+    (see :func:`groupnorm`, a second kernel on the stream).  Returns
+    (normalised y, state_out)."""
     dt = _qkv(q, k, v)
     s = _shape(q, v)
     y = out if out is not None else torch.empty(v.shape, dtype=v.dtype, device=v.device)

@@ -73,12 +73,6 @@ struct CwArgs {
   const float* seg_state;   // [BH][n_seg][dk][dv] initial states when n_seg > 1
   WaitLimit lim;
   int debug_drop_block;     // fault injection: block whose K load is never issued (-1 = none)
-  // group normalisation fused into the dk = 256 kernel (its kNorm instance)
-  int n_vt;                 // dv slices per head = CTAs per cluster
-  float gn_eps;
-  const float* gn_w;        // [H*dv] or null
-  const float* gn_b;        // [H*dv] or null
-  float2* gnx;              // [BH][n_seg][2][n_vt][128] per-row statistics exchange
 };
 
 struct CwSmem {
@@ -750,7 +744,6 @@ __host__ __device__ inline Cw256Smem cw256_smem_plan(int C) {
   return s;
 }
 
-template <bool kNorm>
 __global__ void __launch_bounds__(kCW_MainThreads, 1)
 chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                        const __grid_constant__ CUtensorMap mapV, const CwArgs a,
@@ -783,9 +776,6 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14) + 1;
   float* pw = reinterpret_cast<float*>(bars + 16);  // gamma^0 .. gamma^128
-  // group normalisation (kNorm): block parity p's per-row statistics of every
-  // dv slice of the cluster have arrived (128 arrivals per slice)
-  uint64_t* gnfull = bars + 96;    // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int vt = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;
@@ -809,10 +799,6 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
     mbar_init(mma3done, 1);
     mbar_init(ofree, 128);
     mbar_init(fin, 1);
-    if constexpr (kNorm) {
-      mbar_init(&gnfull[0], 128u * (uint32_t)a.n_vt);
-      mbar_init(&gnfull[1], 128u * (uint32_t)a.n_vt);
-    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -831,10 +817,6 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
   }
   tc_fence_before();
   __syncthreads();
-  // every CTA of the cluster has initialised its barriers before any remote arrive
-  if constexpr (kNorm) {
-    if (a.n_vt > 1) cluster_sync_all();
-  }
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
 
@@ -1126,94 +1108,17 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) * rho : 1.f;
         __nv_bfloat16* wrow0 = a.y + ((size_t)bh * a.L + t0 + row_lo) * a.dv + vt * kCW_DVT;
         uint32_t yb[4][16];
-        if constexpr (!kNorm) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tm + lane_off + TM_X + 32 * c, o);
-            tmem_ld_wait();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tm + lane_off + TM_X + 32 * c, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
-              yb[c][u] = pack_bf16x2(yf * __uint_as_float(o[2 * u]), yf * __uint_as_float(o[2 * u + 1]));
-          }
-          tc_fence_before();
-          mbar_arrive(ofree);
-        } else {
-          // Group normalisation of the row over all dv slices of the head.  Per
-          // 32-column piece: its mean m_c and the residuals y - m_c (packed bf16,
-          // small next to y, so precise).  X is then released as usual.
-          float cm[4], m2 = 0.f;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tm + lane_off + TM_X + 32 * c, o);
-            tmem_ld_wait();
-            float s = 0.f;
-#pragma unroll
-            for (int u = 0; u < 32; ++u) s += yf * __uint_as_float(o[u]);
-            const float m = s * (1.f / 32.f);
-            float q = 0.f;
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              const float d = yf * __uint_as_float(o[u]) - m;
-              q += d * d;
-            }
-#pragma unroll
-            for (int u = 0; u < 16; ++u)
-              yb[c][u] = pack_bf16x2(yf * __uint_as_float(o[2 * u]) - m, yf * __uint_as_float(o[2 * u + 1]) - m);
-            cm[c] = m;
-            m2 += q;
-          }
-          tc_fence_before();
-          mbar_arrive(ofree);
-          // this slice's (mean, sum of squared deviations) over its 128 columns
-          const float mt = 0.25f * (cm[0] + cm[1] + cm[2] + cm[3]);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) m2 += 32.f * (cm[c] - mt) * (cm[c] - mt);
-          float mean = mt, M2 = m2;
-          if (a.n_vt > 1) {
-            // publish through L2, then signal every CTA of the cluster
-            float2* slot = a.gnx + (((size_t)bh * a.n_seg + seg) * 2 + (it & 1)) * (size_t)a.n_vt * 128;
-            __stcg(slot + (size_t)vt * 128 + r, make_float2(mt, m2));
-            __threadfence();
-            __syncwarp();
-            if (lane == 0)
-              for (int p = 0; p < a.n_vt; ++p) mbar_arrive_remote(mapa_shared(smem_u32(&gnfull[it & 1]), p), 32);
-            if (!mbar_wait_cluster(&gnfull[it & 1], (it >> 1) & 1, abort_flag, a.lim)) break;
-            float2 t[8];
-            mean = 0.f;
-#pragma unroll
-            for (int p = 0; p < 8; ++p)
-              if (p < a.n_vt) {
-                t[p] = __ldcg(slot + (size_t)p * 128 + r);
-                mean += t[p].x;
-              }
-            mean /= (float)a.n_vt;
-            M2 = 0.f;
-#pragma unroll
-            for (int p = 0; p < 8; ++p)
-              if (p < a.n_vt) M2 += t[p].y + 128.f * (t[p].x - mean) * (t[p].x - mean);
-          }
-          const float rstd = rsqrtf(M2 / (float)(128 * a.n_vt) + a.gn_eps);
-          const size_t ch = (size_t)(bh % a.H) * a.dv + (size_t)vt * kCW_DVT;  // first channel of the slice
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float sh = cm[c] - mean;
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              float z0 = (bf16lo_to_f32(yb[c][u]) + sh) * rstd, z1 = (bf16hi_to_f32(yb[c][u]) + sh) * rstd;
-              if (a.gn_w) {
-                z0 *= __ldg(a.gn_w + ch + 32 * c + 2 * u);
-                z1 *= __ldg(a.gn_w + ch + 32 * c + 2 * u + 1);
-              }
-              if (a.gn_b) {
-                z0 += __ldg(a.gn_b + ch + 32 * c + 2 * u);
-                z1 += __ldg(a.gn_b + ch + 32 * c + 2 * u + 1);
-              }
-              yb[c][u] = pack_bf16x2(z0, z1);
-            }
-          }
+          for (int u = 0; u < 16; ++u)
+            yb[c][u] = pack_bf16x2(yf * __uint_as_float(o[2 * u]), yf * __uint_as_float(o[2 * u + 1]));
         }
+        tc_fence_before();
+        mbar_arrive(ofree);
 #pragma unroll
         for (int c = 0; c < 4; ++c) store_rows_packed_quad(wrow0 + 32 * c, (size_t)a.dv, lane, yb[c], l - row_lo);
       }
@@ -1223,10 +1128,6 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
   }
   tc_fence_before();
   __syncthreads();
-  // no CTA leaves while another CTA of the cluster may still arrive on its barriers
-  if constexpr (kNorm) {
-    if (a.n_vt > 1) cluster_sync_all();
-  }
   if (warp == kWarpMma) {
     __syncwarp();
     tc_fence_after();

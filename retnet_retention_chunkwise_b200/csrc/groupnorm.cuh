@@ -8,8 +8,7 @@
 // with the biased variance, and w, bias optional (null: 1 and 0).
 //
 // This kernel runs on a finished y (one warp per row, fp32 statistics in two
-// passes over registers).  The dk = 256 chunkwise kernel can instead fuse the
-// same normalisation into its output epilogue.
+// passes over registers): it reads and writes y once, so it is bound by HBM.
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -47,14 +46,35 @@ __device__ __forceinline__ void gn_store4<__nv_bfloat16>(__nv_bfloat16* p, const
   *reinterpret_cast<uint2*>(p) = v;
 }
 
+// 8 bf16 (16 bytes) at once
+__device__ __forceinline__ void gn_load8(const __nv_bfloat16* p, float (&x)[8]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void gn_store8(__nv_bfloat16* p, const float (&x)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-// One warp per (b, h, n) row.  Vectorised (4 values per lane per step) when
-// dv % 128 == 0, else one value per lane per step; dv <= 1024.  out may alias y.
+// One warp per (b, h, n) row.  Vectorised (VEC values per lane per step: 8
+// for bf16 when dv % 256 == 0, 4 when dv % 128 == 0), else one value per lane
+// per step; dv <= 1024.  out may alias y.
 template <typename T, int VEC>
 __global__ void __launch_bounds__(32 * kGN_RowsPerBlock)
 groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, float eps,
@@ -74,7 +94,9 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
 #pragma unroll
     for (int e = 0; e < VEC; ++e) x[i][e] = 0.f;
     if (c < dv) {
-      if constexpr (VEC == 4) {
+      if constexpr (VEC == 8) {
+        gn_load8(yr + c, x[i]);
+      } else if constexpr (VEC == 4) {
         gn_load4<T>(yr + c, x[i]);
       } else {
         x[i][0] = (float)yr[c];
@@ -109,7 +131,9 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
         if (wr) z[e] *= wr[c + e];
         if (br) z[e] += br[c + e];
       }
-      if constexpr (VEC == 4) {
+      if constexpr (VEC == 8) {
+        gn_store8(orow + c, z);
+      } else if constexpr (VEC == 4) {
         gn_store4<T>(orow + c, z);
       } else {
         orow[c] = (T)z[0];

@@ -159,24 +159,10 @@ size_t seg_workspace_bytes(const ret_shape& s, int n_seg) {
   return (size_t)s.B * s.H * n_seg * (size_t)s.dk * s.dv * sizeof(float);
 }
 
-// Group normalisation fused into the dk = 256 chunkwise kernel.
-struct GnCfg {
-  float eps;
-  const float* w;  // device [H*dv] or null
-  const float* b;  // device [H*dv] or null
-};
-
-size_t gn_exchange_bytes(const ret_shape& s, int n_seg) {
-  return (size_t)s.B * s.H * n_seg * 2 * (s.dv / kCW_DVT) * 128 * sizeof(float2);
-}
-
-size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
-
 template <int DK>
 ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, const float* gamma,
                                void* y, const float* state_in, float* state_out, int C,
-                               const ret_shape& s, void* ws, size_t ws_bytes, cudaStream_t st,
-                               const GnCfg* gn = nullptr) {
+                               const ret_shape& s, void* ws, size_t ws_bytes, cudaStream_t st) {
   const int BH = s.B * s.H;
   CUtensorMap mq, mk, mv, my;
   if (!make_map(&mq, q, DK, s.L, BH, C) || !make_map(&mk, k, DK, s.L, BH, C) ||
@@ -200,12 +186,7 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
 
   int n_seg = 1, seg_chunks = 0;
   plan_segments(s, C, &n_seg, &seg_chunks);
-  // with group normalisation the statistics exchange sits after the split's
-  // scratch in the workspace
-  auto ws_need = [&](int ns) {
-    return gn ? align256(seg_workspace_bytes(s, ns)) + gn_exchange_bytes(s, ns) : seg_workspace_bytes(s, ns);
-  };
-  while (n_seg > 1 && (ws == nullptr || ws_need(n_seg) > ws_bytes)) {
+  while (n_seg > 1 && (ws == nullptr || seg_workspace_bytes(s, n_seg) > ws_bytes)) {
     // not enough workspace for this split: fall back to fewer segments
     const int n_chunks = (s.L + C - 1) / C;
     int g = n_seg - 1;
@@ -232,15 +213,6 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
   a.seg_state = static_cast<const float*>(ws);
   a.lim = wait_limit();
   a.debug_drop_block = debug_drop_block();
-  a.n_vt = s.dv / kCW_DVT;
-  a.gn_eps = gn ? gn->eps : 0.f;
-  a.gn_w = gn ? gn->w : nullptr;
-  a.gn_b = gn ? gn->b : nullptr;
-  a.gnx = nullptr;
-  if (gn) {
-    if (ws == nullptr || ws_need(n_seg) > ws_bytes) return RET_EUNSUPPORTED;  // caller falls back
-    a.gnx = reinterpret_cast<float2*>(static_cast<char*>(ws) + align256(seg_workspace_bytes(s, n_seg)));
-  }
 
   if (n_seg > 1) {
     // segment sums -> workspace slots 1..n_seg-1, then the scan fills every slot
@@ -270,31 +242,10 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
     const Cw256Smem p256 = cw256_smem_plan(C);
     if ((int)p256.total > smax) return RET_EUNSUPPORTED;
     a.nstages = 1;
-    if (!gn) {
-      if (cudaFuncSetAttribute(chunkwise_tc256_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)p256.total) != cudaSuccess)
-        return RET_ECUDA;
-      chunkwise_tc256_kernel<false><<<grid, kCW_MainThreads, p256.total, st>>>(mq, mk, mv, a, dec);
-      return launch_status();
-    }
-    // the dv slices of one (b, h, segment) form a cluster for the statistics exchange
-    if (cudaFuncSetAttribute(chunkwise_tc256_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(chunkwise_tc256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)p256.total) != cudaSuccess)
       return RET_ECUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(kCW_MainThreads);
-    cfg.dynamicSmemBytes = p256.total;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)a.n_vt;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, chunkwise_tc256_kernel<true>, mq, mk, mv, a, dec) != cudaSuccess)
-      return RET_ECUDA;
+    chunkwise_tc256_kernel<<<grid, kCW_MainThreads, p256.total, st>>>(mq, mk, mv, a, dec);
     return launch_status();
   } else {
     if (C > 128) {
@@ -359,8 +310,12 @@ ret_status launch_groupnorm(const void* y, void* out, float eps, const float* w,
   if (dt == RET_BF16) {
     auto yi = static_cast<const __nv_bfloat16*>(y);
     auto yo = static_cast<__nv_bfloat16*>(out);
-    if (vec) groupnorm_rows_kernel<__nv_bfloat16, 4><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
-    else groupnorm_rows_kernel<__nv_bfloat16, 1><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
+    if (s.dv % 256 == 0)
+      groupnorm_rows_kernel<__nv_bfloat16, 8><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
+    else if (vec)
+      groupnorm_rows_kernel<__nv_bfloat16, 4><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
+    else
+      groupnorm_rows_kernel<__nv_bfloat16, 1><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
   } else {
     auto yi = static_cast<const float*>(y);
     auto yo = static_cast<float*>(out);
@@ -368,11 +323,6 @@ ret_status launch_groupnorm(const void* y, void* out, float eps, const float* w,
     else groupnorm_rows_kernel<float, 1><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
   }
   return launch_status();
-}
-
-bool gn_fusable(int chunk, const ret_shape& s, ret_dtype dt) {
-  return dt == RET_BF16 && s.dk == 256 && chunk <= 128 && tc_chunk_ok(chunk, s.dk) && tc_shape_ok(s) &&
-         s.dv / kCW_DVT <= 8;
 }
 
 // ---------------------------------------------------------------------------
@@ -761,11 +711,7 @@ ret_status retention_groupnorm(const void* y, void* out, float eps, const float*
 }
 
 size_t retention_chunkwise_gn_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
-  if (check_shape(s, true) != RET_OK || s.L < 1) return 0;
-  if (!gn_fusable(chunk, s, dt)) return retention_chunkwise_workspace_bytes(chunk, s, dt);
-  int n_seg = 1, seg_chunks = 1;
-  plan_segments(s, chunk, &n_seg, &seg_chunks);
-  return align256(seg_workspace_bytes(s, n_seg)) + gn_exchange_bytes(s, n_seg);
+  return retention_chunkwise_workspace_bytes(chunk, s, dt);
 }
 
 ret_status retention_chunkwise_gn(const void* q, const void* k, const void* v, const float* gamma, void* y,
@@ -774,22 +720,6 @@ ret_status retention_chunkwise_gn(const void* q, const void* k, const void* v, c
                                   size_t workspace_bytes, void* stream) {
   if (!(eps >= 0.f) || !std::isfinite(eps)) return RET_EINVAL;
   if (s.dv > kGN_MaxDv) return RET_EUNSUPPORTED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (s.L > 0 && gn_fusable(chunk, s, dt) && workspace &&
-      !(reinterpret_cast<uintptr_t>(workspace) & 255u)) {
-    // the same argument checks as retention_chunkwise, then the fused kernel
-    ret_status rc = check_shape(s, true);
-    if (rc != RET_OK) return rc;
-    if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
-    if (!q || !k || !v || !y) return RET_EINVAL;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y)) return RET_EINVAL;
-    if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out))) return RET_EINVAL;
-    if (!device_is_sm100()) return RET_EUNSUPPORTED;
-    const GnCfg gn{eps, weight, bias};
-    rc = launch_chunkwise_tc<256>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st,
-                                  &gn);
-    if (rc != RET_EUNSUPPORTED) return rc;  // not enough workspace for the exchange: unfused below
-  }
   ret_status rc = retention_chunkwise(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, workspace,
                                       workspace_bytes, stream);
   if (rc != RET_OK || s.L == 0) return rc;
