@@ -11,7 +11,8 @@ Also measured in the same run (same timing rules, reported under "forms"):
   parallel   -- parallel form, B=2, H=8, L=2048, dk=64, dv=128 (MSR core);
   chunkwise_msr_core -- chunkwise C=64 on the same MSR-core shape;
   long_context_C{64,128,256} -- B=1, H=16, L=65536, dk=128, dv=256 as four
-                16384-token calls with the state carried in place.
+                16384-token calls with the state carried in place;
+  groupnorm  -- per-head group normalisation of a headline-sized output.
 
 Timing: CUDA events on the launching stream, >= 3 warm-up steps, barrier +
 synchronize on both sides, max over ranks.  The headline inputs (537 MB) exceed
@@ -404,6 +405,19 @@ def bench_small(ret, args, dist, peaks):
             "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3), "ms_per_65536_tokens": round(t, 4),
             "hbm_frac": round(nb / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
             "tensor_frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+    del parts, y
+    # per-head group normalisation of a headline-sized output (268 MB, larger than L2), in place
+    w = HEADLINE
+    y = (torch.randn((w.B, w.H, w.L, w.dv), device="cuda") * 0.5).to(torch.bfloat16)
+    per, _ = time_calls(lambda: ret.groupnorm(y, 1e-5, out=y), 20, max(args.warmup, 3), dist)
+    t = dist.max(statistics.median(per))
+    nb = 2 * y.numel() * y.element_size()
+    out["groupnorm"] = {"workload": "per-head group normalisation of y: B=4 H=8 L=8192 dv=512 bf16, in place",
+                        "kernel_ms": round(t, 4), "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3),
+                        "roofline": {"bound": "hbm", "achieved": round(nb / (t * 1e-3) / 1e9, 1),
+                                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": round(nb / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                                     "algorithmic_bytes": nb, "kernel": "groupnorm_rows_kernel<bf16>"}}
     return out
 
 
