@@ -451,6 +451,16 @@ def cpu_baseline():
                       f"of the headline workload ({dt:.1f} s), tokens scaled by heads/H"}
 
 
+def headline_config(world: int) -> dict:
+    """The workload both arms report (the reference arm times a sample of it)."""
+    w = HEADLINE
+    return {"workload": "retnet1p3b_layer_bf16: chunkwise forward, C=128, fp32 state out",
+            "global_batch": w.B * world, "B_per_gpu": w.B, "H": w.H, "seq_len": w.L,
+            "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
+            "parallelism": f"dp{world}: independent (b, h) replicas, no collective",
+            "l2": "inputs 537 MB > 126 MB L2, no flush"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -468,8 +478,7 @@ def run_reference(args):
             "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "retnet1p3b_layer_bf16 (sample)", "B": w.B, "H": w.H, "L": w.L, "dk": w.dk,
-                       "dv": w.dv, "chunk": w.chunk},
+            "config": headline_config(int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
                              "sample": f"each step: fp64 recurrent oracle on {nthreads} heads x {L} positions "
                                        f"of the headline workload, tokens scaled by heads/H"},
@@ -550,11 +559,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: seeded N(0,1)/sqrt(dk) bf16 q,k,v; gamma_h = 1 - 2^(-5-h)",
-            "config": {"workload": "retnet1p3b_layer_bf16: chunkwise forward, C=128, fp32 state out",
-                       "global_batch": w.B * dist.world, "B_per_gpu": w.B, "H": w.H, "seq_len": w.L,
-                       "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
-                       "parallelism": f"dp{dist.world}: independent (b, h) replicas, no collective",
-                       "l2": "inputs 537 MB > 126 MB L2, no flush"},
+            "config": headline_config(dist.world),
             "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": head["gpu_launches"], "clocks": head["clocks"], "forms": forms}
     if dist.rank == 0:
