@@ -17,6 +17,9 @@ arrays.  Each C function cites the passage it follows:
   (same section), plus gamma^(n+1) q_n S_in for a carried-in state.
 * ``chunkwise``  -- the block form of the same section, derived by splitting
   the sum at each block start.
+* ``parallel_backward`` -- dq, dk, dv of the parallel form for an upstream dy:
+  the chain rule on each term of the definition's double sum (the pages give
+  no backward pass).
 * ``groupnorm``  -- one normalisation group per head over its dv values (author
   responses on paperhub.cn, reply on GroupNorm vs LayerNorm), mean and biased
   variance per (b, h, n), optional per-channel affine.
@@ -68,7 +71,9 @@ def load(path: str | None = None):
     lib.oracle_parallel.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
     lib.oracle_chunkwise.argtypes = [i, i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
     lib.oracle_groupnorm.argtypes = [i, i, i, i, dp, ctypes.c_double, dp, dp, dp]
-    for f in (lib.oracle_recurrent, lib.oracle_parallel, lib.oracle_chunkwise, lib.oracle_groupnorm):
+    lib.oracle_parallel_backward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp]
+    for f in (lib.oracle_recurrent, lib.oracle_parallel, lib.oracle_chunkwise, lib.oracle_groupnorm,
+              lib.oracle_parallel_backward):
         f.restype = ctypes.c_int
     if path == _LIB:
         _lib = lib
@@ -151,3 +156,21 @@ def groupnorm(y, eps: float = 1e-5, weight=None, bias=None, lib=None):
     if lib.oracle_groupnorm(B, H, L, dv, _ptr(y), float(eps), _ptr(w), _ptr(b), _ptr(out)) != 0:
         raise ValueError("oracle_groupnorm: invalid arguments")
     return out
+
+
+def parallel_backward(q, k, v, gamma, dy, lib=None):
+    """Gradients (dq, dk, dv) of the parallel form (no carried state) for upstream dy, in fp64."""
+    lib = lib or load()
+    q, k, v, dy = _f64(q), _f64(k), _f64(v), _f64(dy)
+    gamma = _f64(gamma).reshape(-1)
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L) or dy.shape != v.shape or gamma.shape[0] != H:
+        raise ValueError("oracle: shape mismatch")
+    dq = np.zeros_like(q)
+    dkk = np.zeros_like(k)
+    dvv = np.zeros_like(v)
+    if lib.oracle_parallel_backward(B, H, L, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(dy), _ptr(dq),
+                                    _ptr(dkk), _ptr(dvv)) != 0:
+        raise ValueError("oracle_parallel_backward: invalid arguments")
+    return dq, dkk, dvv

@@ -272,3 +272,43 @@ int oracle_groupnorm(int B, int H, int L, int dv, const double* y, double eps,
     }
     return 0;
 }
+
+/*
+ * Gradients of the parallel form (no carried state) for an upstream gradient
+ * dy [B][H][L][dv]: with y_n = sum_{m<=n} gamma^(n-m) (q_n . k_m) v_m (page
+ * "Retentive Networks -- Microsoft Propone l'Alternativa Architetturale ai
+ * Transformer", section "Il meccanismo: Multi-Scale Retention"), the chain
+ * rule on each term of the double sum gives, for m <= n and w = gamma^(n-m),
+ *     dq_n += w (dy_n . v_m) k_m
+ *     dk_m += w (dy_n . v_m) q_n
+ *     dv_m += w (q_n . k_m) dy_n
+ * The pages give no backward pass; this is the derivative of their definition.
+ * Outputs dq, dk [B][H][L][dk], dv [B][H][L][dv] are overwritten.
+ */
+int oracle_parallel_backward(int B, int H, int L, int dk, int dv, const double* q, const double* k,
+                             const double* v, const double* gamma, const double* dy, double* dq,
+                             double* dkk, double* dvv) {
+    if (B < 0 || H < 1 || L < 0 || dk < 1 || dv < 1 || !q || !k || !v || !gamma || !dy || !dq || !dkk || !dvv)
+        return -1;
+    memset(dq, 0, sizeof(double) * (size_t)B * H * L * dk);
+    memset(dkk, 0, sizeof(double) * (size_t)B * H * L * dk);
+    memset(dvv, 0, sizeof(double) * (size_t)B * H * L * dv);
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const size_t ok = ((size_t)b * H + h) * L * dk, ov = ((size_t)b * H + h) * L * dv;
+            const double g = gamma[h];
+            for (int n = 0; n < L; ++n)
+                for (int m = 0; m <= n; ++m) {
+                    const double w = gpow(g, n - m);
+                    double qk = 0.0, dyv = 0.0;
+                    for (int i = 0; i < dk; ++i) qk += q[ok + (size_t)n * dk + i] * k[ok + (size_t)m * dk + i];
+                    for (int j = 0; j < dv; ++j) dyv += dy[ov + (size_t)n * dv + j] * v[ov + (size_t)m * dv + j];
+                    for (int i = 0; i < dk; ++i) {
+                        dq[ok + (size_t)n * dk + i] += w * dyv * k[ok + (size_t)m * dk + i];
+                        dkk[ok + (size_t)m * dk + i] += w * dyv * q[ok + (size_t)n * dk + i];
+                    }
+                    for (int j = 0; j < dv; ++j) dvv[ov + (size_t)m * dv + j] += w * qk * dy[ov + (size_t)n * dv + j];
+                }
+        }
+    return 0;
+}

@@ -221,10 +221,45 @@ def pin_groupnorm_heads(lib):
     assert np.allclose(out[0, 1], 2.0 * base[0, 1] + 0.25, atol=1e-12)
 
 
+def pin_backward_central_differences(lib):
+    # L = sum(dy * y) is linear in each of q, k, v, so a central difference in
+    # one entry is exact up to rounding
+    rng = np.random.default_rng(9)
+    B, H, L, dk, dv = 1, 2, 6, 3, 4
+    q, k, v = (rng.standard_normal((B, H, L, d)) for d in (dk, dk, dv))
+    dy = rng.standard_normal((B, H, L, dv))
+    gam = np.array([0.8, 0.95])
+    dq, dkk, dvv = oracle.parallel_backward(q, k, v, gam, dy, lib=lib)
+
+    def loss(q_, k_, v_):
+        return float(np.sum(dy * oracle.recurrent(q_, k_, v_, gam, lib=lib)[0]))
+
+    eps = 0.5
+    for arr, grad, which in ((q, dq, 0), (k, dkk, 1), (v, dvv, 2)):
+        for idx in ((0, 0, 0, 0), (0, 1, 3, 1), (0, 1, 5, 2), (0, 0, 2, arr.shape[-1] - 1)):
+            plus, minus = [x.copy() for x in (q, k, v)], [x.copy() for x in (q, k, v)]
+            plus[which][idx] += eps
+            minus[which][idx] -= eps
+            fd = (loss(*plus) - loss(*minus)) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-9 * max(1.0, abs(fd)), (which, idx, fd, grad[idx])
+
+
+def pin_backward_gamma_zero(lib):
+    # gamma = 0 keeps only m = n: dq_n = (dy_n . v_n) k_n, dk_n = (dy_n . v_n) q_n, dv_n = (q_n . k_n) dy_n
+    rng = np.random.default_rng(10)
+    q, k = rng.standard_normal((2, 1, 2, 5, 3))
+    v, dy = rng.standard_normal((2, 1, 2, 5, 4))
+    dq, dkk, dvv = oracle.parallel_backward(q, k, v, np.zeros(2), dy, lib=lib)
+    dyv = np.einsum("bhnj,bhnj->bhn", dy, v)[..., None]
+    qk = np.einsum("bhni,bhni->bhn", q, k)[..., None]
+    assert np.allclose(dq, dyv * k) and np.allclose(dkk, dyv * q) and np.allclose(dvv, qk * dy)
+
+
 ALL_PINS = [pin_three_token, pin_one_token_with_state, pin_multihead_gamma_indexing,
             pin_exact_rational, pin_gamma_one_is_unnormalised_linear_attention,
             pin_gamma_zero_is_diagonal, pin_forms_agree, pin_split_call, pin_linearity,
-            pin_groupnorm_golden, pin_groupnorm_invariants, pin_groupnorm_heads]
+            pin_groupnorm_golden, pin_groupnorm_invariants, pin_groupnorm_heads,
+            pin_backward_central_differences, pin_backward_gamma_zero]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -285,6 +320,12 @@ MUTATIONS = [
     ("groupnorm drops eps", "sqrt(var + eps)", "sqrt(var)"),
     ("groupnorm wrong head's weight", "w[(size_t)h * dv + c]", "w[(size_t)((h + 1) % H) * dv + c]"),
     ("groupnorm mean off by one element", "mean /= dv;", "mean /= (dv + 1);"),
+    ("backward dq uses q for k", "+= w * dyv * k[ok + (size_t)m * dk + i];", "+= w * dyv * q[ok + (size_t)m * dk + i];"),
+    ("backward dk from the wrong row", "dkk[ok + (size_t)m * dk + i] += w * dyv * q[ok + (size_t)n * dk + i];",
+     "dkk[ok + (size_t)m * dk + i] += w * dyv * q[ok + (size_t)m * dk + i];"),
+    ("backward dv drops the decay", "dvv[ov + (size_t)m * dv + j] += w * qk", "dvv[ov + (size_t)m * dv + j] += qk"),
+    ("backward misses the diagonal", "                for (int m = 0; m <= n; ++m) {\n                    const double w = gpow(g, n - m);",
+     "                for (int m = 0; m < n; ++m) {\n                    const double w = gpow(g, n - m);"),
 ]
 
 
