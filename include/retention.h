@@ -76,7 +76,7 @@ typedef struct {
  * it is Eq. (5) / Fig. 2a in the paperhub.cn author responses (reply on why the
  * two forms of Fig. 2 are equivalent).  No state in or out.
  * Supported: RET_F32 with dk <= 256; RET_BF16 with dk in {64, 128, 256} and
- * dv a multiple of 128.  Pointers must be 16-byte aligned.
+ * dv a multiple of 64.  Pointers must be 16-byte aligned.
  */
 RET_API ret_status retention_parallel(const void* q, const void* k, const void* v, const float* gamma,
                               void* y, ret_shape s, ret_dtype dt, void* stream);
@@ -211,6 +211,30 @@ RET_API ret_status retention_chunkwise_gn(const void* q, const void* k, const vo
 
 /* Workspace size for retention_chunkwise_gn (that of the chunkwise call). */
 RET_API size_t retention_chunkwise_gn_workspace_bytes(int chunk, ret_shape s, ret_dtype dt);
+
+/*
+ * Backward pass of retention_parallel: for the upstream gradient dy of
+ * y = retention_parallel(q, k, v), writes
+ *     dq_n = sum_{m<=n} gamma^(n-m) (dy_n . v_m) k_m
+ *     dk_m = sum_{n>=m} gamma^(n-m) (dy_n . v_m) q_n
+ *     dv_m = sum_{n>=m} gamma^(n-m) (q_n . k_m) dy_n
+ * (the derivative of the retention sum of the page "Retentive Networks --
+ * Microsoft ...", section "Il meccanismo"; the pages give no backward pass).
+ * Each is a retention sum itself: dq on (dy, v, k), and dk, dv on the
+ * time-reversed sequences; the call runs three parallel-form launches and the
+ * reversals on `stream`.
+ * q, k, dq, dk : device [B][H][L][dk]; v, dy, dv : device [B][H][L][dv]; all in
+ *             the call's dtype, 16-byte aligned.
+ * workspace : device scratch of retention_parallel_backward_workspace_bytes()
+ *             bytes, 256-byte aligned (reversed inputs and results).
+ * Supported: bf16 with dk and dv in {64, 128, 256}; fp32 with dk, dv <= 256.
+ */
+RET_API ret_status retention_parallel_backward(const void* q, const void* k, const void* v, const float* gamma,
+                                               const void* dy, void* dq, void* dk, void* dv, ret_shape s,
+                                               ret_dtype dt, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace size of retention_parallel_backward. */
+RET_API size_t retention_parallel_backward_workspace_bytes(ret_shape s, ret_dtype dt);
 
 /* Synchronises `stream`, then returns and clears the device status word:
  * RET_OK, RET_ETIMEOUT if a kernel's bounded wait expired since the last

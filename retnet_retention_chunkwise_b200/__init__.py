@@ -272,6 +272,26 @@ def chunkwise_groupnorm(q, k, v, gamma, chunk: int, eps: float = 1e-5, *, weight
     return y, state_out
 
 
+def parallel_backward(q, k, v, gamma, dy, *, workspace=None):
+    """Gradients (dq, dk, dv) of :func:`parallel` for the upstream gradient dy
+    (retention_parallel_backward).  ``workspace``: a CUDA tensor of at least
+    ``retention_parallel_backward_workspace_bytes`` bytes, or None to allocate."""
+    dt = _qkv(q, k, v)
+    _cuda(dy, "dy")
+    if dy.shape != v.shape or dy.dtype != v.dtype:
+        raise ValueError("retention: dy must match v")
+    s = _shape(q, v)
+    need = int(library().retention_parallel_backward_workspace_bytes(s, dt))
+    if workspace is None:
+        workspace = torch.empty((need + 3) // 4, dtype=torch.float32, device=q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    _check(library().retention_parallel_backward(_ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(dy),
+                                                 _ptr(dq), _ptr(dk), _ptr(dv), s, dt, _ptr(workspace), wbytes,
+                                                 _stream()), "retention_parallel_backward")
+    return dq, dk, dv
+
+
 def recurrent_step(q, k, v, gamma, state, *, out=None):
     """One decode step in place on ``state``: S <- gamma S + k^T v, y = q S.
 

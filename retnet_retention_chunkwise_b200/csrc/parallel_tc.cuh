@@ -3,7 +3,8 @@
 // y = (Q K^T (.) D) V with D_nm = gamma^(n-m) for m <= n, 0 above the diagonal
 // (page "Retentive Networks -- Microsoft ...", section "Il meccanismo", parallel
 // form; Eq. (5) / Fig. 2a of the paperhub.cn author responses).  The score
-// matrix never reaches HBM.  One CTA owns (b, h, a 128-column dv slice) and a
+// matrix never reaches HBM.  One CTA owns (b, h, a DVT-column dv slice, DVT = 128,
+// or 64 for dv not a multiple of 128) and a
 // PAIR of 128-row query tiles, the heaviest with the lightest (qa = n-1-y and
 // qb = y), so every CTA walks about the same number of causal key tiles and
 // the grid fits in one wave.  For every (query tile, key tile kt <= qt):
@@ -48,11 +49,11 @@ struct PaSmem {
 };
 
 // Two Q buffers (one per query tile of the pair), NS stages of K and V tiles.
-__host__ __device__ inline PaSmem pa_smem_plan(int DK, int ns) {
+__host__ __device__ inline PaSmem pa_smem_plan(int DK, int DVT, int ns) {
   PaSmem s;
   s.q_buf = (uint32_t)(DK / 64) * 16384u;
   s.k_stage = (uint32_t)(DK / 64) * 16384u;
-  s.v_stage = 2u * 16384u;
+  s.v_stage = (uint32_t)(DVT / 64) * 16384u;
   s.q = 0;
   s.k = s.q + 2u * s.q_buf;
   s.v = s.k + (uint32_t)ns * s.k_stage;
@@ -61,12 +62,13 @@ __host__ __device__ inline PaSmem pa_smem_plan(int DK, int ns) {
   return s;
 }
 
-template <int DK>
+template <int DK, int DVT>
 __global__ void __launch_bounds__(kPA_Threads, 1)
 parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, const PaArgs a,
                    const __grid_constant__ CwDecay dec) {
   static_assert(DK == 64 || DK == 128 || DK == 256, "dk must be 64, 128 or 256");
+  static_assert(DVT == 64 || DVT == 128, "dv slice of 64 or 128 columns");
   // TMEM: two P buffers [0, 256), one O accumulator per query tile of the pair
   // [256, 512), so the second tile's MMAs never wait for the first tile's read-out.
   constexpr uint32_t TM_P = 0, TM_O = 256, kTmemCols = 512;
@@ -74,7 +76,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align_smem(smem_raw);
   const int NS = a.nstages;
-  const PaSmem sp = pa_smem_plan(DK, NS);
+  const PaSmem sp = pa_smem_plan(DK, DVT, NS);
   uint8_t* sQ = base + sp.q;
   uint8_t* sK = base + sp.k;
   uint8_t* sV = base + sp.v;
@@ -140,7 +142,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         for (int b = 0; b < DK / 64; ++b)
           tma_load_3d(sQ + t * sp.q_buf + b * 16384, &mapQ, &qfull[t], b * 64, (t ? qt1 : qt0) * 128, bh);
       }
-      const uint32_t bytes = (uint32_t)(DK + 128) * 128u * 2u;
+      const uint32_t bytes = (uint32_t)(DK + DVT) * 128u * 2u;
       int issued = 0;
       for (int i = 0; i < nitems; ++i) {
         int t, qt, kt;
@@ -150,8 +152,8 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         mbar_arrive_expect_tx(&full[s], bytes);
         for (int b = 0; b < DK / 64; ++b)
           tma_load_3d(sK + s * sp.k_stage + b * 16384, &mapK, &full[s], b * 64, kt * 128, bh);
-        for (int b = 0; b < 2; ++b)
-          tma_load_3d(sV + s * sp.v_stage + b * 16384, &mapV, &full[s], vt * 128 + b * 64, kt * 128, bh);
+        for (int b = 0; b < DVT / 64; ++b)
+          tma_load_3d(sV + s * sp.v_stage + b * 16384, &mapV, &full[s], vt * DVT + b * 64, kt * 128, bh);
         issued = i + 1;
       }
       for (int t = 0; t < ntile; ++t) mbar_drain(&qfull[t], 0, a.lim);
@@ -160,7 +162,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
   } else if (warp == kPA_WarpMma) {
     if (lane == 0) {
       const uint32_t id1 = idesc_bf16(128, 128, false, false);
-      const uint32_t id3 = idesc_bf16(128, 128, false, true);
+      const uint32_t id3 = idesc_bf16(128, DVT, false, true);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       bool ok = true;
       // O[t] += P~[i] V[i]; the first key tile of a query tile starts O[t]
@@ -270,14 +272,15 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
       tc_fence_before();
       mbar_arrive(&e1done[pb]);
       if (kt == qt) {
-        // query tile complete: O[t] -> y (this warp: its 32 rows, columns cbase .. cbase+63)
+        // query tile complete: O[t] -> y (this warp: its 32 rows, DVT/2 of the columns)
         if (!mbar_wait(ofull, t, abort_flag, a.lim)) { ok = false; break; }
         tc_fence_after();
         const int row0 = qt * 128 + row_lo;
-        __nv_bfloat16* wrow0 = a.y + ((size_t)bh * a.L + row0) * a.dv + vt * 128 + cbase;
-        for (int c0 = 0; c0 < 64; c0 += 32) {
+        const int obase = (warp >> 2) * (DVT / 2);
+        __nv_bfloat16* wrow0 = a.y + ((size_t)bh * a.L + row0) * a.dv + vt * DVT + obase;
+        for (int c0 = 0; c0 < DVT / 2; c0 += 32) {
           uint32_t o[32];
-          tmem_ld32(tm + lane_off + TM_O + t * 128 + cbase + c0, o);
+          tmem_ld32(tm + lane_off + TM_O + t * 128 + obase + c0, o);
           tmem_ld_wait();
           store_rows_bf16_quad(wrow0 + c0, (size_t)a.dv, lane, o, 1.f, a.L - row0);
         }

@@ -17,6 +17,7 @@
 #include "chunkwise_tc.cuh"
 #include "chunkwise_wide.cuh"
 #include "groupnorm.cuh"
+#include "backward.cuh"
 #include "decode.cuh"
 #include "parallel_tc.cuh"
 #include "simt_f32.cuh"
@@ -126,6 +127,11 @@ ret_status launch_status() { return cudaGetLastError() == cudaSuccess ? RET_OK :
 
 bool tc_shape_ok(const ret_shape& s) {
   return (s.dk == 64 || s.dk == 128 || s.dk == 256) && (s.dv % kCW_DVT) == 0;
+}
+
+// Shapes of the bf16 parallel path: dk in {64, 128, 256}, dv a multiple of 64.
+bool parallel_tc_shape_ok(const ret_shape& s) {
+  return (s.dk == 64 || s.dk == 128 || s.dk == 256) && s.dv % 64 == 0;
 }
 
 // Block lengths of the bf16 chunkwise path: multiples of 16 up to 128 for
@@ -264,7 +270,7 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
   }
 }
 
-template <int DK>
+template <int DK, int DVT>
 ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const float* gamma, void* y,
                               const ret_shape& s, cudaStream_t st) {
   const int BH = s.B * s.H;
@@ -279,9 +285,9 @@ ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const
   const int smax = max_smem_optin();
   int ns = 0;
   for (int n = kCW_MaxStages; n >= 1; --n)
-    if ((int)pa_smem_plan(DK, n).total <= smax) { ns = n; break; }
+    if ((int)pa_smem_plan(DK, DVT, n).total <= smax) { ns = n; break; }
   if (ns == 0) return RET_EUNSUPPORTED;
-  const PaSmem plan = pa_smem_plan(DK, ns);
+  const PaSmem plan = pa_smem_plan(DK, DVT, ns);
   PaArgs a;
   a.B = s.B;
   a.H = s.H;
@@ -291,12 +297,12 @@ ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const
   a.nstages = ns;
   a.y = static_cast<__nv_bfloat16*>(y);
   a.lim = wait_limit();
-  if (cudaFuncSetAttribute(parallel_tc_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(parallel_tc_kernel<DK, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)plan.total) != cudaSuccess)
     return RET_ECUDA;
   // blockIdx.y = y pairs query tiles n_qt-1-y and y (one tile when they meet)
-  dim3 grid(s.dv / 128, (a.n_qt + 1) / 2, BH);
-  parallel_tc_kernel<DK><<<grid, kPA_Threads, plan.total, st>>>(mq, mk, mv, a, dec);
+  dim3 grid(s.dv / DVT, (a.n_qt + 1) / 2, BH);
+  parallel_tc_kernel<DK, DVT><<<grid, kPA_Threads, plan.total, st>>>(mq, mk, mv, a, dec);
   return launch_status();
 }
 
@@ -323,6 +329,43 @@ ret_status launch_groupnorm(const void* y, void* out, float eps, const float* w,
     else groupnorm_rows_kernel<float, 1><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
   }
   return launch_status();
+}
+
+// Reverse the sequence axis of a [BH][L][d] tensor (d * es bytes per row).
+ret_status launch_reverse(const void* in, void* out, long long BH, int L, int d, size_t es, cudaStream_t st) {
+  const size_t row = (size_t)d * es;
+  const long long rows = BH * L;
+  if (rows == 0) return RET_OK;
+  auto grid = [&](long long units) {
+    return (unsigned)std::min<long long>((units + 255) / 256, 8LL * sm_count());
+  };
+  if (row % 16 == 0) {
+    const int u = (int)(row / 16);
+    reverse_rows_kernel<uint4><<<grid(rows * u), 256, 0, st>>>(static_cast<const uint4*>(in), static_cast<uint4*>(out),
+                                                               BH, L, u);
+  } else if (row % 4 == 0) {
+    const int u = (int)(row / 4);
+    reverse_rows_kernel<uint32_t><<<grid(rows * u), 256, 0, st>>>(static_cast<const uint32_t*>(in),
+                                                                  static_cast<uint32_t*>(out), BH, L, u);
+  } else {
+    const int u = (int)(row / 2);
+    reverse_rows_kernel<uint16_t><<<grid(rows * u), 256, 0, st>>>(static_cast<const uint16_t*>(in),
+                                                                  static_cast<uint16_t*>(out), BH, L, u);
+  }
+  return launch_status();
+}
+
+// Workspace of the parallel backward pass: reversed q, k, v, dy and the two
+// reversed results, each region 256-byte aligned.
+size_t parallel_backward_ws(const ret_shape& s, size_t es, size_t* off) {
+  const size_t nk = (size_t)s.B * s.H * s.L * s.dk * es, nv = (size_t)s.B * s.H * s.L * s.dv * es;
+  const size_t sz[6] = {nk, nk, nv, nv, nk, nv};  // Rq, Rk, Rv, Rdy, T (-> dk), T2 (-> dv)
+  size_t o = 0;
+  for (int i = 0; i < 6; ++i) {
+    if (off) off[i] = o;
+    o += (sz[i] + 255) & ~size_t(255);
+  }
+  return o;
 }
 
 // ---------------------------------------------------------------------------
@@ -511,11 +554,15 @@ ret_status retention_parallel(const void* q, const void* k, const void* v, const
     return launch_status();
   }
   if (dt != RET_BF16) return RET_EINVAL;
-  if (!tc_shape_ok(s) || !device_is_sm100()) return RET_EUNSUPPORTED;
+  if (!parallel_tc_shape_ok(s) || !device_is_sm100()) return RET_EUNSUPPORTED;
+  const bool wide = s.dv % 128 == 0;  // 128-column dv slices, else 64
   switch (s.dk) {
-    case 64: return launch_parallel_tc<64>(q, k, v, gamma, y, s, st);
-    case 128: return launch_parallel_tc<128>(q, k, v, gamma, y, s, st);
-    default: return launch_parallel_tc<256>(q, k, v, gamma, y, s, st);
+    case 64: return wide ? launch_parallel_tc<64, 128>(q, k, v, gamma, y, s, st)
+                         : launch_parallel_tc<64, 64>(q, k, v, gamma, y, s, st);
+    case 128: return wide ? launch_parallel_tc<128, 128>(q, k, v, gamma, y, s, st)
+                          : launch_parallel_tc<128, 64>(q, k, v, gamma, y, s, st);
+    default: return wide ? launch_parallel_tc<256, 128>(q, k, v, gamma, y, s, st)
+                         : launch_parallel_tc<256, 64>(q, k, v, gamma, y, s, st);
   }
 }
 
@@ -724,6 +771,53 @@ ret_status retention_chunkwise_gn(const void* q, const void* k, const void* v, c
                                       workspace_bytes, stream);
   if (rc != RET_OK || s.L == 0) return rc;
   return retention_groupnorm(y, y, eps, weight, bias, s, dt, stream);
+}
+
+size_t retention_parallel_backward_workspace_bytes(ret_shape s, ret_dtype dt) {
+  if (check_shape(s, true) != RET_OK || (dt != RET_F32 && dt != RET_BF16)) return 0;
+  return parallel_backward_ws(s, dt == RET_BF16 ? 2 : 4, nullptr);
+}
+
+ret_status retention_parallel_backward(const void* q, const void* k, const void* v, const float* gamma,
+                                       const void* dy, void* dq, void* dk, void* dv, ret_shape s, ret_dtype dt,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  ret_status rc = check_shape(s, true);
+  if (rc != RET_OK) return rc;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
+  if (s.L == 0) return RET_OK;
+  if (!q || !k || !v || !dy || !dq || !dk || !dv) return RET_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return RET_EINVAL;
+  // the three forward calls take (dy, v, k), (Rv, Rdy, Rq) and (Rk, Rq, Rdy):
+  // both dk and dv play the role of the key width
+  if (dt == RET_BF16) {
+    const ret_shape a{s.B, s.H, s.L, s.dv, s.dk}, b{s.B, s.H, s.L, s.dk, s.dv};
+    if (!parallel_tc_shape_ok(a) || !parallel_tc_shape_ok(b) || !device_is_sm100()) return RET_EUNSUPPORTED;
+  } else if (s.dk > 256 || s.dv > 256) {
+    return RET_EUNSUPPORTED;
+  }
+  const size_t es = dt == RET_BF16 ? 2 : 4;
+  size_t off[6];
+  const size_t need = parallel_backward_ws(s, es, off);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RET_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(workspace);
+  void *rq = w + off[0], *rk = w + off[1], *rv = w + off[2], *rdy = w + off[3], *t1 = w + off[4], *t2 = w + off[5];
+  const long long BH = (long long)s.B * s.H;
+  const ret_shape swapped{s.B, s.H, s.L, s.dv, s.dk};  // key width dv, value width dk
+  // dq = retention(dy, v, k)
+  if ((rc = retention_parallel(dy, v, k, gamma, dq, swapped, dt, stream)) != RET_OK) return rc;
+  if ((rc = launch_reverse(q, rq, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
+  if ((rc = launch_reverse(k, rk, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
+  if ((rc = launch_reverse(v, rv, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
+  if ((rc = launch_reverse(dy, rdy, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
+  // dk = R(retention(Rv, Rdy, Rq)),  dv = R(retention(Rk, Rq, Rdy))
+  if ((rc = retention_parallel(rv, rdy, rq, gamma, t1, swapped, dt, stream)) != RET_OK) return rc;
+  if ((rc = launch_reverse(t1, dk, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
+  if ((rc = retention_parallel(rk, rq, rdy, gamma, t2, s, dt, stream)) != RET_OK) return rc;
+  return launch_reverse(t2, dv, BH, s.L, s.dv, es, st);
 }
 
 }  // extern "C"

@@ -154,3 +154,17 @@ def test_host_entry_workspace_query(lib):
     n = lib.retention_chunkwise_host_workspace_bytes(128, s, _abi.RET_BF16, 8)
     assert n == lib.retention_chunkwise_workspace_bytes(128, _abi.RetShape(1, 4, 8192, 128, 256), _abi.RET_BF16)
     assert n > 0
+
+
+def test_parallel_backward_validation(lib):
+    s = _abi.RetShape(1, 2, 64, 64, 128)
+    g = _g(0.5, 0.9)
+    need = lib.retention_parallel_backward_workspace_bytes(s, _abi.RET_F32)
+    assert need >= 3 * 64 * 64 * 4 * 2 + 3 * 64 * 128 * 4 * 2  # reversed q, k, v, dy and two results
+    call = lambda ws, nbytes, dt=_abi.RET_F32, shape=s, dy=FAKE: lib.retention_parallel_backward(  # noqa: E731
+        FAKE, FAKE, FAKE, g, dy, FAKE, FAKE, FAKE, shape, dt, ws, nbytes, None)
+    assert call(None, 0) == _abi.RET_EINVAL                      # no workspace
+    assert call(ctypes.c_void_p(0x100000), need - 1) == _abi.RET_EINVAL  # too small
+    assert call(ctypes.c_void_p(0x100000), need, dy=None) == _abi.RET_EINVAL
+    assert call(ctypes.c_void_p(0x100000), need, _abi.RET_BF16,
+                _abi.RetShape(1, 2, 64, 96, 128)) == _abi.RET_EUNSUPPORTED

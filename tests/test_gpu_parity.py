@@ -4,6 +4,8 @@ Metric (per tensor): max |gpu - oracle| / max |oracle|.  Bounds: 1e-4 for fp32
 inputs, 2e-2 for bf16 inputs (fp32 accumulation and state).  Both sides read the
 same seeded bytes; the oracle widens them to fp64 exactly.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -283,3 +285,34 @@ def test_chunkwise_groupnorm(B, H, L, dk, dv, C):
     # the same as the two calls in sequence
     y2, _ = ret.chunkwise(qd, kd, vd, gam, C, state_in=sd)
     assert torch.equal(ret.groupnorm(y2, 1e-5, weight=w.cuda(), bias=b.cuda()), z)
+
+
+@pytest.mark.parametrize("B,H,L,dk,dv", [(1, 2, 300, 128, 64), (2, 1, 1000, 64, 192)])
+def test_parallel_64_column_slices(B, H, L, dk, dv):
+    q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed=dv + L)
+    gam = inputs.multiscale_gammas(H)
+    y_ref, _ = oracle.recurrent(q, k, v, gam)
+    qd, kd, vd = dev(q, k, v)
+    assert rel(ret.parallel(qd, kd, vd, gam), y_ref) <= 2e-2
+
+
+# ------------------------------------------------ backward of the parallel form
+@pytest.mark.parametrize("dt,B,H,L,dk,dv", [
+    (torch.bfloat16, 2, 4, 300, 64, 128),
+    (torch.bfloat16, 1, 2, 1000, 128, 64),
+    (torch.bfloat16, 1, 3, 257, 64, 64),
+    (torch.bfloat16, 1, 2, 520, 128, 256),
+    (torch.float32, 1, 2, 70, 32, 48),
+])
+def test_parallel_backward(dt, B, H, L, dk, dv):
+    q, k, v = inputs.qkv(B, H, L, dk, dv, dt, seed=L + dk)
+    g = torch.Generator("cpu").manual_seed(L)
+    dy = (torch.randn((B, H, L, dv), generator=g) / math.sqrt(dv)).to(dt)
+    gam = inputs.multiscale_gammas(H) if H != 3 else torch.tensor([0.0, 1.0, 0.9])
+    dq_r, dk_r, dv_r = oracle.parallel_backward(q, k, v, gam, dy)
+    qd, kd, vd, dyd = dev(q, k, v, dy)
+    dq, dkk, dvv = ret.parallel_backward(qd, kd, vd, gam, dyd)
+    assert ret.device_status() == 0
+    tol = 1e-4 if dt == torch.float32 else 2e-2
+    errs = (rel(dq, dq_r), rel(dkk, dk_r), rel(dvv, dv_r))
+    assert max(errs) <= tol, errs
