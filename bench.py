@@ -9,6 +9,7 @@ Also measured in the same run (same timing rules, reported under "forms"):
   decode     -- 1024 recurrent steps, B=64, H=16, dk=256, dv=512, fp32 state
                 after a 512-token chunkwise prefill (6.7B-shaped heads);
   parallel   -- parallel form, B=2, H=8, L=2048, dk=64, dv=128 (MSR core);
+  parallel_backward -- its gradients dq, dk, dv on the same shape;
   chunkwise_msr_core -- chunkwise C=64 on the same MSR-core shape;
   long_context_C{64,128,256} -- B=1, H=16, L=65536, dk=128, dv=256 as four
                 16384-token calls with the state carried in place;
@@ -358,6 +359,11 @@ def bench_decode(ret, args, dist, peaks):
             "gpu_launches": steps}
 
 
+def _shape_of(w):
+    from retnet_retention_chunkwise_b200 import _abi
+    return _abi.RetShape(w.B, w.H, w.L, w.dk, w.dv)
+
+
 def bench_small(ret, args, dist, peaks):
     out = {}
     w = inputs.WORKLOADS["msr_core_bf16"]
@@ -374,6 +380,19 @@ def bench_small(ret, args, dist, peaks):
                                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                     "frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
                                     "algorithmic_flops": fl, "kernel": "parallel_tc_kernel<64>"}}
+    dy = torch.randn_like(v) / math.sqrt(w.dv)
+    ws = torch.empty(int(ret.library().retention_parallel_backward_workspace_bytes(
+        _shape_of(w), 1)) // 4 + 64, dtype=torch.float32, device="cuda")
+    per, _ = time_calls(lambda: ret.parallel_backward(q, k, v, gam, dy, workspace=ws), n, max(args.warmup, 3),
+                        dist, flush=True)
+    t = dist.max(statistics.median(per))
+    out["parallel_backward"] = {"workload": "msr_core: B=2 H=8 L=2048 dk=64 dv=128, dq dk dv for an upstream dy "
+                                            "(L2 flushed per call)",
+                                "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3), "call_ms": round(t, 4),
+                                "tensor": {"achieved_tflops": round(3 * fl / (t * 1e-3) / 1e12, 1),
+                                           "frac": round(3 * fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                                           "algorithmic_flops": 3 * fl}}
+    del dy, ws
     per, _ = time_calls(lambda: ret.chunkwise(q, k, v, gam, w.chunk, out=y, return_state=False), n,
                         max(args.warmup, 3), dist, flush=True)
     t = dist.max(statistics.median(per))
