@@ -316,3 +316,35 @@ def test_parallel_backward(dt, B, H, L, dk, dv):
     tol = 1e-4 if dt == torch.float32 else 2e-2
     errs = (rel(dq, dq_r), rel(dkk, dk_r), rel(dvv, dv_r))
     assert max(errs) <= tol, errs
+
+
+# ------------------------------------------------------------- guard bands
+def _guarded(shape, dtype, fill):
+    """A tensor of `shape` at the start of a larger buffer whose tail (64 KB)
+    holds `fill`; returns (tensor, tail)."""
+    n = int(np.prod(shape))
+    pad = 65536 // torch.tensor([], dtype=dtype).element_size()
+    buf = torch.full((n + pad,), fill, dtype=dtype, device="cuda")
+    return buf[:n].view(shape), buf[n:]
+
+
+@pytest.mark.parametrize("B,H,L,dk,dv,C", [(1, 2, 333, 64, 128, 64), (1, 1, 200, 128, 256, 256),
+                                          (1, 2, 150, 256, 128, 128), (2, 1, 77, 128, 128, 16)])
+def test_outputs_stay_inside_their_buffers(B, H, L, dk, dv, C):
+    q, k, v = dev(*inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed=3))
+    gam = inputs.multiscale_gammas(H)
+    y, y_tail = _guarded((B, H, L, dv), torch.bfloat16, 7.0)
+    s, s_tail = _guarded((B, H, dk, dv), torch.float32, 7.0)
+    ret.chunkwise(q, k, v, gam, C, state_out=s, out=y)
+    yp, yp_tail = _guarded((B, H, L, dv), torch.bfloat16, 7.0)
+    ret.parallel(q, k, v, gam, out=yp)
+    yd, yd_tail = _guarded((B, H, 1, dv), torch.bfloat16, 7.0)
+    st = torch.zeros((B, H, dk, dv), dtype=torch.float32, device="cuda")
+    ret.recurrent_step(q[:, :, :1].contiguous(), k[:, :, :1].contiguous(), v[:, :, :1].contiguous(), gam, st, out=yd)
+    z, z_tail = _guarded((B, H, L, dv), torch.bfloat16, 7.0)
+    ret.groupnorm(yp, 1e-5, out=z)
+    torch.cuda.synchronize()
+    assert ret.device_status() == 0
+    for name, tail in (("chunkwise y", y_tail), ("state", s_tail), ("parallel y", yp_tail),
+                       ("decode y", yd_tail), ("groupnorm", z_tail)):
+        assert bool((tail == 7.0).all()), f"{name}: write past the end of the output"
