@@ -100,6 +100,9 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
   const int nk0 = qt0 + 1;
   const int nitems = nk0 + (ntile == 2 ? qt1 + 1 : 0);
   const float l2g = dec.l2g[bh % a.H];
+  const int cta_id = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  (void)cta_id;
+  RET_TRACE_INIT();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) {
@@ -149,6 +152,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         item(i, t, qt, kt);
         const int s = i % NS;
         if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, i, 0);
         mbar_arrive_expect_tx(&full[s], bytes);
         for (int b = 0; b < DK / 64; ++b)
           tma_load_3d(sK + s * sp.k_stage + b * 16384, &mapK, &full[s], b * 64, kt * 128, bh);
@@ -174,6 +178,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         item(i, t, qt, kt);
         const int s = i % NS, pb = i & 1;
         if (!mbar_wait(&e1done[pb], (i >> 1) & 1, abort_flag, a.lim)) return false;
+        RET_TRACE_STAMP(cta_id, i, 2);
         tc_fence_after();
         const uint32_t v_s = aV + s * sp.v_stage;
 #pragma unroll
@@ -192,6 +197,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         const int s = i % NS, pb = i & 1;
         if (kt == 0 && !mbar_wait(&qfull[t], 0, abort_flag, a.lim)) { ok = false; break; }
         if (!mbar_wait(&full[s], (i / NS) & 1, abort_flag, a.lim)) { ok = false; break; }
+        RET_TRACE_STAMP(cta_id, i, 1);
         // P buffer pb was last read by MMA3(i-2), issued before this MMA1 by
         // this thread (MMAs of one thread run in order), and written by the
         // epilogue for item i-2 before that MMA3 was issued: no wait needed.
@@ -236,6 +242,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
       item(i, t, qt, kt);
       const int pb = i & 1;
       if (!mbar_wait(&pfull[pb], (i >> 1) & 1, abort_flag, a.lim)) { ok = false; break; }
+      if (threadIdx.x == 0) RET_TRACE_STAMP(cta_id, i, 3);
       tc_fence_after();
       const uint32_t tp = tm + lane_off + TM_P + pb * 128;
       const bool diag = (kt == qt);
@@ -271,6 +278,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&e1done[pb]);
+      if (threadIdx.x == 0) RET_TRACE_STAMP(cta_id, i, 4);
       if (kt == qt) {
         // query tile complete: O[t] -> y (this warp: its 32 rows, DVT/2 of the columns)
         if (!mbar_wait(ofull, t, abort_flag, a.lim)) { ok = false; break; }
@@ -284,6 +292,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
           tmem_ld_wait();
           store_rows_bf16_quad(wrow0 + c0, (size_t)a.dv, lane, o, 1.f, a.L - row0);
         }
+        if (threadIdx.x == 0) RET_TRACE_STAMP(cta_id, i, 5);
       }
     }
     (void)ok;
