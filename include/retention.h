@@ -236,6 +236,26 @@ RET_API ret_status retention_parallel_backward(const void* q, const void* k, con
 /* Workspace size of retention_parallel_backward. */
 RET_API size_t retention_parallel_backward_workspace_bytes(ret_shape s, ret_dtype dt);
 
+/*
+ * The same gradients through the chunkwise form (blocks of `chunk`, zero
+ * initial state): the three retention sums of retention_parallel_backward
+ * computed by retention_chunkwise, so the cost grows linearly with L.  No
+ * state gradient: the forward call it differentiates starts from a zero state
+ * and its state_out is not used.
+ * Supported: bf16 with dk and dv in {128, 256} (each is the value width of one
+ * of the three calls) and a chunk the chunkwise path takes for both; fp32 with
+ * dk, dv <= 256 and chunk <= 128.  Workspace: the reversal buffers plus the
+ * chunkwise calls' sequence-split scratch,
+ * retention_chunkwise_backward_workspace_bytes() bytes, 256-byte aligned.
+ */
+RET_API ret_status retention_chunkwise_backward(const void* q, const void* k, const void* v, const float* gamma,
+                                                const void* dy, void* dq, void* dk, void* dv, int chunk, ret_shape s,
+                                                ret_dtype dt, void* workspace, size_t workspace_bytes,
+                                                void* stream);
+
+/* Workspace size of retention_chunkwise_backward. */
+RET_API size_t retention_chunkwise_backward_workspace_bytes(int chunk, ret_shape s, ret_dtype dt);
+
 /* Synchronises `stream`, then returns and clears the device status word:
  * RET_OK, RET_ETIMEOUT if a kernel's bounded wait expired since the last
  * query, or RET_ECUDA if the stream reported an error. */

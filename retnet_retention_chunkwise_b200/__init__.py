@@ -292,6 +292,26 @@ def parallel_backward(q, k, v, gamma, dy, *, workspace=None):
     return dq, dk, dv
 
 
+def chunkwise_backward(q, k, v, gamma, dy, chunk: int, *, workspace=None):
+    """Gradients (dq, dk, dv) of :func:`chunkwise` from a zero state, for the
+    upstream gradient dy of y, through the chunkwise form (cost linear in L;
+    retention_chunkwise_backward)."""
+    dt = _qkv(q, k, v)
+    _cuda(dy, "dy")
+    if dy.shape != v.shape or dy.dtype != v.dtype:
+        raise ValueError("retention: dy must match v")
+    s = _shape(q, v)
+    need = int(library().retention_chunkwise_backward_workspace_bytes(int(chunk), s, dt))
+    if workspace is None:
+        workspace = torch.empty((need + 3) // 4, dtype=torch.float32, device=q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    _check(library().retention_chunkwise_backward(_ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(dy),
+                                                  _ptr(dq), _ptr(dk), _ptr(dv), int(chunk), s, dt, _ptr(workspace),
+                                                  wbytes, _stream()), "retention_chunkwise_backward")
+    return dq, dk, dv
+
+
 def recurrent_step(q, k, v, gamma, state, *, out=None):
     """One decode step in place on ``state``: S <- gamma S + k^T v, y = q S.
 

@@ -33,6 +33,8 @@ EXPORTS = (
     "retention_chunkwise_gn_workspace_bytes",
     "retention_parallel_backward",
     "retention_parallel_backward_workspace_bytes",
+    "retention_chunkwise_backward",
+    "retention_chunkwise_backward_workspace_bytes",
 )
 STATIC_WS_BYTES = 16 << 20  # scratch array behind retention_chunkwise_static_ws
 
@@ -76,6 +78,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.retention_parallel_backward.restype = ctypes.c_int
     lib.retention_parallel_backward_workspace_bytes.argtypes = [RetShape, i]
     lib.retention_parallel_backward_workspace_bytes.restype = sz
+    lib.retention_chunkwise_backward.argtypes = [vp, vp, vp, fp, vp, vp, vp, vp, i, RetShape, i, vp, sz, vp]
+    lib.retention_chunkwise_backward.restype = ctypes.c_int
+    lib.retention_chunkwise_backward_workspace_bytes.argtypes = [i, RetShape, i]
+    lib.retention_chunkwise_backward_workspace_bytes.restype = sz
     for name in ("retention_parallel", "retention_chunkwise", "retention_recurrent_step",
                  "retention_get_device_status", "retention_abi_version"):
         getattr(lib, name).restype = ctypes.c_int

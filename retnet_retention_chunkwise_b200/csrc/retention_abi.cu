@@ -820,4 +820,68 @@ ret_status retention_parallel_backward(const void* q, const void* k, const void*
   return launch_reverse(t2, dv, BH, s.L, s.dv, es, st);
 }
 
+// Chunkwise variant: the same three retention sums through the chunkwise form
+// (zero initial state), after the reversal buffers the workspace holds the
+// scratch of the largest of the three chunkwise calls.
+size_t chunkwise_backward_split_ws(int chunk, const ret_shape& s, ret_dtype dt) {
+  const ret_shape swapped{s.B, s.H, s.L, s.dv, s.dk};
+  return std::max(retention_chunkwise_workspace_bytes(chunk, swapped, dt),
+                  retention_chunkwise_workspace_bytes(chunk, s, dt));
+}
+
+size_t retention_chunkwise_backward_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
+  if (check_shape(s, true) != RET_OK || (dt != RET_F32 && dt != RET_BF16)) return 0;
+  return parallel_backward_ws(s, dt == RET_BF16 ? 2 : 4, nullptr) + chunkwise_backward_split_ws(chunk, s, dt);
+}
+
+ret_status retention_chunkwise_backward(const void* q, const void* k, const void* v, const float* gamma,
+                                        const void* dy, void* dq, void* dk, void* dv, int chunk, ret_shape s,
+                                        ret_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+  ret_status rc = check_shape(s, true);
+  if (rc != RET_OK) return rc;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
+  if (chunk < 1) return RET_EINVAL;
+  if (s.L == 0) return RET_OK;
+  if (!q || !k || !v || !dy || !dq || !dk || !dv) return RET_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return RET_EINVAL;
+  const ret_shape swapped{s.B, s.H, s.L, s.dv, s.dk};  // key width dv, value width dk
+  if (dt == RET_BF16) {
+    if (!tc_shape_ok(s) || !tc_shape_ok(swapped) || !tc_chunk_ok(chunk, s.dk) || !tc_chunk_ok(chunk, s.dv) ||
+        !device_is_sm100())
+      return RET_EUNSUPPORTED;
+  } else if (s.dk > 256 || s.dv > 256 || chunk > kCF_MaxC) {
+    return RET_EUNSUPPORTED;
+  }
+  const size_t es = dt == RET_BF16 ? 2 : 4;
+  size_t off[6];
+  const size_t rev = parallel_backward_ws(s, es, off);
+  const size_t split = chunkwise_backward_split_ws(chunk, s, dt);
+  if (!workspace || workspace_bytes < rev + split || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return RET_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(workspace);
+  void *rq = w + off[0], *rk = w + off[1], *rv = w + off[2], *rdy = w + off[3], *t1 = w + off[4], *t2 = w + off[5];
+  void* sw = split ? w + rev : nullptr;
+  const long long BH = (long long)s.B * s.H;
+  // dq = retention(dy, v, k)
+  if ((rc = retention_chunkwise(dy, v, k, gamma, dq, nullptr, nullptr, chunk, swapped, dt, sw, split, stream)) !=
+      RET_OK)
+    return rc;
+  if ((rc = launch_reverse(q, rq, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
+  if ((rc = launch_reverse(k, rk, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
+  if ((rc = launch_reverse(v, rv, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
+  if ((rc = launch_reverse(dy, rdy, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
+  // dk = R(retention(Rv, Rdy, Rq)),  dv = R(retention(Rk, Rq, Rdy))
+  if ((rc = retention_chunkwise(rv, rdy, rq, gamma, t1, nullptr, nullptr, chunk, swapped, dt, sw, split, stream)) !=
+      RET_OK)
+    return rc;
+  if ((rc = launch_reverse(t1, dk, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
+  if ((rc = retention_chunkwise(rk, rq, rdy, gamma, t2, nullptr, nullptr, chunk, s, dt, sw, split, stream)) != RET_OK)
+    return rc;
+  return launch_reverse(t2, dv, BH, s.L, s.dv, es, st);
+}
+
 }  // extern "C"

@@ -348,3 +348,24 @@ def test_outputs_stay_inside_their_buffers(B, H, L, dk, dv, C):
     for name, tail in (("chunkwise y", y_tail), ("state", s_tail), ("parallel y", yp_tail),
                        ("decode y", yd_tail), ("groupnorm", z_tail)):
         assert bool((tail == 7.0).all()), f"{name}: write past the end of the output"
+
+
+@pytest.mark.parametrize("dt,B,H,L,dk,dv,C", [
+    (torch.bfloat16, 1, 2, 700, 128, 256, 128),
+    (torch.bfloat16, 1, 2, 1000, 256, 128, 64),
+    (torch.bfloat16, 1, 1, 600, 128, 128, 256),    # 256-row blocks
+    (torch.bfloat16, 1, 2, 4096, 128, 128, 128),   # sequence split in all three calls
+    (torch.float32, 1, 2, 70, 32, 48, 16),
+])
+def test_chunkwise_backward(dt, B, H, L, dk, dv, C):
+    q, k, v = inputs.qkv(B, H, L, dk, dv, dt, seed=L + C)
+    g = torch.Generator("cpu").manual_seed(L + 1)
+    dy = (torch.randn((B, H, L, dv), generator=g) / math.sqrt(dv)).to(dt)
+    gam = inputs.multiscale_gammas(H)
+    dq_r, dk_r, dv_r = oracle.parallel_backward(q, k, v, gam, dy)
+    qd, kd, vd, dyd = dev(q, k, v, dy)
+    dq, dkk, dvv = ret.chunkwise_backward(qd, kd, vd, gam, dyd, C)
+    assert ret.device_status() == 0
+    tol = 1e-4 if dt == torch.float32 else 2e-2
+    errs = (rel(dq, dq_r), rel(dkk, dk_r), rel(dvv, dv_r))
+    assert max(errs) <= tol, errs
