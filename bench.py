@@ -10,6 +10,8 @@ Also measured in the same run (same timing rules, reported under "forms"):
                 after a 512-token chunkwise prefill (6.7B-shaped heads);
   parallel   -- parallel form, B=2, H=8, L=2048, dk=64, dv=128 (MSR core);
   parallel_backward -- its gradients dq, dk, dv on the same shape;
+  chunkwise_backward_long_context -- the gradients through the chunkwise form,
+                one 16384-token call of the long-context layout;
   chunkwise_msr_core -- chunkwise C=64 on the same MSR-core shape;
   long_context_C{64,128,256} -- B=1, H=16, L=65536, dk=128, dv=256 as four
                 16384-token calls with the state carried in place;
@@ -424,7 +426,17 @@ def bench_small(ret, args, dist, peaks):
             "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3), "ms_per_65536_tokens": round(t, 4),
             "hbm_frac": round(nb / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
             "tensor_frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
-    del parts, y
+    # backward through the chunkwise form, one 16384-token call of the same layout
+    qq, kk, vv = parts[0]
+    dy = torch.randn_like(vv) / math.sqrt(w.dv)
+    per, _ = time_calls(lambda: ret.chunkwise_backward(qq, kk, vv, gam, dy, 128), 10, max(args.warmup, 3), dist)
+    t = dist.max(statistics.median(per))
+    fl = 3 * w.B * w.H * seg * chunk_flops_per_head_token(128, w.dk, w.dv)
+    out["chunkwise_backward_long_context"] = {
+        "workload": "long_context layout, one 16384-token call: dq dk dv through the chunkwise form, C=128",
+        "tokens_per_s": dist.sum(w.B * seg) / (t * 1e-3), "call_ms": round(t, 4),
+        "tensor_frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+    del parts, y, dy
     # per-head group normalisation of a headline-sized output (268 MB, larger than L2), in place
     w = HEADLINE
     y = (torch.randn((w.B, w.H, w.L, w.dv), device="cuda") * 0.5).to(torch.bfloat16)
