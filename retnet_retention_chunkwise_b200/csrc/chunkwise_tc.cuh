@@ -8,31 +8,41 @@
 //   S   = gamma^l S_prev + K_c^T diag(zeta) V_c        xi_i = gamma^(i+1), zeta_j = gamma^(l-1-j)
 //
 // One CTA owns (b, h, a 128-column slice of dv, a run of consecutive blocks)
-// and walks its blocks in order with the fp32 state slice resident in TMEM.
-// Warp roles (192 threads):
-//   warps 0-3  epilogue: TMEM lane r = thread r (0..127).  Turns P into the
-//              decayed bf16 P~ in place, scales rows of K_c by zeta, scales O
-//              by xi, keeps the state (rescale by gamma^l, bf16 copy for the
-//              next block's Q S term), writes y.
-//   warp 4     TMA producer: Q_c, K_c and the V_c slice per block, NS stages.
-//   warp 5     TMEM allocator; lane 0 issues every tcgen05.mma.
-// Per block the MMA warp issues, in order,
-//   MMA1  P[pb] = Q K^T            A = Q  (smem, K-major)   B = K  (smem, K-major)
-//   MMA4  O     = Q Sb             A = Q  (smem, K-major)   B = Sb (smem, K-major; bf16 S^T)
-//   MMA3  O    += P~ V             A = P~ (TMEM, bf16)      B = V  (smem, MN-major)
-//   MMA5  S^T  += V^T (zeta K)     A = V  (smem, MN-major)  B = zeta K (smem, MN-major)
-// with xi applied to O between MMA4 and MMA3 (a TMEM read-modify-write), so the
-// cross-block and intra-block terms share one accumulator.  The state is held
-// transposed (lanes = the 128 dv columns, columns = dk) so MMA5 has M = 128
-// for every dk.
+// and walks its blocks in order with the fp32 state slice resident in TMEM,
+// held transposed (lanes = the 128 dv columns, columns = dk) so the state
+// update has M = 128 for every dk.  Warp roles (448 threads, both kernels):
+//   warps 0-3    P/O group: TMEM lane r = row r of the block.  P -> P~ in place
+//                (bf16 pairs), xi on O in the direct form, y out.
+//   warps 4-7    S group: the state copy Sb for the next block's cross term
+//                (and the state rescale when it is due), state_out.
+//   warps 8-11   V group: zeta on the rows of V (rescaled form) or of K, or
+//                (zeta V)^T in TMEM (direct form); in the dk = 256 kernel it
+//                also keeps half of the state.
+//   warp 12      TMA producer: Q, K, V of each block on their own barriers.
+//   warp 13      TMEM allocator; lane 0 issues every tcgen05.mma.
 //
-// TMEM columns: S^T [0, DK), P buffers [DK, DK + 128*NP), O [DK + 128*NP, +128).
-// DK = 256 fits one P buffer (512 columns in all); DK <= 128 double-buffers P.
+// Two forms of the decay (chosen per head, uniform over the CTA):
+//   rescaled (gamma^(C-1) >= 2^-64): V scaled by zeta_j / rho, P~ = P masked
+//     to j <= i, y_i = gamma^(i+1-l) rho O_i.  The state is kept scaled: TMEM
+//     holds U with the decayed state rho U, and U is multiplied through only
+//     when rho would drop below 2^-64 (cw_rho_next).
+//   direct (smaller gamma): P~_ij = P_ij gamma^(i-j), O scaled by xi after the
+//     cross term, the state decayed by gamma^l in TMEM each block.
+//
+// chunkwise_tc_kernel<DK> (DK 64, 128; NS = 2..4 stages, P double-buffered):
+//   MMA1  P[pb] = Q K^T            A = Q  (smem, K-major)   B = K  (smem, K-major)
+//   MMA5  S^T  += (zeta V)^T K     A = V  (smem, MN-major, or TMEM)  B = K (smem, MN-major)
+//   MMA4  O     = Q Sb             A = Q  (smem, K-major)   B = Sb (smem, K-major)
+//   MMA3  O    += P~ V             A = P~ (TMEM, bf16)      B = V  (smem, MN-major)
+//   TMEM: S^T [0, DK), P buffers [DK, DK + 256), O [DK + 256, DK + 384).
+// chunkwise_tc256_kernel (DK = 256, one stage): the scores and the cross term
+// in one N = C + 128 MMA, [P | X] = Q [K ; Sb]^T, then the state update and
+// P~ V (see there).
 //
 // Decay factors come from a per-CTA table pw[n] = gamma^n, n = 0..128 (exp2 of
 // n*log2(gamma), gamma^0 = 1): the intra-block mask uses pw[i-j], xi = pw[i+1],
-// zeta = pw[l-1-j], the state rescale pw[l].  No negative exponent appears, so
-// small gamma underflows to 0 instead of overflowing.
+// zeta = pw[l-1-j], the state decay pw[l].  Only the y factor of the rescaled
+// form has a negative exponent, bounded by the same 2^-64 test.
 //
 // Long sequences with few (b, h) are split into segments run by separate CTAs:
 // chunk_state_kernel computes each segment's decayed K^T V sum, state_scan_kernel
