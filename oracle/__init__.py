@@ -72,8 +72,9 @@ def load(path: str | None = None):
     lib.oracle_chunkwise.argtypes = [i, i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, i]
     lib.oracle_groupnorm.argtypes = [i, i, i, i, dp, ctypes.c_double, dp, dp, dp]
     lib.oracle_parallel_backward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp]
+    lib.oracle_state_backward.argtypes = [i, i, i, i, i] + [dp] * 11
     for f in (lib.oracle_recurrent, lib.oracle_parallel, lib.oracle_chunkwise, lib.oracle_groupnorm,
-              lib.oracle_parallel_backward):
+              lib.oracle_parallel_backward, lib.oracle_state_backward):
         f.restype = ctypes.c_int
     if path == _LIB:
         _lib = lib
@@ -174,3 +175,28 @@ def parallel_backward(q, k, v, gamma, dy, lib=None):
                                     _ptr(dkk), _ptr(dvv)) != 0:
         raise ValueError("oracle_parallel_backward: invalid arguments")
     return dq, dkk, dvv
+
+
+def backward(q, k, v, gamma, dy, state_in=None, dstate_out=None, lib=None):
+    """Gradients (dq, dk, dv, dstate_in) of y and state_out with respect to q,
+    k, v and state_in, for upstream dy and dstate_out (None: zero), in fp64.
+
+    The terms without state come from oracle_parallel_backward, the terms of
+    the carried state from oracle_state_backward."""
+    lib = lib or load()
+    dq, dkk, dvv = parallel_backward(q, k, v, gamma, dy, lib=lib)
+    q, k, v, dy = _f64(q), _f64(k), _f64(v), _f64(dy)
+    gamma = _f64(gamma).reshape(-1)
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    s0 = None if state_in is None else _f64(state_in)
+    dso = None if dstate_out is None else _f64(dstate_out)
+    for t in (s0, dso):
+        if t is not None and t.shape != (B, H, dk, dv):
+            raise ValueError("oracle: state shape mismatch")
+    ds0 = np.zeros((B, H, dk, dv))
+    if lib.oracle_state_backward(B, H, L, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(dy),
+                                 _ptr(s0), _ptr(dso),
+                                 _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(ds0)) != 0:
+        raise ValueError("oracle_state_backward: invalid arguments")
+    return dq, dkk, dvv, ds0

@@ -312,3 +312,53 @@ int oracle_parallel_backward(int B, int H, int L, int dk, int dv, const double* 
         }
     return 0;
 }
+
+/*
+ * The terms a carried state adds to the gradients.  With state_in S0 and
+ * state_out S_out (same page and section: the recurrence S_n = gamma S_{n-1} +
+ * k_n^T v_n started from S0), unrolling gives
+ *     y_n   gains  gamma^(n+1) q_n S0
+ *     S_out =      gamma^L S0 + sum_m gamma^(L-1-m) k_m^T v_m
+ * and for upstream gradients dy [B][H][L][dv] and dS_out [B][H][dk][dv]:
+ *     dq_n  += gamma^(n+1) dy_n S0^T
+ *     dk_m  += gamma^(L-1-m) v_m dS_out^T
+ *     dv_m  += gamma^(L-1-m) k_m dS_out
+ *     dS0    = gamma^L dS_out + sum_n gamma^(n+1) q_n^T dy_n
+ * s0 or dsout may be null (zero).  dq, dk, dv are ADDED to (call
+ * oracle_parallel_backward first for the terms without state); ds0 may be
+ * null, else it is overwritten.
+ */
+int oracle_state_backward(int B, int H, int L, int dk, int dv, const double* q, const double* k,
+                          const double* v, const double* gamma, const double* dy, const double* s0,
+                          const double* dsout, double* dq, double* dkk, double* dvv, double* ds0) {
+    if (B < 0 || H < 1 || L < 0 || dk < 1 || dv < 1 || !q || !k || !v || !gamma || !dy || !dq || !dkk || !dvv)
+        return -1;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const size_t ok = ((size_t)b * H + h) * L * dk, ov = ((size_t)b * H + h) * L * dv;
+            const size_t os = ((size_t)b * H + h) * dk * dv;
+            const double g = gamma[h];
+            for (int n = 0; n < L; ++n) {
+                const double wq = gpow(g, (long)n + 1), ws = gpow(g, (long)L - 1 - n);
+                for (int i = 0; i < dk; ++i)
+                    for (int j = 0; j < dv; ++j) {
+                        if (s0) dq[ok + (size_t)n * dk + i] += wq * dy[ov + (size_t)n * dv + j] * s0[os + (size_t)i * dv + j];
+                        if (dsout) {
+                            const double d = dsout[os + (size_t)i * dv + j];
+                            dkk[ok + (size_t)n * dk + i] += ws * v[ov + (size_t)n * dv + j] * d;
+                            dvv[ov + (size_t)n * dv + j] += ws * k[ok + (size_t)n * dk + i] * d;
+                        }
+                    }
+            }
+            if (!ds0) continue;
+            const double gL = gpow(g, (long)L);
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) {
+                    double acc = dsout ? gL * dsout[os + (size_t)i * dv + j] : 0.0;
+                    for (int n = 0; n < L; ++n)
+                        acc += gpow(g, (long)n + 1) * q[ok + (size_t)n * dk + i] * dy[ov + (size_t)n * dv + j];
+                    ds0[os + (size_t)i * dv + j] = acc;
+                }
+        }
+    return 0;
+}

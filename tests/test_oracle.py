@@ -255,11 +255,68 @@ def pin_backward_gamma_zero(lib):
     assert np.allclose(dq, dyv * k) and np.allclose(dkk, dyv * q) and np.allclose(dvv, qk * dy)
 
 
+def pin_state_backward_central_differences(lib):
+    # L = sum(dy * y) + sum(dS_out * S_out) is linear in each of q, k, v and
+    # state_in separately, so a central difference in one entry is exact up to
+    # rounding.  The forward is the pinned recurrence.
+    rng = np.random.default_rng(11)
+    B, H, L, dk, dv = 1, 2, 5, 3, 4
+    q, k, v = (rng.standard_normal((B, H, L, d)) for d in (dk, dk, dv))
+    s0 = rng.standard_normal((B, H, dk, dv))
+    dy = rng.standard_normal((B, H, L, dv))
+    dso = rng.standard_normal((B, H, dk, dv))
+    gam = np.array([0.7, 0.9])
+    grads = oracle.backward(q, k, v, gam, dy, s0, dso, lib=lib)
+
+    def loss(q_, k_, v_, s_):
+        y, so = oracle.recurrent(q_, k_, v_, gam, s_, lib=lib)
+        return float(np.sum(dy * y) + np.sum(dso * so))
+
+    eps = 0.5
+    for which, idxs in ((0, ((0, 0, 0, 0), (0, 1, 4, 2))), (1, ((0, 0, 4, 1), (0, 1, 2, 0), (0, 1, 0, 2))),
+                        (2, ((0, 0, 4, 3), (0, 1, 1, 0), (0, 0, 0, 2))), (3, ((0, 0, 0, 0), (0, 1, 2, 3)))):
+        for idx in idxs:
+            plus, minus = [x.copy() for x in (q, k, v, s0)], [x.copy() for x in (q, k, v, s0)]
+            plus[which][idx] += eps
+            minus[which][idx] -= eps
+            fd = (loss(*plus) - loss(*minus)) / (2 * eps)
+            g = grads[which][idx]
+            assert abs(fd - g) <= 1e-9 * max(1.0, abs(fd)), (which, idx, fd, g)
+
+
+def pin_state_backward_closed_forms(lib):
+    rng = np.random.default_rng(12)
+    q, k = rng.standard_normal((2, 1, 1, 4, 3))
+    v, dy = rng.standard_normal((2, 1, 1, 4, 2))
+    s0, dso = rng.standard_normal((2, 1, 1, 3, 2))
+    # gamma = 1: plain sums; S_out = S0 + sum_m k_m^T v_m and y_n gains q_n S0
+    dq, dkk, dvv, ds0 = oracle.backward(q, k, v, np.ones(1), dy, s0, dso, lib=lib)
+    bq, bk, bv = oracle.parallel_backward(q, k, v, np.ones(1), dy, lib=lib)
+    assert np.allclose(ds0[0, 0], dso[0, 0] + q[0, 0].T @ dy[0, 0])
+    assert np.allclose(dq[0, 0], bq[0, 0] + dy[0, 0] @ s0[0, 0].T)
+    assert np.allclose(dkk[0, 0], bk[0, 0] + v[0, 0] @ dso[0, 0].T)
+    assert np.allclose(dvv[0, 0], bv[0, 0] + k[0, 0] @ dso[0, 0])
+    # gamma = 0: S0 never reaches y or S_out; only the last token reaches S_out
+    dq, dkk, dvv, ds0 = oracle.backward(q, k, v, np.zeros(1), dy, s0, dso, lib=lib)
+    bq, bk, bv = oracle.parallel_backward(q, k, v, np.zeros(1), dy, lib=lib)
+    assert np.array_equal(ds0, np.zeros_like(ds0)) and np.allclose(dq, bq)
+    assert np.allclose(dkk[0, 0, :3], bk[0, 0, :3]) and np.allclose(dvv[0, 0, :3], bv[0, 0, :3])
+    assert np.allclose(dkk[0, 0, 3], bk[0, 0, 3] + dso[0, 0] @ v[0, 0, 3])
+    assert np.allclose(dvv[0, 0, 3], bv[0, 0, 3] + k[0, 0, 3] @ dso[0, 0])
+    # no state given: the same as the backward without state, dS0 from dy alone
+    dq, dkk, dvv, ds0 = oracle.backward(q, k, v, np.full(1, 0.5), dy, lib=lib)
+    bq, bk, bv = oracle.parallel_backward(q, k, v, np.full(1, 0.5), dy, lib=lib)
+    assert np.array_equal(dq, bq) and np.array_equal(dkk, bk) and np.array_equal(dvv, bv)
+    w = 0.5 ** np.arange(1, 5)
+    assert np.allclose(ds0[0, 0], (q[0, 0] * w[:, None]).T @ dy[0, 0])
+
+
 ALL_PINS = [pin_three_token, pin_one_token_with_state, pin_multihead_gamma_indexing,
             pin_exact_rational, pin_gamma_one_is_unnormalised_linear_attention,
             pin_gamma_zero_is_diagonal, pin_forms_agree, pin_split_call, pin_linearity,
             pin_groupnorm_golden, pin_groupnorm_invariants, pin_groupnorm_heads,
-            pin_backward_central_differences, pin_backward_gamma_zero]
+            pin_backward_central_differences, pin_backward_gamma_zero,
+            pin_state_backward_central_differences, pin_state_backward_closed_forms]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -324,6 +381,12 @@ MUTATIONS = [
     ("backward dk from the wrong row", "dkk[ok + (size_t)m * dk + i] += w * dyv * q[ok + (size_t)n * dk + i];",
      "dkk[ok + (size_t)m * dk + i] += w * dyv * q[ok + (size_t)m * dk + i];"),
     ("backward dv drops the decay", "dvv[ov + (size_t)m * dv + j] += w * qk", "dvv[ov + (size_t)m * dv + j] += qk"),
+    ("state backward dq decay off by one", "const double wq = gpow(g, (long)n + 1)", "const double wq = gpow(g, (long)n)"),
+    ("state backward dk decay off by one", "ws = gpow(g, (long)L - 1 - n)", "ws = gpow(g, (long)L - n)"),
+    ("state backward dk uses dy for v", "+= ws * v[ov + (size_t)n * dv + j] * d;", "+= ws * dy[ov + (size_t)n * dv + j] * d;"),
+    ("state backward dq reads S0 untransposed", "* s0[os + (size_t)i * dv + j];", "* s0[os + (size_t)(dk - 1 - i) * dv + j];"),
+    ("dS0 drops gamma^L", "gL * dsout[", "dsout["),
+    ("dS0 sum decay off by one", "acc += gpow(g, (long)n + 1) * q[", "acc += gpow(g, (long)n) * q["),
     ("backward misses the diagonal", "                for (int m = 0; m <= n; ++m) {\n                    const double w = gpow(g, n - m);",
      "                for (int m = 0; m < n; ++m) {\n                    const double w = gpow(g, n - m);"),
 ]
