@@ -12,6 +12,8 @@ Also measured in the same run (same timing rules, reported under "forms"):
   parallel_backward -- its gradients dq, dk, dv on the same shape;
   chunkwise_backward_long_context -- the gradients through the chunkwise form,
                 one 16384-token call of the long-context layout;
+  chunkwise_backward_state_long_context -- the same with a carried state
+                (state_in, the gradient of state_out, the gradient of state_in);
   chunkwise_msr_core -- chunkwise C=64 on the same MSR-core shape;
   long_context_C{64,128,256} -- B=1, H=16, L=65536, dk=128, dv=256 as four
                 16384-token calls with the state carried in place;
@@ -436,7 +438,18 @@ def bench_small(ret, args, dist, peaks):
         "workload": "long_context layout, one 16384-token call: dq dk dv through the chunkwise form, C=128",
         "tokens_per_s": dist.sum(w.B * seg) / (t * 1e-3), "call_ms": round(t, 4),
         "tensor_frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
-    del parts, y, dy
+    # the same call carrying a state: state_in, dstate_out in, dstate_in out
+    s0 = torch.randn((w.B, w.H, w.dk, w.dv), device="cuda") / math.sqrt(w.dk)
+    dso = torch.randn_like(s0) / math.sqrt(w.dv)
+    ds0 = torch.empty_like(s0)
+    per, _ = time_calls(lambda: ret.chunkwise_backward_state(qq, kk, vv, gam, dy, 128, s0, dso, dstate_in=ds0), 10,
+                        max(args.warmup, 3), dist)
+    t = dist.max(statistics.median(per))
+    out["chunkwise_backward_state_long_context"] = {
+        "workload": "as chunkwise_backward_long_context, with state_in, dstate_out and dstate_in (fp32 states)",
+        "tokens_per_s": dist.sum(w.B * seg) / (t * 1e-3), "call_ms": round(t, 4),
+        "tensor_frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+    del parts, y, dy, s0, dso, ds0
     # per-head group normalisation of a headline-sized output (268 MB, larger than L2), in place
     w = HEADLINE
     y = (torch.randn((w.B, w.H, w.L, w.dv), device="cuda") * 0.5).to(torch.bfloat16)

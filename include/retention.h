@@ -256,6 +256,45 @@ RET_API ret_status retention_chunkwise_backward(const void* q, const void* k, co
 /* Workspace size of retention_chunkwise_backward. */
 RET_API size_t retention_chunkwise_backward_workspace_bytes(int chunk, ret_shape s, ret_dtype dt);
 
+/*
+ * Backward pass of a retention_chunkwise call that carries a state: the
+ * gradients of y and state_out with respect to q, k, v and state_in.  With
+ * state_in S0 the forward gives y_n += gamma^(n+1) q_n S0 and
+ * state_out = gamma^L S0 + sum_m gamma^(L-1-m) k_m^T v_m (the recurrence of
+ * the page "Retentive Networks -- Microsoft ...", section "Il meccanismo",
+ * started from S0), so for upstream gradients dy and dS_out this call adds to
+ * the sums of retention_chunkwise_backward
+ *     dq_n += gamma^(n+1) dy_n S0^T
+ *     dk_m += gamma^(L-1-m) v_m dS_out^T,   dv_m += gamma^(L-1-m) k_m dS_out
+ * and writes dS0 = gamma^L dS_out + sum_n gamma^(n+1) q_n^T dy_n.  Each extra
+ * term is the initial-state term of one of the three chunkwise sums, so the
+ * cost is that of retention_chunkwise_backward plus a transpose of the states.
+ * state_in   : device fp32 [B][H][dk][dv] the forward call started from, or
+ *              NULL (zero state).
+ * dstate_out : device fp32 [B][H][dk][dv] gradient of state_out, or NULL
+ *              (state_out unused).
+ * dstate_in  : device fp32 [B][H][dk][dv] receives dS0, or NULL (not wanted).
+ *              May alias state_in or dstate_out (both are consumed first), so a
+ *              caller walking a long sequence backwards call by call can keep
+ *              one state-gradient buffer.
+ * All three 16-byte aligned.  With L = 0 the call writes dS0 = dS_out (zero
+ * when dstate_out is NULL) and nothing else.
+ * Heads with gamma below 2^-60 drop the dS_out terms of rows m < L-1 of dk and
+ * dv, whose factor gamma^(L-1-m) is below 2^-60; every other term is kept.
+ * Supported shapes, dtypes and chunks: those of retention_chunkwise_backward.
+ * workspace : retention_chunkwise_backward_state_workspace_bytes() bytes,
+ *             256-byte aligned (that of retention_chunkwise_backward plus
+ *             three fp32 states when any state pointer is given).
+ */
+RET_API ret_status retention_chunkwise_backward_state(const void* q, const void* k, const void* v,
+                                                      const float* gamma, const void* dy, const float* state_in,
+                                                      const float* dstate_out, void* dq, void* dk, void* dv,
+                                                      float* dstate_in, int chunk, ret_shape s, ret_dtype dt,
+                                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace size of retention_chunkwise_backward_state (any state pointer given). */
+RET_API size_t retention_chunkwise_backward_state_workspace_bytes(int chunk, ret_shape s, ret_dtype dt);
+
 /* Synchronises `stream`, then returns and clears the device status word:
  * RET_OK, RET_ETIMEOUT if a kernel's bounded wait expired since the last
  * query, or RET_ECUDA if the stream reported an error. */

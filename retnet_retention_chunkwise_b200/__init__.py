@@ -24,8 +24,9 @@ import torch
 
 from . import _abi
 
-__all__ = ["parallel", "chunkwise", "recurrent_step", "device_status", "workspace_bytes",
-           "RetentionError", "library"]
+__all__ = ["parallel", "chunkwise", "chunkwise_host", "recurrent_step", "groupnorm", "chunkwise_groupnorm",
+           "parallel_backward", "chunkwise_backward", "chunkwise_backward_state", "device_status",
+           "workspace_bytes", "RetentionError", "library"]
 
 _LIB = None
 _LOCK = threading.Lock()
@@ -310,6 +311,37 @@ def chunkwise_backward(q, k, v, gamma, dy, chunk: int, *, workspace=None):
                                                   _ptr(dq), _ptr(dk), _ptr(dv), int(chunk), s, dt, _ptr(workspace),
                                                   wbytes, _stream()), "retention_chunkwise_backward")
     return dq, dk, dv
+
+
+def chunkwise_backward_state(q, k, v, gamma, dy, chunk: int, state_in=None, dstate_out=None, *,
+                             dstate_in=None, workspace=None):
+    """Gradients (dq, dk, dv, dstate_in) of :func:`chunkwise` started from
+    ``state_in`` (None: zero), for upstream gradients dy of y and
+    ``dstate_out`` of its state_out (None: unused); retention_chunkwise_backward_state.
+
+    ``dstate_in`` may be given as the output buffer (fp32 [B,H,dk,dv]); it may be
+    the same tensor as ``dstate_out``."""
+    dt = _qkv(q, k, v)
+    _cuda(dy, "dy")
+    if dy.shape != v.shape or dy.dtype != v.dtype:
+        raise ValueError("retention: dy must match v")
+    s = _shape(q, v)
+    for name, t in (("state_in", state_in), ("dstate_out", dstate_out), ("dstate_in", dstate_in)):
+        if t is not None:
+            _cuda(t, name)
+            if t.dtype != torch.float32 or tuple(t.shape) != (s.B, s.H, s.dk, s.dv) or not t.is_contiguous():
+                raise ValueError(f"retention: {name} must be contiguous fp32 [B,H,dk,dv]")
+    if dstate_in is None:
+        dstate_in = torch.empty((s.B, s.H, s.dk, s.dv), dtype=torch.float32, device=q.device)
+    need = int(library().retention_chunkwise_backward_state_workspace_bytes(int(chunk), s, dt))
+    if workspace is None:
+        workspace = torch.empty((need + 3) // 4, dtype=torch.float32, device=q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    _check(library().retention_chunkwise_backward_state(
+        _ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(dy), _ptr(state_in), _ptr(dstate_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dstate_in),
+        int(chunk), s, dt, _ptr(workspace), wbytes, _stream()), "retention_chunkwise_backward_state")
+    return dq, dk, dv, dstate_in
 
 
 def recurrent_step(q, k, v, gamma, state, *, out=None):

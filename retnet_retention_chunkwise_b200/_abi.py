@@ -35,6 +35,8 @@ EXPORTS = (
     "retention_parallel_backward_workspace_bytes",
     "retention_chunkwise_backward",
     "retention_chunkwise_backward_workspace_bytes",
+    "retention_chunkwise_backward_state",
+    "retention_chunkwise_backward_state_workspace_bytes",
 )
 STATIC_WS_BYTES = 16 << 20  # scratch array behind retention_chunkwise_static_ws
 
@@ -82,6 +84,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.retention_chunkwise_backward.restype = ctypes.c_int
     lib.retention_chunkwise_backward_workspace_bytes.argtypes = [i, RetShape, i]
     lib.retention_chunkwise_backward_workspace_bytes.restype = sz
+    lib.retention_chunkwise_backward_state.argtypes = [vp, vp, vp, fp, vp, vp, vp, vp, vp, vp, vp, i, RetShape, i,
+                                                       vp, sz, vp]
+    lib.retention_chunkwise_backward_state.restype = ctypes.c_int
+    lib.retention_chunkwise_backward_state_workspace_bytes.argtypes = [i, RetShape, i]
+    lib.retention_chunkwise_backward_state_workspace_bytes.restype = sz
     for name in ("retention_parallel", "retention_chunkwise", "retention_recurrent_step",
                  "retention_get_device_status", "retention_abi_version"):
         getattr(lib, name).restype = ctypes.c_int

@@ -469,7 +469,7 @@ RET_API int retention_debug_trace(void* buf, int blocks, int events) {
 }
 #endif
 
-int retention_abi_version(void) { return 101; }
+int retention_abi_version(void) { return 102; }
 
 const char* retention_status_str(ret_status st) {
   switch (st) {
@@ -823,6 +823,11 @@ ret_status retention_parallel_backward(const void* q, const void* k, const void*
 // Chunkwise variant: the same three retention sums through the chunkwise form
 // (zero initial state), after the reversal buffers the workspace holds the
 // scratch of the largest of the three chunkwise calls.
+// One fp32 [B][H][dk][dv] state, rounded up to 256 bytes.
+size_t state_region_bytes(const ret_shape& s) {
+  return ((size_t)s.B * s.H * s.dk * s.dv * sizeof(float) + 255) & ~size_t(255);
+}
+
 size_t chunkwise_backward_split_ws(int chunk, const ret_shape& s, ret_dtype dt) {
   const ret_shape swapped{s.B, s.H, s.L, s.dv, s.dk};
   return std::max(retention_chunkwise_workspace_bytes(chunk, swapped, dt),
@@ -834,15 +839,43 @@ size_t retention_chunkwise_backward_workspace_bytes(int chunk, ret_shape s, ret_
   return parallel_backward_ws(s, dt == RET_BF16 ? 2 : 4, nullptr) + chunkwise_backward_split_ws(chunk, s, dt);
 }
 
+size_t retention_chunkwise_backward_state_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
+  const size_t base = retention_chunkwise_backward_workspace_bytes(chunk, s, dt);
+  if (!base) return 0;
+  return base + 3 * state_region_bytes(s);
+}
+
 ret_status retention_chunkwise_backward(const void* q, const void* k, const void* v, const float* gamma,
                                         const void* dy, void* dq, void* dk, void* dv, int chunk, ret_shape s,
                                         ret_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+  return retention_chunkwise_backward_state(q, k, v, gamma, dy, nullptr, nullptr, dq, dk, dv, nullptr, chunk, s, dt,
+                                            workspace, workspace_bytes, stream);
+}
+
+ret_status retention_chunkwise_backward_state(const void* q, const void* k, const void* v, const float* gamma,
+                                              const void* dy, const float* state_in, const float* dstate_out,
+                                              void* dq, void* dk, void* dv, float* dstate_in, int chunk,
+                                              ret_shape s, ret_dtype dt, void* workspace, size_t workspace_bytes,
+                                              void* stream) {
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
   if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
   if (chunk < 1) return RET_EINVAL;
-  if (s.L == 0) return RET_OK;
+  const bool carried = state_in || dstate_out || dstate_in;
+  if ((state_in && !aligned16(state_in)) || (dstate_out && !aligned16(dstate_out)) ||
+      (dstate_in && !aligned16(dstate_in)))
+    return RET_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t sbytes = (size_t)s.B * s.H * s.dk * s.dv * sizeof(float);
+  if (s.L == 0) {  // S_out = S0: dS0 = dS_out
+    if (!dstate_in) return RET_OK;
+    const cudaError_t e = dstate_out ? (dstate_out == dstate_in ? cudaSuccess
+                                                                 : cudaMemcpyAsync(dstate_in, dstate_out, sbytes,
+                                                                                   cudaMemcpyDeviceToDevice, st))
+                                     : cudaMemsetAsync(dstate_in, 0, sbytes, st);
+    return e == cudaSuccess ? RET_OK : RET_ECUDA;
+  }
   if (!q || !k || !v || !dy || !dq || !dk || !dv) return RET_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) || !aligned16(dk) ||
       !aligned16(dv))
@@ -859,29 +892,68 @@ ret_status retention_chunkwise_backward(const void* q, const void* k, const void
   size_t off[6];
   const size_t rev = parallel_backward_ws(s, es, off);
   const size_t split = chunkwise_backward_split_ws(chunk, s, dt);
-  if (!workspace || workspace_bytes < rev + split || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  const size_t sreg = carried ? state_region_bytes(s) : 0;
+  if (!workspace || workspace_bytes < rev + split + 3 * sreg || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return RET_EINVAL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(workspace);
   void *rq = w + off[0], *rk = w + off[1], *rv = w + off[2], *rdy = w + off[3], *t1 = w + off[4], *t2 = w + off[5];
   void* sw = split ? w + rev : nullptr;
+  // initial states of the three sums: S0^T, (dS_out / gamma)^T, dS_out / gamma;
+  // the x2 region later takes the dv sum's state_out
+  float* s0t = carried ? reinterpret_cast<float*>(w + rev + split) : nullptr;
+  float* x2 = carried ? reinterpret_cast<float*>(w + rev + split + sreg) : nullptr;
+  float* x3 = carried ? reinterpret_cast<float*>(w + rev + split + 2 * sreg) : nullptr;
   const long long BH = (long long)s.B * s.H;
-  // dq = retention(dy, v, k)
-  if ((rc = retention_chunkwise(dy, v, k, gamma, dq, nullptr, nullptr, chunk, swapped, dt, sw, split, stream)) !=
-      RET_OK)
+  HeadGamma hg, gl;
+  bool any_small = false;
+  for (int h = 0; h < s.H; ++h) {
+    hg.g[h] = gamma[h];
+    const bool small = !(gamma[h] >= kBwdMinGamma);
+    gl.g[h] = small ? (float)std::pow((double)gamma[h], (double)s.L) : 0.f;
+    any_small |= small;
+  }
+  for (int h = s.H; h < RET_MAX_HEADS; ++h) hg.g[h] = gl.g[h] = 0.f;
+  if (state_in || dstate_out) {
+    dim3 grid((s.dv + 31) / 32, (s.dk + 31) / 32, (unsigned)BH);
+    bwd_state_prep_kernel<<<grid, dim3(32, 8), 0, st>>>(state_in, dstate_out, s0t, x2, x3, s.H, s.dk, s.dv, hg);
+    if ((rc = launch_status()) != RET_OK) return rc;
+  }
+  // dq = retention(dy, v, k; S0^T)
+  if ((rc = retention_chunkwise(dy, v, k, gamma, dq, state_in ? s0t : nullptr, nullptr, chunk, swapped, dt, sw,
+                                split, stream)) != RET_OK)
     return rc;
   if ((rc = launch_reverse(q, rq, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
   if ((rc = launch_reverse(k, rk, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
   if ((rc = launch_reverse(v, rv, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
   if ((rc = launch_reverse(dy, rdy, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
-  // dk = R(retention(Rv, Rdy, Rq)),  dv = R(retention(Rk, Rq, Rdy))
-  if ((rc = retention_chunkwise(rv, rdy, rq, gamma, t1, nullptr, nullptr, chunk, swapped, dt, sw, split, stream)) !=
-      RET_OK)
+  // dk = R(retention(Rv, Rdy, Rq; x2)),  dv = R(retention(Rk, Rq, Rdy; x3)) with state_out T -> x2
+  if ((rc = retention_chunkwise(rv, rdy, rq, gamma, t1, dstate_out ? x2 : nullptr, nullptr, chunk, swapped, dt, sw,
+                                split, stream)) != RET_OK)
     return rc;
   if ((rc = launch_reverse(t1, dk, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
-  if ((rc = retention_chunkwise(rk, rq, rdy, gamma, t2, nullptr, nullptr, chunk, s, dt, sw, split, stream)) != RET_OK)
+  if ((rc = retention_chunkwise(rk, rq, rdy, gamma, t2, dstate_out ? x3 : nullptr, dstate_in ? x2 : nullptr, chunk,
+                                s, dt, sw, split, stream)) != RET_OK)
     return rc;
-  return launch_reverse(t2, dv, BH, s.L, s.dv, es, st);
+  if ((rc = launch_reverse(t2, dv, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
+  if (dstate_out && any_small) {
+    if (dt == RET_BF16)
+      bwd_last_token_kernel<__nv_bfloat16><<<(unsigned)BH, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), dstate_out,
+          static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), s.H, s.L, s.dk, s.dv, hg);
+    else
+      bwd_last_token_kernel<float><<<(unsigned)BH, 256, 0, st>>>(static_cast<const float*>(k),
+                                                                 static_cast<const float*>(v), dstate_out,
+                                                                 static_cast<float*>(dk), static_cast<float*>(dv),
+                                                                 s.H, s.L, s.dk, s.dv, hg);
+    if ((rc = launch_status()) != RET_OK) return rc;
+  }
+  if (dstate_in) {
+    const long long total = BH * s.dk * s.dv;
+    const unsigned grid = (unsigned)std::min<long long>((total + 255) / 256, 8LL * sm_count());
+    bwd_finish_state_kernel<<<grid, 256, 0, st>>>(x2, dstate_out, dstate_in, BH, s.H, s.dk * s.dv, hg, gl);
+    if ((rc = launch_status()) != RET_OK) return rc;
+  }
+  return RET_OK;
 }
 
 }  // extern "C"

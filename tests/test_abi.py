@@ -49,7 +49,7 @@ def test_status_strings_and_version(lib):
     names = [lib.retention_status_str(i).decode() for i in range(5)]
     assert names == ["RET_OK", "RET_EINVAL", "RET_EUNSUPPORTED", "RET_ECUDA", "RET_ETIMEOUT"]
     assert lib.retention_status_str(99).decode() == "RET_UNKNOWN"
-    assert lib.retention_abi_version() == 101
+    assert lib.retention_abi_version() == 102
 
 
 def _g(*vals):
@@ -168,3 +168,29 @@ def test_parallel_backward_validation(lib):
     assert call(ctypes.c_void_p(0x100000), need, dy=None) == _abi.RET_EINVAL
     assert call(ctypes.c_void_p(0x100000), need, _abi.RET_BF16,
                 _abi.RetShape(1, 2, 64, 96, 128)) == _abi.RET_EUNSUPPORTED
+
+
+def test_chunkwise_backward_state_validation(lib):
+    # every case below returns before any launch
+    s = _abi.RetShape(1, 2, 64, 64, 128)
+    g = _g(0.5, 0.9)
+    base = lib.retention_chunkwise_backward_workspace_bytes(64, s, _abi.RET_F32)
+    need = lib.retention_chunkwise_backward_state_workspace_bytes(64, s, _abi.RET_F32)
+    assert base > 0 and need == base + 3 * ((2 * 64 * 128 * 4 + 255) // 256 * 256)
+    ws = ctypes.c_void_p(0x100000)
+
+    def call(nbytes, s0=FAKE, dso=FAKE, ds0=FAKE, chunk=64, dt=_abi.RET_F32, shape=s, dy=FAKE, w=ws):
+        return lib.retention_chunkwise_backward_state(FAKE, FAKE, FAKE, g, dy, s0, dso, FAKE, FAKE, FAKE, ds0,
+                                                      chunk, shape, dt, w, nbytes, None)
+
+    assert call(need - 1) == _abi.RET_EINVAL                       # states need their three regions
+    assert call(base, s0=None, dso=None) == _abi.RET_EINVAL        # dstate_in alone needs them too
+    assert call(need, ds0=ctypes.c_void_p(0x1008)) == _abi.RET_EINVAL  # misaligned state
+    assert call(need, s0=ctypes.c_void_p(0x1004)) == _abi.RET_EINVAL
+    assert call(need, dy=None) == _abi.RET_EINVAL
+    assert call(need, chunk=0) == _abi.RET_EINVAL
+    assert call(need, w=ctypes.c_void_p(0x100010)) == _abi.RET_EINVAL  # workspace not 256-byte aligned
+    assert call(need, dt=_abi.RET_F32, shape=_abi.RetShape(1, 2, 64, 64, 512)) == _abi.RET_EUNSUPPORTED
+    assert lib.retention_chunkwise_backward_state(FAKE, FAKE, FAKE, _g(1.5, 0.9), FAKE, FAKE, FAKE, FAKE, FAKE,
+                                                  FAKE, FAKE, 64, s, _abi.RET_F32, ws, need,
+                                                  None) == _abi.RET_EINVAL  # gamma outside [0, 1]

@@ -369,3 +369,96 @@ def test_chunkwise_backward(dt, B, H, L, dk, dv, C):
     tol = 1e-4 if dt == torch.float32 else 2e-2
     errs = (rel(dq, dq_r), rel(dkk, dk_r), rel(dvv, dv_r))
     assert max(errs) <= tol, errs
+
+
+def _state_grad_inputs(dt, B, H, L, dk, dv, seed):
+    q, k, v = inputs.qkv(B, H, L, dk, dv, dt, seed=seed)
+    g = torch.Generator("cpu").manual_seed(seed + 1)
+    dy = (torch.randn((B, H, L, dv), generator=g) / math.sqrt(dv)).to(dt)
+    s0 = torch.randn((B, H, dk, dv), generator=g) / math.sqrt(dk)
+    dso = torch.randn((B, H, dk, dv), generator=g) / math.sqrt(dv)
+    return q, k, v, dy, s0, dso
+
+
+@pytest.mark.parametrize("dt,B,H,L,dk,dv,C", [
+    (torch.bfloat16, 1, 2, 700, 128, 256, 128),
+    (torch.bfloat16, 2, 2, 1000, 256, 128, 64),
+    (torch.bfloat16, 1, 1, 600, 128, 128, 256),    # 256-row blocks
+    (torch.bfloat16, 1, 2, 4096, 128, 128, 128),   # sequence split in all three calls
+    (torch.float32, 1, 2, 70, 32, 48, 16),
+])
+def test_chunkwise_backward_state(dt, B, H, L, dk, dv, C):
+    q, k, v, dy, s0, dso = _state_grad_inputs(dt, B, H, L, dk, dv, L + C + 3)
+    gam = inputs.multiscale_gammas(H)
+    ref = oracle.backward(q, k, v, gam, dy, s0, dso)
+    qd, kd, vd, dyd, s0d, dsod = dev(q, k, v, dy, s0, dso)
+    got = ret.chunkwise_backward_state(qd, kd, vd, gam, dyd, C, s0d, dsod)
+    assert ret.device_status() == 0
+    tol = 1e-4 if dt == torch.float32 else 2e-2
+    errs = [rel(a, b) for a, b in zip(got, ref)]
+    assert max(errs) <= tol, errs
+
+
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_chunkwise_backward_state_small_gamma_heads(dt):
+    # gamma 0 and 2^-70 take the zero-state route with the last-row term;
+    # 0.5 and 1 the scaled initial state; checked head by head
+    B, H, L, dk, dv, C = 1, 4, 37, 128, 128, 16
+    q, k, v, dy, s0, dso = _state_grad_inputs(dt, B, H, L, dk, dv, 91)
+    gam = np.array([0.0, 2.0 ** -70, 0.5, 1.0])
+    ref = oracle.backward(q, k, v, gam, dy, s0, dso)
+    got = ret.chunkwise_backward_state(*dev(q, k, v), gam, dy.cuda(), C, s0.cuda(), dso.cuda())
+    assert ret.device_status() == 0
+    tol = 1e-4 if dt == torch.float32 else 2e-2
+    for h in range(H):
+        errs = [rel(a[:, h], b[:, h]) for a, b in zip(got, ref) if np.max(np.abs(b[:, h])) > 0]
+        assert max(errs) <= tol, (h, errs)
+    assert torch.count_nonzero(got[3][:, 0]) == 0  # gamma = 0: dS0 = 0
+
+
+def test_chunkwise_backward_state_aliasing_and_optional_states():
+    dt, B, H, L, dk, dv, C = torch.bfloat16, 1, 2, 300, 128, 128, 64
+    q, k, v, dy, s0, dso = _state_grad_inputs(dt, B, H, L, dk, dv, 17)
+    gam = inputs.multiscale_gammas(H)
+    qd, kd, vd, dyd, s0d, dsod = dev(q, k, v, dy, s0, dso)
+    base = ret.chunkwise_backward_state(qd, kd, vd, gam, dyd, C, s0d, dsod)
+    # dstate_in written over dstate_out: the same bits
+    buf = dsod.clone()
+    al = ret.chunkwise_backward_state(qd, kd, vd, gam, dyd, C, s0d, buf, dstate_in=buf)
+    assert all(torch.equal(a, b) for a, b in zip(al, base))
+    # and over state_in
+    buf = s0d.clone()
+    al = ret.chunkwise_backward_state(qd, kd, vd, gam, dyd, C, buf, dsod, dstate_in=buf)
+    assert all(torch.equal(a, b) for a, b in zip(al, base))
+    # no state at all: the same as chunkwise_backward, dS0 still returned
+    dq, dkk, dvv, ds0 = ret.chunkwise_backward_state(qd, kd, vd, gam, dyd, C)
+    plain = ret.chunkwise_backward(qd, kd, vd, gam, dyd, C)
+    assert torch.equal(dq, plain[0]) and torch.equal(dkk, plain[1]) and torch.equal(dvv, plain[2])
+    assert rel(ds0, oracle.backward(q, k, v, gam, dy)[3]) <= 2e-2
+    # L = 0: dS0 = dS_out, zero without it
+    e = torch.empty((B, H, 0, dk), dtype=dt, device="cuda")
+    ev = torch.empty((B, H, 0, dv), dtype=dt, device="cuda")
+    assert torch.equal(ret.chunkwise_backward_state(e, e, ev, gam, ev, C, s0d, dsod)[3], dsod)
+    assert torch.count_nonzero(ret.chunkwise_backward_state(e, e, ev, gam, ev, C, s0d)[3]) == 0
+    assert ret.device_status() == 0
+
+
+def test_chunkwise_backward_state_chained_calls():
+    # a sequence run as two calls with the state carried, differentiated call by
+    # call from the end, gives the gradients of the whole sequence
+    dt, B, H, L, dk, dv, C, cut = torch.bfloat16, 1, 2, 900, 128, 256, 128, 512
+    q, k, v, dy, s0, dso = _state_grad_inputs(dt, B, H, L, dk, dv, 5)
+    gam = inputs.multiscale_gammas(H)
+    ref = oracle.backward(q, k, v, gam, dy, s0, dso)
+    qd, kd, vd, dyd, s0d, dsod = dev(q, k, v, dy, s0, dso)
+    parts = [slice(0, cut), slice(cut, L)]
+    cont = lambda t, p: t[:, :, p].contiguous()  # noqa: E731
+    _, s1 = ret.chunkwise(cont(qd, parts[0]), cont(kd, parts[0]), cont(vd, parts[0]), gam, C, state_in=s0d)
+    g2 = ret.chunkwise_backward_state(cont(qd, parts[1]), cont(kd, parts[1]), cont(vd, parts[1]), gam,
+                                      cont(dyd, parts[1]), C, s1, dsod)
+    g1 = ret.chunkwise_backward_state(cont(qd, parts[0]), cont(kd, parts[0]), cont(vd, parts[0]), gam,
+                                      cont(dyd, parts[0]), C, s0d, g2[3])
+    assert ret.device_status() == 0
+    for i in range(3):
+        assert rel(torch.cat([g1[i], g2[i]], dim=2), ref[i]) <= 2e-2, i
+    assert rel(g1[3], ref[3]) <= 2e-2
