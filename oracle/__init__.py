@@ -73,8 +73,9 @@ def load(path: str | None = None):
     lib.oracle_groupnorm.argtypes = [i, i, i, i, dp, ctypes.c_double, dp, dp, dp]
     lib.oracle_parallel_backward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp, dp]
     lib.oracle_state_backward.argtypes = [i, i, i, i, i] + [dp] * 11
+    lib.oracle_gate.argtypes = [ctypes.c_long, dp, dp, i, dp]
     for f in (lib.oracle_recurrent, lib.oracle_parallel, lib.oracle_chunkwise, lib.oracle_groupnorm,
-              lib.oracle_parallel_backward, lib.oracle_state_backward):
+              lib.oracle_parallel_backward, lib.oracle_state_backward, lib.oracle_gate):
         f.restype = ctypes.c_int
     if path == _LIB:
         _lib = lib
@@ -156,6 +157,21 @@ def groupnorm(y, eps: float = 1e-5, weight=None, bias=None, lib=None):
     out = np.zeros_like(y)
     if lib.oracle_groupnorm(B, H, L, dv, _ptr(y), float(eps), _ptr(w), _ptr(b), _ptr(out)) != 0:
         raise ValueError("oracle_groupnorm: invalid arguments")
+    return out
+
+
+GATE_ACTS = {"none": 0, "swish": 1, "sigmoid": 2}
+
+
+def gate(z, g, act: str = "swish", lib=None):
+    """out = act(g) * z elementwise in fp64 (act: "none", "swish", "sigmoid")."""
+    lib = lib or load()
+    z, g = _f64(z), _f64(g)
+    if z.shape != g.shape:
+        raise ValueError("oracle: gate shape mismatch")
+    out = np.zeros_like(z)
+    if lib.oracle_gate(z.size, _ptr(z), _ptr(g), GATE_ACTS[act], _ptr(out)) != 0:
+        raise ValueError("oracle_gate: invalid arguments")
     return out
 
 

@@ -362,3 +362,25 @@ int oracle_state_backward(int B, int H, int L, int dk, int dv, const double* q, 
         }
     return 0;
 }
+
+/*
+ * Output gate of the retention layer.  The author responses on paperhub.cn
+ * ("Retentive Network: A Successor to Transformer ...", reply on the
+ * "transformer without softmax" remark) name gated multi-scale retention next
+ * to group normalisation but give no formula.  Reading: the gate multiplies
+ * the normalised output elementwise by an activation of a gate input g of the
+ * same shape,
+ *     out = act(g) * z,   act(x) = x (act 0), x sigmoid(x) (act 1, swish),
+ *                         sigmoid(x) (act 2),  sigmoid(x) = 1 / (1 + exp(-x)).
+ * n values; out may alias z.
+ */
+int oracle_gate(long n, const double* z, const double* g, int act, double* out) {
+    if (n < 0 || !z || !g || !out || act < 0 || act > 2) return -1;
+    for (long i = 0; i < n; ++i) {
+        const double x = g[i];
+        const double s = 1.0 / (1.0 + exp(-x));
+        const double a = act == 0 ? x : (act == 1 ? x * s : s);
+        out[i] = a * z[i];
+    }
+    return 0;
+}

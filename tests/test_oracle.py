@@ -15,6 +15,7 @@
 mistake at a time and checks that these pins catch every one.
 """
 from fractions import Fraction
+import math
 import os
 import re
 import shutil
@@ -311,12 +312,28 @@ def pin_state_backward_closed_forms(lib):
     assert np.allclose(ds0[0, 0], (q[0, 0] * w[:, None]).T @ dy[0, 0])
 
 
+def pin_gate_closed_forms(lib):
+    ln3 = math.log(3.0)
+    z = np.array([2.0, -3.0, 5.0, 7.0, 0.5])
+    g = np.array([0.0, ln3, -ln3, 40.0, -1.5])
+    sig = oracle.gate(z, g, "sigmoid", lib=lib)
+    assert np.allclose(sig[:3], z[:3] * np.array([0.5, 0.75, 0.25]), rtol=1e-14, atol=0)
+    sw = oracle.gate(z, g, "swish", lib=lib)
+    assert np.allclose(sw[:3], z[:3] * np.array([0.0, 0.75 * ln3, -0.25 * ln3]), rtol=1e-14, atol=0)
+    assert abs(sw[3] - 40.0 * 7.0) < 1e-12  # swish(x) -> x for large x
+    assert np.array_equal(oracle.gate(z, g, "none", lib=lib), g * z)
+    # sigmoid(x) + sigmoid(-x) = 1 and swish(x) - swish(-x) = x, elementwise
+    ones = np.ones_like(z)
+    assert np.allclose(oracle.gate(ones, g, "sigmoid", lib=lib) + oracle.gate(ones, -g, "sigmoid", lib=lib), 1.0)
+    assert np.allclose(oracle.gate(ones, g, "swish", lib=lib) - oracle.gate(ones, -g, "swish", lib=lib), g)
+
+
 ALL_PINS = [pin_three_token, pin_one_token_with_state, pin_multihead_gamma_indexing,
             pin_exact_rational, pin_gamma_one_is_unnormalised_linear_attention,
             pin_gamma_zero_is_diagonal, pin_forms_agree, pin_split_call, pin_linearity,
             pin_groupnorm_golden, pin_groupnorm_invariants, pin_groupnorm_heads,
             pin_backward_central_differences, pin_backward_gamma_zero,
-            pin_state_backward_central_differences, pin_state_backward_closed_forms]
+            pin_state_backward_central_differences, pin_state_backward_closed_forms, pin_gate_closed_forms]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -387,6 +404,9 @@ MUTATIONS = [
     ("state backward dq reads S0 untransposed", "* s0[os + (size_t)i * dv + j];", "* s0[os + (size_t)(dk - 1 - i) * dv + j];"),
     ("dS0 drops gamma^L", "gL * dsout[", "dsout["),
     ("dS0 sum decay off by one", "acc += gpow(g, (long)n + 1) * q[", "acc += gpow(g, (long)n) * q["),
+    ("gate sigmoid of -x", "1.0 / (1.0 + exp(-x))", "1.0 / (1.0 + exp(x))"),
+    ("swish drops the x factor", "act == 1 ? x * s : s", "act == 1 ? s : s"),
+    ("gate multiplies the wrong element", "out[i] = a * z[i];", "out[i] = a * z[n - 1 - i];"),
     ("backward misses the diagonal", "                for (int m = 0; m <= n; ++m) {\n                    const double w = gpow(g, n - m);",
      "                for (int m = 0; m < n; ++m) {\n                    const double w = gpow(g, n - m);"),
 ]
