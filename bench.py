@@ -17,7 +17,8 @@ Also measured in the same run (same timing rules, reported under "forms"):
   chunkwise_msr_core -- chunkwise C=64 on the same MSR-core shape;
   long_context_C{64,128,256} -- B=1, H=16, L=65536, dk=128, dv=256 as four
                 16384-token calls with the state carried in place;
-  groupnorm  -- per-head group normalisation of a headline-sized output.
+  groupnorm  -- per-head group normalisation of a headline-sized output;
+  groupnorm_gated -- the same followed by the swish output gate.
 
 Timing: CUDA events on the launching stream, >= 3 warm-up steps, barrier +
 synchronize on both sides, max over ranks.  The headline inputs (537 MB) exceed
@@ -462,6 +463,18 @@ def bench_small(ret, args, dist, peaks):
                                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                      "frac": round(nb / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                                      "algorithmic_bytes": nb, "kernel": "groupnorm_rows_kernel<bf16>"}}
+    # the same with the swish output gate: y and the gate read once, the result written once
+    gate = torch.randn_like(y)
+    per, _ = time_calls(lambda: ret.groupnorm(y, 1e-5, out=y, gate=gate, act="swish"), 20, max(args.warmup, 3), dist)
+    t = dist.max(statistics.median(per))
+    nb = 3 * y.numel() * y.element_size()
+    out["groupnorm_gated"] = {"workload": "GroupNorm then swish gate: B=4 H=8 L=8192 dv=512 bf16, in place",
+                              "kernel_ms": round(t, 4), "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3),
+                              "roofline": {"bound": "hbm", "achieved": round(nb / (t * 1e-3) / 1e9, 1),
+                                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                           "frac": round(nb / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                                           "algorithmic_bytes": nb, "kernel": "groupnorm_rows_kernel<bf16>"}}
+    del y, gate
     return out
 
 

@@ -198,6 +198,26 @@ RET_API size_t retention_chunkwise_host_workspace_bytes(int chunk, ret_shape s, 
 RET_API ret_status retention_groupnorm(const void* y, void* out, float eps, const float* weight,
                                        const float* bias, ret_shape s, ret_dtype dt, void* stream);
 
+/* Activations of the output gate. */
+typedef enum { RET_GATE_NONE = 0, RET_GATE_SWISH = 1, RET_GATE_SIGMOID = 2 } ret_gate_act;
+
+/*
+ * retention_groupnorm followed by the output gate of gated multi-scale
+ * retention (named next to GroupNorm in the same author responses, reply on
+ * the "transformer without softmax" remark, with no formula).  Reading taken:
+ *     out_c = GroupNorm(y)_c * act(gate_c)
+ * with act(x) = x (RET_GATE_NONE), x / (1 + e^-x) (RET_GATE_SWISH) or
+ * 1 / (1 + e^-x) (RET_GATE_SIGMOID), in one pass over y and gate.
+ * gate : device [B][H][L][dv] in the call's dtype (the gate input, e.g. the
+ *        caller's projection of the layer input), or NULL for no gate; same
+ *        alignment rule as y.  out may be y (not gate).
+ * act  : a ret_gate_act; anything else is RET_EINVAL.
+ * Other arguments and limits as retention_groupnorm.
+ */
+RET_API ret_status retention_groupnorm_gated(const void* y, const void* gate, void* out, float eps,
+                                             const float* weight, const float* bias, int act, ret_shape s,
+                                             ret_dtype dt, void* stream);
+
 /*
  * Chunkwise form followed by retention_groupnorm on its output, in place: y
  * receives the normalised output.  The other arguments are as for

@@ -226,10 +226,13 @@ def _gn_params(weight, bias, H: int, dv: int, device):
                 raise ValueError(f"retention: {n} must be fp32 with H*dv values on the device of y")
 
 
-def groupnorm(y, eps: float = 1e-5, *, weight=None, bias=None, out=None):
+def groupnorm(y, eps: float = 1e-5, *, weight=None, bias=None, out=None, gate=None, act: str = "swish"):
     """Per-head group normalisation of y [B,H,L,dv]: each (b, h, n) row of dv
     values by its own mean and biased variance, then ``* weight + bias`` per
-    channel (fp32 [H*dv] CUDA tensors, optional).  ``out`` may be ``y``."""
+    channel (fp32 [H*dv] CUDA tensors, optional).  ``out`` may be ``y``.
+
+    With ``gate`` (y's shape and dtype) the result is multiplied by
+    ``act(gate)``, act one of "none", "swish", "sigmoid" (retention_groupnorm_gated)."""
     _cuda(y, "y")
     dt = _dtype(y)
     if y.dim() != 4:
@@ -240,8 +243,19 @@ def groupnorm(y, eps: float = 1e-5, *, weight=None, bias=None, out=None):
     if out.shape != y.shape or out.dtype != y.dtype:
         raise ValueError("retention: out must match y")
     _gn_params(weight, bias, H, dv, y.device)
-    _check(library().retention_groupnorm(_ptr(y), _ptr(out), float(eps), _ptr(weight), _ptr(bias),
-                                         _abi.RetShape(B, H, L, 1, dv), dt, _stream()), "retention_groupnorm")
+    s = _abi.RetShape(B, H, L, 1, dv)
+    if gate is None:
+        _check(library().retention_groupnorm(_ptr(y), _ptr(out), float(eps), _ptr(weight), _ptr(bias), s, dt,
+                                             _stream()), "retention_groupnorm")
+        return out
+    _cuda(gate, "gate")
+    if gate.shape != y.shape or gate.dtype != y.dtype:
+        raise ValueError("retention: gate must match y")
+    if act not in _abi.GATE_ACTS:
+        raise ValueError(f"retention: act must be one of {sorted(_abi.GATE_ACTS)}")
+    _check(library().retention_groupnorm_gated(_ptr(y), _ptr(gate), _ptr(out), float(eps), _ptr(weight),
+                                               _ptr(bias), _abi.GATE_ACTS[act], s, dt, _stream()),
+           "retention_groupnorm_gated")
     return out
 
 

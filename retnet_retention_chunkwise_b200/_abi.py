@@ -29,6 +29,7 @@ EXPORTS = (
     "retention_chunkwise_host",
     "retention_chunkwise_host_workspace_bytes",
     "retention_groupnorm",
+    "retention_groupnorm_gated",
     "retention_chunkwise_gn",
     "retention_chunkwise_gn_workspace_bytes",
     "retention_parallel_backward",
@@ -38,6 +39,7 @@ EXPORTS = (
     "retention_chunkwise_backward_state",
     "retention_chunkwise_backward_state_workspace_bytes",
 )
+GATE_ACTS = {"none": 0, "swish": 1, "sigmoid": 2}  # ret_gate_act
 STATIC_WS_BYTES = 16 << 20  # scratch array behind retention_chunkwise_static_ws
 
 
@@ -72,6 +74,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     f32 = ctypes.c_float
     lib.retention_groupnorm.argtypes = [vp, vp, f32, vp, vp, RetShape, i, vp]
     lib.retention_groupnorm.restype = ctypes.c_int
+    lib.retention_groupnorm_gated.argtypes = [vp, vp, vp, f32, vp, vp, i, RetShape, i, vp]
+    lib.retention_groupnorm_gated.restype = ctypes.c_int
     lib.retention_chunkwise_gn.argtypes = [vp, vp, vp, fp, vp, vp, vp, i, RetShape, i, f32, vp, vp, vp, sz, vp]
     lib.retention_chunkwise_gn.restype = ctypes.c_int
     lib.retention_chunkwise_gn_workspace_bytes.argtypes = [i, RetShape, i]

@@ -7,8 +7,14 @@
 //     out_c = (y_c - mean) / sqrt(var + eps) * w[h*dv + c] + bias[h*dv + c]
 // with the biased variance, and w, bias optional (null: 1 and 0).
 //
+// An optional output gate follows (same page, reply on the "transformer without
+// softmax" remark: gated multi-scale retention, no formula given).  Reading:
+//     out_c *= act(g_c),  act = identity, swish x sigmoid(x), or sigmoid(x)
+// with g a gate input of y's shape.
+//
 // This kernel runs on a finished y (one warp per row, fp32 statistics in two
-// passes over registers): it reads and writes y once, so it is bound by HBM.
+// passes over registers): it reads y (and g) once and writes the output once,
+// so it is bound by HBM.
 #pragma once
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -66,6 +72,14 @@ __device__ __forceinline__ void gn_store8(__nv_bfloat16* p, const float (&x)[8])
   *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+enum GateAct { kGateNone = 0, kGateSwish = 1, kGateSigmoid = 2 };
+
+__device__ __forceinline__ float gate_act(float x, int act) {
+  if (act == kGateNone) return x;
+  const float sg = 1.f / (1.f + expf(-x));
+  return act == kGateSwish ? x * sg : sg;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -74,17 +88,20 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // One warp per (b, h, n) row.  Vectorised (VEC values per lane per step: 8
 // for bf16 when dv % 256 == 0, 4 when dv % 128 == 0), else one value per lane
-// per step; dv <= 1024.  out may alias y.
+// per step; dv <= 1024.  out may alias y.  gate: null, or act(gate) multiplies
+// the result.
 template <typename T, int VEC>
 __global__ void __launch_bounds__(32 * kGN_RowsPerBlock)
 groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, float eps,
-                      const float* __restrict__ w, const float* __restrict__ bias) {
+                      const float* __restrict__ w, const float* __restrict__ bias, const T* __restrict__ gate,
+                      int act) {
   constexpr int kSteps = kGN_MaxDv / (32 * VEC);
   const int lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * kGN_RowsPerBlock + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int h = (int)((row / L) % H);
   const T* yr = y + row * dv;
+  const T* gr = gate ? gate + row * dv : nullptr;
   T* orow = out + row * dv;
   float x[kSteps][VEC];
   float s = 0.f;
@@ -130,6 +147,18 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
         z[e] = (x[i][e] - mean) * rstd;
         if (wr) z[e] *= wr[c + e];
         if (br) z[e] += br[c + e];
+      }
+      if (gr) {
+        float gv[VEC];
+        if constexpr (VEC == 8) {
+          gn_load8(gr + c, gv);
+        } else if constexpr (VEC == 4) {
+          gn_load4<T>(gr + c, gv);
+        } else {
+          gv[0] = (float)gr[c];
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) z[e] *= gate_act(gv[e], act);
       }
       if constexpr (VEC == 8) {
         gn_store8(orow + c, z);

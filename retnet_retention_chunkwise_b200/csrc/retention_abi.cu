@@ -307,26 +307,32 @@ ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const
 }
 
 ret_status launch_groupnorm(const void* y, void* out, float eps, const float* w, const float* b,
-                            const ret_shape& s, ret_dtype dt, cudaStream_t st) {
+                            const ret_shape& s, ret_dtype dt, cudaStream_t st, const void* gate = nullptr,
+                            int act = 0) {
   const long long rows = (long long)s.B * s.H * s.L;
   if (rows == 0) return RET_OK;
   const unsigned blocks = (unsigned)((rows + kGN_RowsPerBlock - 1) / kGN_RowsPerBlock);
   const bool vec = s.dv % 128 == 0;
   const int thr = 32 * kGN_RowsPerBlock;
   if (dt == RET_BF16) {
-    auto yi = static_cast<const __nv_bfloat16*>(y);
-    auto yo = static_cast<__nv_bfloat16*>(out);
+    using T = __nv_bfloat16;
+    auto yi = static_cast<const T*>(y);
+    auto yo = static_cast<T*>(out);
+    auto gi = static_cast<const T*>(gate);
     if (s.dv % 256 == 0)
-      groupnorm_rows_kernel<__nv_bfloat16, 8><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
+      groupnorm_rows_kernel<T, 8><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
     else if (vec)
-      groupnorm_rows_kernel<__nv_bfloat16, 4><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
+      groupnorm_rows_kernel<T, 4><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
     else
-      groupnorm_rows_kernel<__nv_bfloat16, 1><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
+      groupnorm_rows_kernel<T, 1><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
   } else {
     auto yi = static_cast<const float*>(y);
     auto yo = static_cast<float*>(out);
-    if (vec) groupnorm_rows_kernel<float, 4><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
-    else groupnorm_rows_kernel<float, 1><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b);
+    auto gi = static_cast<const float*>(gate);
+    if (vec)
+      groupnorm_rows_kernel<float, 4><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
+    else
+      groupnorm_rows_kernel<float, 1><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
   }
   return launch_status();
 }
@@ -743,18 +749,26 @@ ret_status retention_chunkwise_host(const void* q_host, const void* k_host, cons
   return RET_OK;
 }
 
-ret_status retention_groupnorm(const void* y, void* out, float eps, const float* weight, const float* bias,
-                               ret_shape s, ret_dtype dt, void* stream) {
+ret_status retention_groupnorm_gated(const void* y, const void* gate, void* out, float eps, const float* weight,
+                                     const float* bias, int act, ret_shape s, ret_dtype dt, void* stream) {
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
   if (!(eps >= 0.f) || !std::isfinite(eps)) return RET_EINVAL;
+  if (act < kGateNone || act > kGateSigmoid) return RET_EINVAL;
   if (s.L > 0 && (!y || !out)) return RET_EINVAL;
   if (s.dv > kGN_MaxDv) return RET_EUNSUPPORTED;
   const size_t es = dt == RET_BF16 ? 2 : 4;
-  if (s.dv % 128 == 0 && (!aligned16(y) || !aligned16(out))) return RET_EINVAL;
-  if (s.L > 0 && ((reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(out)) % es)) return RET_EINVAL;
-  return launch_groupnorm(y, out, eps, weight, bias, s, dt, static_cast<cudaStream_t>(stream));
+  if (s.dv % 128 == 0 && (!aligned16(y) || !aligned16(out) || (gate && !aligned16(gate)))) return RET_EINVAL;
+  if (s.L > 0 &&
+      ((reinterpret_cast<uintptr_t>(y) | reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(gate)) % es))
+    return RET_EINVAL;
+  return launch_groupnorm(y, out, eps, weight, bias, s, dt, static_cast<cudaStream_t>(stream), gate, act);
+}
+
+ret_status retention_groupnorm(const void* y, void* out, float eps, const float* weight, const float* bias,
+                               ret_shape s, ret_dtype dt, void* stream) {
+  return retention_groupnorm_gated(y, nullptr, out, eps, weight, bias, kGateNone, s, dt, stream);
 }
 
 size_t retention_chunkwise_gn_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {

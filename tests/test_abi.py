@@ -194,3 +194,17 @@ def test_chunkwise_backward_state_validation(lib):
     assert lib.retention_chunkwise_backward_state(FAKE, FAKE, FAKE, _g(1.5, 0.9), FAKE, FAKE, FAKE, FAKE, FAKE,
                                                   FAKE, FAKE, 64, s, _abi.RET_F32, ws, need,
                                                   None) == _abi.RET_EINVAL  # gamma outside [0, 1]
+
+
+def test_groupnorm_gated_validation(lib):
+    s = _abi.RetShape(1, 2, 8, 1, 128)
+    call = lambda gate, act, y=FAKE: lib.retention_groupnorm_gated(  # noqa: E731
+        y, gate, FAKE, 1e-5, None, None, act, s, _abi.RET_BF16, None)
+    assert call(FAKE, 3) == _abi.RET_EINVAL       # unknown activation
+    assert call(FAKE, -1) == _abi.RET_EINVAL
+    assert call(ctypes.c_void_p(0x10008), 1) == _abi.RET_EINVAL  # gate not 16-byte aligned (dv % 128 == 0)
+    assert call(FAKE, 1, y=None) == _abi.RET_EINVAL
+    assert lib.retention_groupnorm_gated(FAKE, FAKE, FAKE, -1.0, None, None, 1, s, _abi.RET_BF16,
+                                         None) == _abi.RET_EINVAL  # eps < 0
+    assert lib.retention_groupnorm_gated(FAKE, FAKE, FAKE, 1e-5, None, None, 1, _abi.RetShape(1, 2, 8, 1, 2048),
+                                         _abi.RET_BF16, None) == _abi.RET_EUNSUPPORTED

@@ -263,6 +263,26 @@ def test_groupnorm_standalone(dt, dv, affine):
     assert torch.equal(yd, out)
 
 
+@pytest.mark.parametrize("dt,dv", [(torch.bfloat16, 512), (torch.bfloat16, 128), (torch.bfloat16, 96),
+                                   (torch.float32, 128), (torch.float32, 48)])
+@pytest.mark.parametrize("act", ["swish", "sigmoid", "none"])
+def test_groupnorm_gated(dt, dv, act):
+    B, H, L = 2, 3, 29
+    g = torch.Generator("cpu").manual_seed(dv + 7)
+    y = (torch.randn((B, H, L, dv), generator=g) * 2.0 + 0.5).to(dt)
+    gate = (torch.randn((B, H, L, dv), generator=g) * 3.0).to(dt)
+    w = torch.rand(H * dv, generator=g) + 0.5
+    b = torch.randn(H * dv, generator=g) * 0.1
+    ref = oracle.gate(oracle.groupnorm(y, eps=1e-5, weight=w, bias=b), gate, act)
+    yd, gd = y.cuda(), gate.cuda()
+    out = ret.groupnorm(yd, 1e-5, weight=w.cuda(), bias=b.cuda(), gate=gd, act=act)
+    tol = 1e-4 if dt == torch.float32 else 2e-2
+    assert rel(out, ref) <= tol
+    ret.groupnorm(yd, 1e-5, weight=w.cuda(), bias=b.cuda(), gate=gd, act=act, out=yd)  # in place
+    assert torch.equal(yd, out)
+    assert ret.device_status() == 0
+
+
 @pytest.mark.parametrize("B,H,L,dk,dv,C", [
     (1, 2, 700, 256, 512, 128),    # sequence split, ragged tail, four dv slices
     (2, 2, 300, 256, 128, 64),
