@@ -17,6 +17,7 @@ Also measured in the same run (same timing rules, reported under "forms"):
   chunkwise_msr_core -- chunkwise C=64 on the same MSR-core shape;
   long_context_C{64,128,256} -- B=1, H=16, L=65536, dk=128, dv=256 as four
                 16384-token calls with the state carried in place;
+  chunkwise_state_headline -- the state-only call (no y) on the headline shape;
   groupnorm  -- per-head group normalisation of a headline-sized output;
   groupnorm_gated -- the same followed by the swish output gate.
 
@@ -451,8 +452,27 @@ def bench_small(ret, args, dist, peaks):
         "tokens_per_s": dist.sum(w.B * seg) / (t * 1e-3), "call_ms": round(t, 4),
         "tensor_frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
     del parts, y, dy, s0, dso, ds0
-    # per-head group normalisation of a headline-sized output (268 MB, larger than L2), in place
+    # state only (no y) on the headline shape: k and v read once (403 MB, larger than L2)
     w = HEADLINE
+    k = (torch.randn((w.B, w.H, w.L, w.dk), device="cuda") / math.sqrt(w.dk)).to(torch.bfloat16)
+    v = (torch.randn((w.B, w.H, w.L, w.dv), device="cuda") / math.sqrt(w.dk)).to(torch.bfloat16)
+    s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device="cuda")
+    need = ret.library().retention_chunkwise_state_workspace_bytes(w.chunk, ret._shape(k, v), ret._abi.RET_BF16)
+    wsb = torch.empty((need + 3) // 4, dtype=torch.float32, device="cuda")
+    per, _ = time_calls(lambda: ret.chunkwise_state(k, v, w.gammas(), w.chunk, out=s_out, workspace=wsb), 20,
+                        max(args.warmup, 3), dist)
+    t = dist.max(statistics.median(per))
+    nb = (k.numel() + v.numel()) * 2 + s_out.numel() * 4
+    fl = 2 * w.B * w.H * w.L * w.dk * w.dv
+    out["chunkwise_state_headline"] = {
+        "workload": "state only (no y): B=4 H=8 L=8192 dk=256 dv=512 C=128, k and v read, fp32 state out",
+        "call_ms": round(t, 4), "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": round(nb / (t * 1e-3) / 1e9, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(nb / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                     "algorithmic_bytes": nb, "kernel": "chunk_state_kernel<256> + state_fold_kernel"},
+        "tensor_frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
+    del k, v, s_out, wsb
+    # per-head group normalisation of a headline-sized output (268 MB, larger than L2), in place
     y = (torch.randn((w.B, w.H, w.L, w.dv), device="cuda") * 0.5).to(torch.bfloat16)
     per, _ = time_calls(lambda: ret.groupnorm(y, 1e-5, out=y), 20, max(args.warmup, 3), dist)
     t = dist.max(statistics.median(per))

@@ -148,6 +148,48 @@ RET_API ret_status retention_chunkwise_static_ws(const void* q, const void* k, c
                                                  ret_dtype dt, void* stream);
 
 /*
+ * The state_out of retention_chunkwise without y: for the L tokens of the call,
+ *     state_out = gamma^L state_in + sum_t gamma^(L-1-t) k_t^T v_t
+ * (the recurrence of the page "Retentive Networks -- Microsoft ...", section
+ * "Il meccanismo", unrolled over the call).  It reads only k and v, so it costs
+ * about a third of the full call.  Uses: a prompt whose outputs are not needed
+ * before decoding, and the first pass of a sequence cut across GPUs (each
+ * rank's run summed from a zero state, then retention_state_fold).
+ * k : device [B][H][L][dk], v : device [B][H][L][dv], the call's dtype, 16-byte
+ *     aligned.  state_in : device fp32 [B][H][dk][dv] or NULL (zero).
+ * state_out : device fp32 [B][H][dk][dv], required; may alias state_in.
+ * bf16: shapes and chunks of the tensor-core chunkwise path; workspace of
+ *     retention_chunkwise_state_workspace_bytes() bytes (256-byte aligned), at
+ *     least two states per (b, h): the run is cut into segments summed in
+ *     parallel, fewer when the workspace is smaller.  fp32: as retention_chunkwise
+ *     (no workspace).
+ * L = 0 copies state_in (or zeros) to state_out.
+ */
+RET_API ret_status retention_chunkwise_state(const void* k, const void* v, const float* gamma,
+                                             const float* state_in, float* state_out, int chunk, ret_shape s,
+                                             ret_dtype dt, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace size of retention_chunkwise_state (0 for fp32 or L = 0). */
+RET_API size_t retention_chunkwise_state_workspace_bytes(int chunk, ret_shape s, ret_dtype dt);
+
+/*
+ * The state at the end of consecutive runs of tokens, from each run's own sum:
+ * with D_i the state of run i from a zero state (retention_chunkwise_state) and
+ * len_i its length,
+ *     S = state_in;  for i = 0 .. n-1:  S = gamma^len_i S + D_i;  state_out = S.
+ * The same page and section: the state after a run is the decayed state before
+ * it plus the run's own sum.  On a sequence cut across ranks, rank r folds the
+ * parts of ranks 0 .. r-1 to get the state its own run starts from.
+ * parts : device fp32 [n][B][H][dk][dv] (the D_i), 16-byte aligned; must not
+ *         alias state_out.
+ * lens  : host int [n], each >= 0.  n in [0, 256].
+ * state_in : device fp32 [B][H][dk][dv] or NULL (zero); state_out : device fp32,
+ *         may alias state_in.  s.L is ignored.  Runs on `stream`.
+ */
+RET_API ret_status retention_state_fold(const float* parts, const int* lens, int n, const float* gamma,
+                                        const float* state_in, float* state_out, ret_shape s, void* stream);
+
+/*
  * Chunkwise form on host buffers: q, k, v are copied from host memory, the
  * chunkwise form runs on the device, and y is copied back to host memory, all
  * inside this call's work on `stream` (the same results as

@@ -25,7 +25,8 @@ import torch
 from . import _abi
 
 __all__ = ["parallel", "chunkwise", "chunkwise_host", "recurrent_step", "groupnorm", "chunkwise_groupnorm",
-           "parallel_backward", "chunkwise_backward", "chunkwise_backward_state", "device_status",
+           "parallel_backward", "chunkwise_backward", "chunkwise_backward_state", "chunkwise_state",
+           "state_fold", "device_status",
            "workspace_bytes", "RetentionError", "library"]
 
 _LIB = None
@@ -356,6 +357,61 @@ def chunkwise_backward_state(q, k, v, gamma, dy, chunk: int, state_in=None, dsta
         _ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(dy), _ptr(state_in), _ptr(dstate_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dstate_in),
         int(chunk), s, dt, _ptr(workspace), wbytes, _stream()), "retention_chunkwise_backward_state")
     return dq, dk, dv, dstate_in
+
+
+def chunkwise_state(k, v, gamma, chunk: int, *, state_in=None, out=None, workspace=None):
+    """The state_out of :func:`chunkwise` on (k, v) without computing y:
+    gamma^L state_in + sum_t gamma^(L-1-t) k_t^T v_t, fp32 [B,H,dk,dv]
+    (retention_chunkwise_state)."""
+    _cuda(k, "k")
+    _cuda(v, "v")
+    dt = _dtype(k)
+    if v.dtype != k.dtype or k.dim() != 4 or v.dim() != 4 or k.shape[:3] != v.shape[:3]:
+        raise ValueError("retention: k [B,H,L,dk] and v [B,H,L,dv] must match in dtype and B, H, L")
+    s = _shape(k, v)
+    shape = (s.B, s.H, s.dk, s.dv)
+    for name, t in (("state_in", state_in), ("out", out)):
+        if t is not None:
+            _cuda(t, name)
+            if t.dtype != torch.float32 or tuple(t.shape) != shape:
+                raise ValueError(f"retention: {name} must be fp32 [B,H,dk,dv]")
+    if out is None:
+        out = torch.empty(shape, dtype=torch.float32, device=k.device)
+    need = int(library().retention_chunkwise_state_workspace_bytes(int(chunk), s, dt))
+    if workspace is None and need > 0:
+        workspace = torch.empty((need + 3) // 4, dtype=torch.float32, device=k.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(library().retention_chunkwise_state(_ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(state_in), _ptr(out),
+                                               int(chunk), s, dt, _ptr(workspace), wbytes, _stream()),
+           "retention_chunkwise_state")
+    return out
+
+
+def state_fold(parts, lens, gamma, *, state_in=None, out=None):
+    """The state after consecutive runs from the runs' own sums: S = state_in,
+    then S = gamma^len_i S + parts[i] for each run i (retention_state_fold).
+
+    parts: fp32 CUDA tensor [n,B,H,dk,dv]; lens: n run lengths (ints)."""
+    _cuda(parts, "parts")
+    if parts.dtype != torch.float32 or parts.dim() != 5:
+        raise ValueError("retention: parts must be fp32 [n,B,H,dk,dv]")
+    n, B, H, dk, dv = parts.shape
+    lens = [int(x) for x in lens]
+    if len(lens) != n:
+        raise ValueError("retention: one length per part")
+    shape = (B, H, dk, dv)
+    for name, t in (("state_in", state_in), ("out", out)):
+        if t is not None:
+            _cuda(t, name)
+            if t.dtype != torch.float32 or tuple(t.shape) != shape:
+                raise ValueError(f"retention: {name} must be fp32 [B,H,dk,dv]")
+    if out is None:
+        out = torch.empty(shape, dtype=torch.float32, device=parts.device)
+    c_lens = (ctypes.c_int * max(n, 1))(*lens)
+    _check(library().retention_state_fold(_ptr(parts) if n > 0 else None, c_lens, n, _gamma(gamma, H),
+                                          _ptr(state_in), _ptr(out), _abi.RetShape(B, H, 0, dk, dv), _stream()),
+           "retention_state_fold")
+    return out
 
 
 def recurrent_step(q, k, v, gamma, state, *, out=None):

@@ -38,6 +38,9 @@ EXPORTS = (
     "retention_chunkwise_backward_workspace_bytes",
     "retention_chunkwise_backward_state",
     "retention_chunkwise_backward_state_workspace_bytes",
+    "retention_chunkwise_state",
+    "retention_chunkwise_state_workspace_bytes",
+    "retention_state_fold",
 )
 GATE_ACTS = {"none": 0, "swish": 1, "sigmoid": 2}  # ret_gate_act
 STATIC_WS_BYTES = 16 << 20  # scratch array behind retention_chunkwise_static_ws
@@ -93,6 +96,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.retention_chunkwise_backward_state.restype = ctypes.c_int
     lib.retention_chunkwise_backward_state_workspace_bytes.argtypes = [i, RetShape, i]
     lib.retention_chunkwise_backward_state_workspace_bytes.restype = sz
+    lib.retention_chunkwise_state.argtypes = [vp, vp, fp, vp, vp, i, RetShape, i, vp, sz, vp]
+    lib.retention_chunkwise_state.restype = ctypes.c_int
+    lib.retention_chunkwise_state_workspace_bytes.argtypes = [i, RetShape, i]
+    lib.retention_chunkwise_state_workspace_bytes.restype = sz
+    lib.retention_state_fold.argtypes = [vp, ctypes.POINTER(ctypes.c_int), i, fp, vp, vp, RetShape, vp]
+    lib.retention_state_fold.restype = ctypes.c_int
     for name in ("retention_parallel", "retention_chunkwise", "retention_recurrent_step",
                  "retention_get_device_status", "retention_abi_version"):
         getattr(lib, name).restype = ctypes.c_int

@@ -21,6 +21,7 @@
 #include "decode.cuh"
 #include "parallel_tc.cuh"
 #include "simt_f32.cuh"
+#include "state_fold.cuh"
 #include "tc_common.cuh"
 
 namespace {
@@ -268,6 +269,85 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
     chunkwise_tc_kernel<DK><<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, my, a, dec);
     return launch_status();
   }
+}
+
+// Launch state_fold_kernel: out = fold of n parts (see state_fold.cuh).
+ret_status launch_state_fold(const float* state_in, const float* parts, float* out, const ret_shape& s,
+                             const float* gamma, int n, const int* lens, long long part_stride,
+                             long long bh_stride, cudaStream_t st) {
+  HeadLog2 hl;
+  FoldLens fl;
+  for (int h = 0; h < s.H; ++h) hl.l2g[h] = log2_gamma(gamma[h]);
+  for (int h = s.H; h < RET_MAX_HEADS; ++h) hl.l2g[h] = 0.f;
+  for (int i = 0; i < kFoldMaxParts; ++i) fl.len[i] = i < n ? lens[i] : 0;
+  const long long BH = (long long)s.B * s.H;
+  const long long total = BH * s.dk * s.dv;
+  const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>((total + 255) / 256, 8LL * sm_count()));
+  state_fold_kernel<<<grid, 256, 0, st>>>(state_in, parts, out, BH, s.H, s.dk * s.dv, n, part_stride, bh_stride,
+                                          hl, fl);
+  return launch_status();
+}
+
+// Segments of a state-only call: as many as the sequence split of the forward
+// call would use, fewer when the workspace (n_seg + 1 states per (b, h)) is
+// short.  Returns 0 when even one segment does not fit.
+int state_only_segments(const ret_shape& s, int C, size_t ws_bytes, int* seg_chunks) {
+  const size_t per = (size_t)s.B * s.H * s.dk * s.dv * sizeof(float);
+  const int n_chunks = (s.L + C - 1) / C;
+  int n_seg = 1, sc = 1;
+  plan_segments(s, C, &n_seg, &sc);
+  n_seg = std::max(1, std::min(n_seg, kFoldMaxParts));
+  while (n_seg > 1 && (size_t)(n_seg + 1) * per > ws_bytes) --n_seg;
+  if ((size_t)(n_seg + 1) * per > ws_bytes) return 0;
+  *seg_chunks = (n_chunks + n_seg - 1) / n_seg;
+  return (n_chunks + *seg_chunks - 1) / *seg_chunks;
+}
+
+// State-only chunkwise pass on the tensor cores: chunk_state_kernel writes each
+// segment's sum D_g to slot g + 1 of the workspace [BH][n_seg + 1][dk][dv], and
+// the fold joins them with state_in.
+template <int DK>
+ret_status launch_chunk_state(const void* k, const void* v, const float* gamma, const float* state_in,
+                              float* state_out, int C, const ret_shape& s, void* ws, size_t ws_bytes,
+                              cudaStream_t st) {
+  const int BH = s.B * s.H;
+  int seg_chunks = 1;
+  const int n_seg = state_only_segments(s, C, ws_bytes, &seg_chunks);
+  if (n_seg == 0 || !ws) return RET_EINVAL;
+  CUtensorMap mk, mv;
+  if (!make_map(&mk, k, DK, s.L, BH, C) || !make_map(&mv, v, s.dv, s.L, BH, C)) return RET_ECUDA;
+  static CwDecay dec;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  fill_l2g(dec, gamma, s.H);
+  const int smax = max_smem_optin();
+  const uint32_t per = (uint32_t)(DK / 64) * C * 128 + 2u * C * 128;
+  int ns = 0;
+  for (int n = kCW_MaxStages; n >= 1; --n)
+    if ((int)(n * per + kMiscBytes + kSmemAlign) <= smax) { ns = n; break; }
+  if (ns == 0) return RET_EUNSUPPORTED;
+  CwArgs a{};
+  a.B = s.B;
+  a.H = s.H;
+  a.L = s.L;
+  a.dv = s.dv;
+  a.C = C;
+  a.seg_chunks = seg_chunks;
+  a.n_seg = n_seg + 1;  // slot stride: slot 0 unused, segment g -> slot g + 1
+  a.nstages = ns;
+  a.lim = wait_limit();
+  a.debug_drop_block = -1;
+  const int smem = (int)(ns * per + kMiscBytes + kSmemAlign);
+  if (cudaFuncSetAttribute(chunk_state_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return RET_ECUDA;
+  dim3 grid(s.dv / kCW_DVT, BH, n_seg);
+  chunk_state_kernel<DK><<<grid, kCW_Threads, smem, st>>>(mk, mv, a, dec, static_cast<float*>(ws));
+  if (launch_status() != RET_OK) return RET_ECUDA;
+  int lens[kFoldMaxParts];
+  for (int g = 0; g < n_seg; ++g) lens[g] = std::min(s.L, (g + 1) * seg_chunks * C) - g * seg_chunks * C;
+  const long long dkdv = (long long)DK * s.dv;
+  return launch_state_fold(state_in, static_cast<const float*>(ws) + dkdv, state_out, s, gamma, n_seg, lens, dkdv,
+                           (long long)(n_seg + 1) * dkdv, st);
 }
 
 template <int DK, int DVT>
@@ -628,6 +708,80 @@ ret_status retention_chunkwise(const void* q, const void* k, const void* v, cons
     case 128: return launch_chunkwise_tc<128>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
     default: return launch_chunkwise_tc<256>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
   }
+}
+
+size_t retention_chunkwise_state_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
+  if (check_shape(s, true) != RET_OK || chunk < 1 || dt != RET_BF16 || s.L == 0) return 0;
+  if (!tc_chunk_ok(chunk, s.dk) || !tc_shape_ok(s)) return 0;
+  int n_seg = 1, sc = 1;
+  plan_segments(s, chunk, &n_seg, &sc);
+  n_seg = std::max(1, std::min(n_seg, kFoldMaxParts));
+  return (size_t)(n_seg + 1) * s.B * s.H * s.dk * s.dv * sizeof(float);
+}
+
+ret_status retention_chunkwise_state(const void* k, const void* v, const float* gamma, const float* state_in,
+                                     float* state_out, int chunk, ret_shape s, ret_dtype dt, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  ret_status rc = check_shape(s, true);
+  if (rc != RET_OK) return rc;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (chunk < 1) return RET_EINVAL;
+  if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
+  if (!state_out || !aligned16(state_out) || (state_in && !aligned16(state_in))) return RET_EINVAL;
+  if (s.L > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return RET_EINVAL;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RET_EINVAL;
+  if (dt == RET_F32) {
+    if (chunk > kCF_MaxC || s.dk > 256) return RET_EUNSUPPORTED;
+  } else {
+    if (!tc_chunk_ok(chunk, s.dk) || !tc_shape_ok(s)) return RET_EUNSUPPORTED;
+    if (s.L > 0 && !device_is_sm100()) return RET_EUNSUPPORTED;
+    if (s.L > 0 && (!workspace || workspace_bytes < (size_t)2 * s.B * s.H * s.dk * s.dv * sizeof(float)))
+      return RET_EINVAL;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.L == 0) {  // the state passes through
+    const size_t sbytes = (size_t)s.B * s.H * s.dk * s.dv * sizeof(float);
+    cudaError_t e = state_in ? (state_in == state_out ? cudaSuccess
+                                                      : cudaMemcpyAsync(state_out, state_in, sbytes,
+                                                                        cudaMemcpyDeviceToDevice, st))
+                             : cudaMemsetAsync(state_out, 0, sbytes, st);
+    return e == cudaSuccess ? RET_OK : RET_ECUDA;
+  }
+  if (dt == RET_F32) {  // the fp32 chunkwise kernel without its output (q unused)
+    static HeadLog2 hl;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int h = 0; h < s.H; ++h) hl.l2g[h] = log2_gamma(gamma[h]);
+    const int smem = (s.dk * kCF_Cols + chunk * (chunk + 1) + chunk + 1) * 4;
+    if (cudaFuncSetAttribute(chunkwise_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return RET_ECUDA;
+    dim3 grid((s.dv + kCF_Cols - 1) / kCF_Cols, s.B * s.H);
+    chunkwise_f32_kernel<<<grid, 256, smem, st>>>(static_cast<const float*>(k), static_cast<const float*>(k),
+                                                  static_cast<const float*>(v), nullptr, state_in, state_out, s.H,
+                                                  s.L, s.dk, s.dv, chunk, hl);
+    return launch_status();
+  }
+  switch (s.dk) {
+    case 64: return launch_chunk_state<64>(k, v, gamma, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+    case 128: return launch_chunk_state<128>(k, v, gamma, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+    default: return launch_chunk_state<256>(k, v, gamma, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+  }
+}
+
+ret_status retention_state_fold(const float* parts, const int* lens, int n, const float* gamma,
+                                const float* state_in, float* state_out, ret_shape s, void* stream) {
+  ret_status rc = check_shape(s, false);
+  if (rc != RET_OK) return rc;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (n < 0 || n > kFoldMaxParts || !state_out) return RET_EINVAL;
+  if (n > 0 && (!parts || !lens)) return RET_EINVAL;
+  for (int i = 0; i < n; ++i)
+    if (lens[i] < 0) return RET_EINVAL;
+  if ((parts && !aligned16(parts)) || !aligned16(state_out) || (state_in && !aligned16(state_in)))
+    return RET_EINVAL;
+  const long long per = (long long)s.B * s.H * s.dk * s.dv;
+  return launch_state_fold(state_in, parts, state_out, s, gamma, n, lens, per, (long long)s.dk * s.dv,
+                           static_cast<cudaStream_t>(stream));
 }
 
 // Chunkwise form with the sequence-split scratch taken from g_static_ws

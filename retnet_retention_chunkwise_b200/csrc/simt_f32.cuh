@@ -98,7 +98,8 @@ parallel_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
 //   y_{t0+i} = sum_{j<=i} gamma^(i-j) (q_i.k_j) v_j + gamma^(i+1) q_i S
 //   S       <- gamma^l S + sum_{j<l} gamma^(l-1-j) k_j^T v_j
 // CTA = (32-column block of the state / y, (b,h)); the state block [dk][32]
-// stays in shared memory for the whole sequence.
+// stays in shared memory for the whole sequence.  With y null only the state is
+// carried (q is not read).
 constexpr int kCF_Cols = 32;
 constexpr int kCF_MaxC = 128;
 
@@ -128,8 +129,8 @@ chunkwise_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
 
   for (int t0 = 0; t0 < L; t0 += C) {
     const int l = min(C, L - t0);
-    // 1. decayed, masked scores P[i][j] = gamma^(i-j) q_i.k_j (j <= i)
-    for (int e = tid; e < l * l; e += 256) {
+    // 1. decayed, masked scores P[i][j] = gamma^(i-j) q_i.k_j (j <= i), for y
+    for (int e = tid; y && e < l * l; e += 256) {
       const int i = e / l, j = e % l;
       float s = 0.f;
       if (j <= i) {
@@ -141,8 +142,9 @@ chunkwise_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
       Ps[i * (C + 1) + j] = s;
     }
     __syncthreads();
-    // 2. outputs: intra-block term + decayed cross-block term from the carried state
-    for (int e = tid; e < l * kCF_Cols; e += 256) {
+    // 2. outputs: intra-block term + decayed cross-block term from the carried
+    // state (skipped when only the state is wanted: y null, uniform per CTA)
+    for (int e = tid; y && e < l * kCF_Cols; e += 256) {
       const int i = e / kCF_Cols, c = e % kCF_Cols;
       if (c0 + c >= dv) continue;
       float a = 0.f;

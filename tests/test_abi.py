@@ -208,3 +208,34 @@ def test_groupnorm_gated_validation(lib):
                                          None) == _abi.RET_EINVAL  # eps < 0
     assert lib.retention_groupnorm_gated(FAKE, FAKE, FAKE, 1e-5, None, None, 1, _abi.RetShape(1, 2, 8, 1, 2048),
                                          _abi.RET_BF16, None) == _abi.RET_EUNSUPPORTED
+
+
+def test_chunkwise_state_and_fold_validation(lib):
+    # every case below returns before any launch
+    s = _abi.RetShape(1, 2, 256, 128, 128)
+    g = _g(0.5, 0.9)
+    need = lib.retention_chunkwise_state_workspace_bytes(64, s, _abi.RET_BF16)
+    assert need >= 2 * 2 * 128 * 128 * 4                      # at least two states per (b, h)
+    assert lib.retention_chunkwise_state_workspace_bytes(64, s, _abi.RET_F32) == 0
+    assert lib.retention_chunkwise_state_workspace_bytes(64, _abi.RetShape(1, 2, 256, 96, 128), _abi.RET_BF16) == 0
+    ws = ctypes.c_void_p(0x100000)
+    call = lambda out=FAKE, s_in=None, chunk=64, shape=s, dt=_abi.RET_BF16, w=ws, nb=need: (  # noqa: E731
+        lib.retention_chunkwise_state(FAKE, FAKE, g, s_in, out, chunk, shape, dt, w, nb, None))
+    assert call(out=None) == _abi.RET_EINVAL                   # state_out is required
+    assert call(out=ctypes.c_void_p(0x10004)) == _abi.RET_EINVAL
+    assert call(s_in=ctypes.c_void_p(0x10008)) == _abi.RET_EINVAL
+    assert call(chunk=0) == _abi.RET_EINVAL
+    assert call(w=ctypes.c_void_p(0x100040)) == _abi.RET_EINVAL  # workspace not 256-byte aligned
+    assert call(shape=_abi.RetShape(1, 2, 256, 96, 128)) == _abi.RET_EUNSUPPORTED
+    assert call(dt=_abi.RET_F32, chunk=256) == _abi.RET_EUNSUPPORTED
+    # fold
+    lens = (ctypes.c_int * 3)(10, 20, 30)
+    fold = lambda parts=FAKE, ln=lens, n=3, out=FAKE: lib.retention_state_fold(  # noqa: E731
+        parts, ln, n, g, None, out, s, None)
+    assert fold(n=257) == _abi.RET_EINVAL                      # at most 256 parts
+    assert fold(n=-1) == _abi.RET_EINVAL
+    assert fold(parts=None) == _abi.RET_EINVAL
+    assert fold(ln=None) == _abi.RET_EINVAL
+    assert fold(ln=(ctypes.c_int * 3)(10, -1, 30)) == _abi.RET_EINVAL
+    assert fold(out=None) == _abi.RET_EINVAL
+    assert fold(parts=ctypes.c_void_p(0x10004)) == _abi.RET_EINVAL
