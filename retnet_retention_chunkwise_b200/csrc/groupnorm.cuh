@@ -74,9 +74,12 @@ __device__ __forceinline__ void gn_store8(__nv_bfloat16* p, const float (&x)[8])
 
 enum GateAct { kGateNone = 0, kGateSwish = 1, kGateSigmoid = 2 };
 
+// sigmoid through the fast exponential and divide (a few ulp; the result is
+// rounded to the output dtype next).  -x is capped at 80 so that 1 + e^-x stays
+// finite and far below the divide's 2^126 range limit; sigmoid(-80) = 1.8e-35.
 __device__ __forceinline__ float gate_act(float x, int act) {
   if (act == kGateNone) return x;
-  const float sg = 1.f / (1.f + expf(-x));
+  const float sg = __fdividef(1.f, 1.f + __expf(fminf(-x, 80.f)));
   return act == kGateSwish ? x * sg : sg;
 }
 
@@ -103,7 +106,7 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
   const T* yr = y + row * dv;
   const T* gr = gate ? gate + row * dv : nullptr;
   T* orow = out + row * dv;
-  float x[kSteps][VEC];
+  float x[kSteps][VEC], gv[kSteps][VEC];
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < kSteps; ++i) {
@@ -111,12 +114,16 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
 #pragma unroll
     for (int e = 0; e < VEC; ++e) x[i][e] = 0.f;
     if (c < dv) {
+      // the gate values are loaded here, with y, so both reads are in flight together
       if constexpr (VEC == 8) {
         gn_load8(yr + c, x[i]);
+        if (gr) gn_load8(gr + c, gv[i]);
       } else if constexpr (VEC == 4) {
         gn_load4<T>(yr + c, x[i]);
+        if (gr) gn_load4<T>(gr + c, gv[i]);
       } else {
         x[i][0] = (float)yr[c];
+        if (gr) gv[i][0] = (float)gr[c];
       }
 #pragma unroll
       for (int e = 0; e < VEC; ++e) s += x[i][e];
@@ -149,16 +156,8 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
         if (br) z[e] += br[c + e];
       }
       if (gr) {
-        float gv[VEC];
-        if constexpr (VEC == 8) {
-          gn_load8(gr + c, gv);
-        } else if constexpr (VEC == 4) {
-          gn_load4<T>(gr + c, gv);
-        } else {
-          gv[0] = (float)gr[c];
-        }
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) z[e] *= gate_act(gv[e], act);
+        for (int e = 0; e < VEC; ++e) z[e] *= gate_act(gv[i][e], act);
       }
       if constexpr (VEC == 8) {
         gn_store8(orow + c, z);

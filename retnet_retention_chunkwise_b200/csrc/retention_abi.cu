@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -288,15 +289,20 @@ ret_status launch_state_fold(const float* state_in, const float* parts, float* o
   return launch_status();
 }
 
-// Segments of a state-only call: as many as the sequence split of the forward
-// call would use, fewer when the workspace (n_seg + 1 states per (b, h)) is
-// short.  Returns 0 when even one segment does not fit.
-int state_only_segments(const ret_shape& s, int C, size_t ws_bytes, int* seg_chunks) {
+// Plan of a state-only call.  Its result does not depend on the block length
+// (every row of K is scaled by its own decay to the segment end, and the sums
+// accumulate in fp32 across blocks), so it runs blocks of kStateC rows, which
+// keep four stages or two CTAs per SM in flight, and enough segments for about
+// two CTAs per SM; fewer when the workspace (n_seg + 1 states per (b, h)) is
+// short.  Returns n_seg, 0 when even one segment does not fit.
+constexpr int kStateC = 64;
+
+int state_only_segments(const ret_shape& s, size_t ws_bytes, int* seg_chunks) {
   const size_t per = (size_t)s.B * s.H * s.dk * s.dv * sizeof(float);
-  const int n_chunks = (s.L + C - 1) / C;
-  int n_seg = 1, sc = 1;
-  plan_segments(s, C, &n_seg, &sc);
-  n_seg = std::max(1, std::min(n_seg, kFoldMaxParts));
+  const int n_chunks = (s.L + kStateC - 1) / kStateC;
+  const long long base = (long long)(s.dv / kCW_DVT) * s.B * s.H;  // CTAs per segment
+  int n_seg = (int)std::max<long long>(1, (2LL * sm_count()) / base);
+  n_seg = std::max(1, std::min({n_seg, std::max(1, n_chunks / 2), kFoldMaxParts}));
   while (n_seg > 1 && (size_t)(n_seg + 1) * per > ws_bytes) --n_seg;
   if ((size_t)(n_seg + 1) * per > ws_bytes) return 0;
   *seg_chunks = (n_chunks + n_seg - 1) / n_seg;
@@ -308,11 +314,10 @@ int state_only_segments(const ret_shape& s, int C, size_t ws_bytes, int* seg_chu
 // the fold joins them with state_in.
 template <int DK>
 ret_status launch_chunk_state(const void* k, const void* v, const float* gamma, const float* state_in,
-                              float* state_out, int C, const ret_shape& s, void* ws, size_t ws_bytes,
-                              cudaStream_t st) {
-  const int BH = s.B * s.H;
+                              float* state_out, const ret_shape& s, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int BH = s.B * s.H, C = kStateC;
   int seg_chunks = 1;
-  const int n_seg = state_only_segments(s, C, ws_bytes, &seg_chunks);
+  const int n_seg = state_only_segments(s, ws_bytes, &seg_chunks);
   if (n_seg == 0 || !ws) return RET_EINVAL;
   CUtensorMap mk, mv;
   if (!make_map(&mk, k, DK, s.L, BH, C) || !make_map(&mv, v, s.dv, s.L, BH, C)) return RET_ECUDA;
@@ -322,8 +327,11 @@ ret_status launch_chunk_state(const void* k, const void* v, const float* gamma, 
   fill_l2g(dec, gamma, s.H);
   const int smax = max_smem_optin();
   const uint32_t per = (uint32_t)(DK / 64) * C * 128 + 2u * C * 128;
+  // two stages per CTA when two CTAs per SM are wanted and fit, else as many as fit
   int ns = 0;
-  for (int n = kCW_MaxStages; n >= 1; --n)
+  const long long ctas = (long long)(s.dv / kCW_DVT) * BH * n_seg;
+  const int cap = (ctas > sm_count() && 2 * (int)(2 * per + kMiscBytes + kSmemAlign) <= smax) ? 2 : kCW_MaxStages;
+  for (int n = cap; n >= 1; --n)
     if ((int)(n * per + kMiscBytes + kSmemAlign) <= smax) { ns = n; break; }
   if (ns == 0) return RET_EUNSUPPORTED;
   CwArgs a{};
@@ -713,9 +721,8 @@ ret_status retention_chunkwise(const void* q, const void* k, const void* v, cons
 size_t retention_chunkwise_state_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
   if (check_shape(s, true) != RET_OK || chunk < 1 || dt != RET_BF16 || s.L == 0) return 0;
   if (!tc_chunk_ok(chunk, s.dk) || !tc_shape_ok(s)) return 0;
-  int n_seg = 1, sc = 1;
-  plan_segments(s, chunk, &n_seg, &sc);
-  n_seg = std::max(1, std::min(n_seg, kFoldMaxParts));
+  int sc = 1;
+  const int n_seg = state_only_segments(s, SIZE_MAX, &sc);
   return (size_t)(n_seg + 1) * s.B * s.H * s.dk * s.dv * sizeof(float);
 }
 
@@ -762,9 +769,9 @@ ret_status retention_chunkwise_state(const void* k, const void* v, const float* 
     return launch_status();
   }
   switch (s.dk) {
-    case 64: return launch_chunk_state<64>(k, v, gamma, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
-    case 128: return launch_chunk_state<128>(k, v, gamma, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
-    default: return launch_chunk_state<256>(k, v, gamma, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+    case 64: return launch_chunk_state<64>(k, v, gamma, state_in, state_out, s, workspace, workspace_bytes, st);
+    case 128: return launch_chunk_state<128>(k, v, gamma, state_in, state_out, s, workspace, workspace_bytes, st);
+    default: return launch_chunk_state<256>(k, v, gamma, state_in, state_out, s, workspace, workspace_bytes, st);
   }
 }
 
