@@ -119,17 +119,20 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, WaitL
 }
 
 // Scale the 128-byte row r of a 128B-swizzled bf16 tile in place by f.
+// Multiply the 8 bf16 values of one 16-byte chunk of shared memory by f.
+__device__ __forceinline__ void scale_chunk_bf16x8(uint8_t* at, float f) {
+  uint4* p = reinterpret_cast<uint4*>(at);
+  uint4 w = *p;
+  w.x = pack_bf16x2(bf16lo_to_f32(w.x) * f, bf16hi_to_f32(w.x) * f);
+  w.y = pack_bf16x2(bf16lo_to_f32(w.y) * f, bf16hi_to_f32(w.y) * f);
+  w.z = pack_bf16x2(bf16lo_to_f32(w.z) * f, bf16hi_to_f32(w.z) * f);
+  w.w = pack_bf16x2(bf16lo_to_f32(w.w) * f, bf16hi_to_f32(w.w) * f);
+  *p = w;
+}
+
 __device__ __forceinline__ void scale_row_sw128(uint8_t* tile, uint32_t r, float f) {
 #pragma unroll
-  for (uint32_t c = 0; c < 8; ++c) {
-    uint4* p = reinterpret_cast<uint4*>(tile + sw128_off(r, c));
-    uint4 w = *p;
-    w.x = pack_bf16x2(bf16lo_to_f32(w.x) * f, bf16hi_to_f32(w.x) * f);
-    w.y = pack_bf16x2(bf16lo_to_f32(w.y) * f, bf16hi_to_f32(w.y) * f);
-    w.z = pack_bf16x2(bf16lo_to_f32(w.z) * f, bf16hi_to_f32(w.z) * f);
-    w.w = pack_bf16x2(bf16lo_to_f32(w.w) * f, bf16hi_to_f32(w.w) * f);
-    *p = w;
-  }
+  for (uint32_t c = 0; c < 8; ++c) scale_chunk_bf16x8(tile + sw128_off(r, c), f);
 }
 
 // Write 32 floats as bf16 into row r, columns [c0, c0+32) of a 128B-swizzled
@@ -1149,7 +1152,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
 // Segment sums for the sequence split: for segment g of one (b, h) and one
 // 128-column dv slice,  D_g^T = sum_{t in g} gamma^(e_g - t) v_t^T k_t  with e_g
 // the segment's last token, written (as [dk][dv], like a state) to slot g+1 of
-// the workspace [BH][n_seg][dk][dv].  Rows of K are scaled by the decay to the
+// the workspace [BH][n_seg][dk][dv].  Rows of V are scaled by the decay to the
 // segment end in shared memory, then accumulated by tcgen05 into TMEM.
 template <int DK>
 __global__ void __launch_bounds__(kCW_Threads)
@@ -1165,7 +1168,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + NS * (k_stage + v_stage));
   uint64_t* full = bars;        // [4]
   uint64_t* empty = bars + 4;   // [4]
-  uint64_t* kready = bars + 8;  // [4] epilogue scaled K -> MMA
+  uint64_t* kready = bars + 8;  // [4] epilogue scaled the V rows -> MMA
   uint64_t* done = bars + 12;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13) + 1;
@@ -1239,10 +1242,15 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
     for (int it = 0; it < nck; ++it) {
       const int s = it % NS;
       if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) { ok = false; break; }
-      for (uint32_t j = r; j < (uint32_t)C; j += 128) {  // rows j and j + 128 (blocks up to 256)
+      // Row j of V times gamma^(e_g - t): 2 boxes x 8 chunks of 16 bytes per row,
+      // one chunk per thread and step.  A row's chunks share its factor, so the
+      // swizzle (a permutation within the row) plays no part.
+      uint8_t* vs = sV + s * v_stage;
+      for (uint32_t e = r; e < (uint32_t)C * 16u; e += 128) {
+        const uint32_t j = e >> 4;
         const int t = (c_begin + it) * C + (int)j;
         const float f = (t <= seg_last) ? (t == seg_last ? 1.f : exp2f((float)(seg_last - t) * l2g)) : 0.f;
-        for (int b = 0; b < DK / 64; ++b) scale_row_sw128(sK + s * k_stage + b * C * 128, j, f);
+        scale_chunk_bf16x8(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u + (e & 7u) * 16u, f);
       }
       fence_proxy_async_smem();
       mbar_arrive(&kready[s]);

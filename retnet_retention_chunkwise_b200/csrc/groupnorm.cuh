@@ -91,25 +91,25 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // One warp per (b, h, n) row.  Vectorised (VEC values per lane per step: 8
 // for bf16 when dv % 256 == 0, 4 when dv % 128 == 0), else one value per lane
-// per step; dv <= 1024.  out may alias y.  gate: null, or act(gate) multiplies
-// the result.
-template <typename T, int VEC>
+// per step; STEPS steps cover dv (<= 1024), so the row lives in VEC * STEPS
+// registers per lane (x2 with the gate).  out may alias y.  GATE: act(gate)
+// multiplies the result.
+template <typename T, int VEC, int STEPS, bool GATE>
 __global__ void __launch_bounds__(32 * kGN_RowsPerBlock)
 groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, float eps,
                       const float* __restrict__ w, const float* __restrict__ bias, const T* __restrict__ gate,
                       int act) {
-  constexpr int kSteps = kGN_MaxDv / (32 * VEC);
   const int lane = threadIdx.x & 31;
   const long long row = (long long)blockIdx.x * kGN_RowsPerBlock + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int h = (int)((row / L) % H);
   const T* yr = y + row * dv;
-  const T* gr = gate ? gate + row * dv : nullptr;
+  const T* gr = GATE ? gate + row * dv : nullptr;
   T* orow = out + row * dv;
-  float x[kSteps][VEC], gv[kSteps][VEC];
+  float x[STEPS][VEC], gv[GATE ? STEPS : 1][VEC];
   float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < kSteps; ++i) {
+  for (int i = 0; i < STEPS; ++i) {
     const int c = (i * 32 + lane) * VEC;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) x[i][e] = 0.f;
@@ -117,13 +117,13 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
       // the gate values are loaded here, with y, so both reads are in flight together
       if constexpr (VEC == 8) {
         gn_load8(yr + c, x[i]);
-        if (gr) gn_load8(gr + c, gv[i]);
+        if constexpr (GATE) gn_load8(gr + c, gv[i]);
       } else if constexpr (VEC == 4) {
         gn_load4<T>(yr + c, x[i]);
-        if (gr) gn_load4<T>(gr + c, gv[i]);
+        if constexpr (GATE) gn_load4<T>(gr + c, gv[i]);
       } else {
         x[i][0] = (float)yr[c];
-        if (gr) gv[i][0] = (float)gr[c];
+        if constexpr (GATE) gv[i][0] = (float)gr[c];
       }
 #pragma unroll
       for (int e = 0; e < VEC; ++e) s += x[i][e];
@@ -132,7 +132,7 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
   const float mean = warp_sum(s) / (float)dv;
   float q = 0.f;
 #pragma unroll
-  for (int i = 0; i < kSteps; ++i) {
+  for (int i = 0; i < STEPS; ++i) {
     if ((i * 32 + lane) * VEC < dv) {
 #pragma unroll
       for (int e = 0; e < VEC; ++e) {
@@ -145,7 +145,7 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
   const float* wr = w ? w + (size_t)h * dv : nullptr;
   const float* br = bias ? bias + (size_t)h * dv : nullptr;
 #pragma unroll
-  for (int i = 0; i < kSteps; ++i) {
+  for (int i = 0; i < STEPS; ++i) {
     const int c = (i * 32 + lane) * VEC;
     if (c < dv) {
       float z[VEC];
@@ -155,7 +155,7 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
         if (wr) z[e] *= wr[c + e];
         if (br) z[e] += br[c + e];
       }
-      if (gr) {
+      if constexpr (GATE) {
 #pragma unroll
         for (int e = 0; e < VEC; ++e) z[e] *= gate_act(gv[i][e], act);
       }
@@ -168,6 +168,21 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
       }
     }
   }
+}
+
+// Launch with the fewest steps (a power of two) that cover dv.
+template <typename T, int VEC, bool GATE, int STEPS = 1>
+void launch_groupnorm_rows(unsigned blocks, cudaStream_t st, const T* y, T* out, long long rows, int H, int L,
+                           int dv, float eps, const float* w, const float* b, const T* gate, int act) {
+  constexpr int kMax = kGN_MaxDv / (32 * VEC);
+  if constexpr (STEPS < kMax) {
+    if (dv > 32 * VEC * STEPS) {
+      launch_groupnorm_rows<T, VEC, GATE, 2 * STEPS>(blocks, st, y, out, rows, H, L, dv, eps, w, b, gate, act);
+      return;
+    }
+  }
+  groupnorm_rows_kernel<T, VEC, STEPS, GATE>
+      <<<blocks, 32 * kGN_RowsPerBlock, 0, st>>>(y, out, rows, H, L, dv, eps, w, b, gate, act);
 }
 
 }  // namespace ret

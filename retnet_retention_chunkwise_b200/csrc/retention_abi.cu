@@ -394,6 +394,18 @@ ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const
   return launch_status();
 }
 
+template <typename T, int VEC>
+void launch_groupnorm_vec(unsigned blocks, cudaStream_t st, const void* y, void* out, long long rows,
+                          const ret_shape& s, float eps, const float* w, const float* b, const void* gate, int act) {
+  auto yi = static_cast<const T*>(y);
+  auto yo = static_cast<T*>(out);
+  auto gi = static_cast<const T*>(gate);
+  if (gate)
+    launch_groupnorm_rows<T, VEC, true>(blocks, st, yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
+  else
+    launch_groupnorm_rows<T, VEC, false>(blocks, st, yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
+}
+
 ret_status launch_groupnorm(const void* y, void* out, float eps, const float* w, const float* b,
                             const ret_shape& s, ret_dtype dt, cudaStream_t st, const void* gate = nullptr,
                             int act = 0) {
@@ -401,26 +413,18 @@ ret_status launch_groupnorm(const void* y, void* out, float eps, const float* w,
   if (rows == 0) return RET_OK;
   const unsigned blocks = (unsigned)((rows + kGN_RowsPerBlock - 1) / kGN_RowsPerBlock);
   const bool vec = s.dv % 128 == 0;
-  const int thr = 32 * kGN_RowsPerBlock;
   if (dt == RET_BF16) {
-    using T = __nv_bfloat16;
-    auto yi = static_cast<const T*>(y);
-    auto yo = static_cast<T*>(out);
-    auto gi = static_cast<const T*>(gate);
     if (s.dv % 256 == 0)
-      groupnorm_rows_kernel<T, 8><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
+      launch_groupnorm_vec<__nv_bfloat16, 8>(blocks, st, y, out, rows, s, eps, w, b, gate, act);
     else if (vec)
-      groupnorm_rows_kernel<T, 4><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
+      launch_groupnorm_vec<__nv_bfloat16, 4>(blocks, st, y, out, rows, s, eps, w, b, gate, act);
     else
-      groupnorm_rows_kernel<T, 1><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
+      launch_groupnorm_vec<__nv_bfloat16, 1>(blocks, st, y, out, rows, s, eps, w, b, gate, act);
   } else {
-    auto yi = static_cast<const float*>(y);
-    auto yo = static_cast<float*>(out);
-    auto gi = static_cast<const float*>(gate);
     if (vec)
-      groupnorm_rows_kernel<float, 4><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
+      launch_groupnorm_vec<float, 4>(blocks, st, y, out, rows, s, eps, w, b, gate, act);
     else
-      groupnorm_rows_kernel<float, 1><<<blocks, thr, 0, st>>>(yi, yo, rows, s.H, s.L, s.dv, eps, w, b, gi, act);
+      launch_groupnorm_vec<float, 1>(blocks, st, y, out, rows, s, eps, w, b, gate, act);
   }
   return launch_status();
 }
