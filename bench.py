@@ -88,13 +88,22 @@ def load_peaks():
                 "source": "fallback (earlier measurement on this pool)"}
 
 
+# The headline kernel's source: chunkwise_tc.cuh up to the start of the
+# sequence-split helpers that follow chunkwise_tc256_kernel (everything the
+# kernel can use is declared above it), plus tc_common.cuh.
+HEADLINE_SOURCE_END = b"// Segment sums for the sequence split"
+
+
 def kernel_source_digest():
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "retnet_retention_chunkwise_b200", "csrc")
-    for f in ("chunkwise_tc.cuh", "tc_common.cuh"):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(fh.read())
+    with open(os.path.join(d, "chunkwise_tc.cuh"), "rb") as fh:
+        src = fh.read()
+    cut = src.find(HEADLINE_SOURCE_END)
+    h.update(src if cut < 0 else src[:cut])
+    with open(os.path.join(d, "tc_common.cuh"), "rb") as fh:
+        h.update(fh.read())
     return h.hexdigest()[:16]
 
 

@@ -119,20 +119,17 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, WaitL
 }
 
 // Scale the 128-byte row r of a 128B-swizzled bf16 tile in place by f.
-// Multiply the 8 bf16 values of one 16-byte chunk of shared memory by f.
-__device__ __forceinline__ void scale_chunk_bf16x8(uint8_t* at, float f) {
-  uint4* p = reinterpret_cast<uint4*>(at);
-  uint4 w = *p;
-  w.x = pack_bf16x2(bf16lo_to_f32(w.x) * f, bf16hi_to_f32(w.x) * f);
-  w.y = pack_bf16x2(bf16lo_to_f32(w.y) * f, bf16hi_to_f32(w.y) * f);
-  w.z = pack_bf16x2(bf16lo_to_f32(w.z) * f, bf16hi_to_f32(w.z) * f);
-  w.w = pack_bf16x2(bf16lo_to_f32(w.w) * f, bf16hi_to_f32(w.w) * f);
-  *p = w;
-}
-
 __device__ __forceinline__ void scale_row_sw128(uint8_t* tile, uint32_t r, float f) {
 #pragma unroll
-  for (uint32_t c = 0; c < 8; ++c) scale_chunk_bf16x8(tile + sw128_off(r, c), f);
+  for (uint32_t c = 0; c < 8; ++c) {
+    uint4* p = reinterpret_cast<uint4*>(tile + sw128_off(r, c));
+    uint4 w = *p;
+    w.x = pack_bf16x2(bf16lo_to_f32(w.x) * f, bf16hi_to_f32(w.x) * f);
+    w.y = pack_bf16x2(bf16lo_to_f32(w.y) * f, bf16hi_to_f32(w.y) * f);
+    w.z = pack_bf16x2(bf16lo_to_f32(w.z) * f, bf16hi_to_f32(w.z) * f);
+    w.w = pack_bf16x2(bf16lo_to_f32(w.w) * f, bf16hi_to_f32(w.w) * f);
+    *p = w;
+  }
 }
 
 // Write 32 floats as bf16 into row r, columns [c0, c0+32) of a 128B-swizzled
@@ -1243,14 +1240,40 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
       const int s = it % NS;
       if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) { ok = false; break; }
       // Row j of V times gamma^(e_g - t): 2 boxes x 8 chunks of 16 bytes per row,
-      // one chunk per thread and step.  A row's chunks share its factor, so the
-      // swizzle (a permutation within the row) plays no part.
+      // chunk e = 16 j + 8 box + c.  Each thread takes every 128th chunk, 8 at a
+      // time: all 8 loads first, then the products and the stores.  A row's
+      // chunks share its factor, so the swizzle (a permutation within the row)
+      // plays no part.
       uint8_t* vs = sV + s * v_stage;
-      for (uint32_t e = r; e < (uint32_t)C * 16u; e += 128) {
-        const uint32_t j = e >> 4;
-        const int t = (c_begin + it) * C + (int)j;
-        const float f = (t <= seg_last) ? (t == seg_last ? 1.f : exp2f((float)(seg_last - t) * l2g)) : 0.f;
-        scale_chunk_bf16x8(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u + (e & 7u) * 16u, f);
+      const uint32_t n_chunks = (uint32_t)C * 16u;
+      for (uint32_t e0 = r; e0 < n_chunks; e0 += 8u * 128u) {
+        uint4 w[8];
+        float f[8];
+#pragma unroll
+        for (uint32_t u = 0; u < 8; ++u) {
+          const uint32_t e = e0 + u * 128u;
+          if (e < n_chunks) {
+            const uint32_t j = e >> 4;
+            w[u] = *reinterpret_cast<const uint4*>(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u +
+                                                    (e & 7u) * 16u);
+            const int t = (c_begin + it) * C + (int)j;
+            f[u] = (t <= seg_last) ? (t == seg_last ? 1.f : exp2f((float)(seg_last - t) * l2g)) : 0.f;
+          }
+        }
+#pragma unroll
+        for (uint32_t u = 0; u < 8; ++u) {
+          const uint32_t e = e0 + u * 128u;
+          if (e < n_chunks) {
+            const uint32_t j = e >> 4;
+            const float g = f[u];
+            uint4 x = w[u];
+            x.x = pack_bf16x2(bf16lo_to_f32(x.x) * g, bf16hi_to_f32(x.x) * g);
+            x.y = pack_bf16x2(bf16lo_to_f32(x.y) * g, bf16hi_to_f32(x.y) * g);
+            x.z = pack_bf16x2(bf16lo_to_f32(x.z) * g, bf16hi_to_f32(x.z) * g);
+            x.w = pack_bf16x2(bf16lo_to_f32(x.w) * g, bf16hi_to_f32(x.w) * g);
+            *reinterpret_cast<uint4*>(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u + (e & 7u) * 16u) = x;
+          }
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(&kready[s]);
