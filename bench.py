@@ -116,7 +116,10 @@ def measured_traffic():
             for ln in f:
                 if ":" in ln and ln.strip().startswith("- "):
                     k, v = ln.strip()[2:].split(":", 1)
-                    kv[k.strip()] = v.strip().strip("`")
+                    v = v.strip()
+                    if v.startswith("`") and "`" in v[1:]:
+                        v = v[1:v.index("`", 1)]  # the first quoted token
+                    kv[k.strip()] = v
         if kv.get("kernel_source_sha256_16") != kernel_source_digest():
             return None
         return float(kv["dram_bytes_per_launch"])
