@@ -1149,8 +1149,9 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
 // Segment sums for the sequence split: for segment g of one (b, h) and one
 // 128-column dv slice,  D_g^T = sum_{t in g} gamma^(e_g - t) v_t^T k_t  with e_g
 // the segment's last token, written (as [dk][dv], like a state) to slot g+1 of
-// the workspace [BH][n_seg][dk][dv].  Rows of V are scaled by the decay to the
-// segment end in shared memory, then accumulated by tcgen05 into TMEM.
+// the workspace [BH][n_seg][dk][dv].  Rows of K (DK <= 128) or of V (DK = 256)
+// are scaled by the decay to the segment end in shared memory, then
+// accumulated by tcgen05 into TMEM.
 template <int DK>
 __global__ void __launch_bounds__(kCW_Threads)
 chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
@@ -1165,7 +1166,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + NS * (k_stage + v_stage));
   uint64_t* full = bars;        // [4]
   uint64_t* empty = bars + 4;   // [4]
-  uint64_t* kready = bars + 8;  // [4] epilogue scaled the V rows -> MMA
+  uint64_t* kready = bars + 8;  // [4] epilogue scaled the K or V rows -> MMA
   uint64_t* done = bars + 12;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13) + 1;
@@ -1239,39 +1240,48 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
     for (int it = 0; it < nck; ++it) {
       const int s = it % NS;
       if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) { ok = false; break; }
-      // Row j of V times gamma^(e_g - t): 2 boxes x 8 chunks of 16 bytes per row,
-      // chunk e = 16 j + 8 box + c.  Each thread takes every 128th chunk, 8 at a
-      // time: all 8 loads first, then the products and the stores.  A row's
-      // chunks share its factor, so the swizzle (a permutation within the row)
-      // plays no part.
-      uint8_t* vs = sV + s * v_stage;
-      const uint32_t n_chunks = (uint32_t)C * 16u;
-      for (uint32_t e0 = r; e0 < n_chunks; e0 += 8u * 128u) {
-        uint4 w[8];
-        float f[8];
-#pragma unroll
-        for (uint32_t u = 0; u < 8; ++u) {
-          const uint32_t e = e0 + u * 128u;
-          if (e < n_chunks) {
-            const uint32_t j = e >> 4;
-            w[u] = *reinterpret_cast<const uint4*>(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u +
-                                                    (e & 7u) * 16u);
-            const int t = (c_begin + it) * C + (int)j;
-            f[u] = (t <= seg_last) ? (t == seg_last ? 1.f : exp2f((float)(seg_last - t) * l2g)) : 0.f;
-          }
+      // Row j of the narrower operand times gamma^(e_g - t).  DK <= 128: rows
+      // of K, one row per thread.  DK = 256: rows of V (half the bytes of K's),
+      // 2 boxes x 8 chunks of 16 bytes per row, chunk e = 16 j + 8 box + c; each
+      // thread takes every 128th chunk, 8 at a time (all 8 loads first).  A
+      // row's chunks share its factor, so the swizzle (a permutation within the
+      // row) plays no part.
+      if constexpr (DK <= kCW_DVT) {
+        for (uint32_t j = r; j < (uint32_t)C; j += 128) {  // rows j and j + 128 (blocks up to 256)
+          const int t = (c_begin + it) * C + (int)j;
+          const float f = (t <= seg_last) ? (t == seg_last ? 1.f : exp2f((float)(seg_last - t) * l2g)) : 0.f;
+          for (int b = 0; b < DK / 64; ++b) scale_row_sw128(sK + s * k_stage + b * C * 128, j, f);
         }
+      } else {
+        uint8_t* vs = sV + s * v_stage;
+        const uint32_t n_chunks = (uint32_t)C * 16u;
+        for (uint32_t e0 = r; e0 < n_chunks; e0 += 8u * 128u) {
+          uint4 w[8];
+          float f[8];
 #pragma unroll
-        for (uint32_t u = 0; u < 8; ++u) {
-          const uint32_t e = e0 + u * 128u;
-          if (e < n_chunks) {
-            const uint32_t j = e >> 4;
-            const float g = f[u];
-            uint4 x = w[u];
-            x.x = pack_bf16x2(bf16lo_to_f32(x.x) * g, bf16hi_to_f32(x.x) * g);
-            x.y = pack_bf16x2(bf16lo_to_f32(x.y) * g, bf16hi_to_f32(x.y) * g);
-            x.z = pack_bf16x2(bf16lo_to_f32(x.z) * g, bf16hi_to_f32(x.z) * g);
-            x.w = pack_bf16x2(bf16lo_to_f32(x.w) * g, bf16hi_to_f32(x.w) * g);
-            *reinterpret_cast<uint4*>(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u + (e & 7u) * 16u) = x;
+          for (uint32_t u = 0; u < 8; ++u) {
+            const uint32_t e = e0 + u * 128u;
+            if (e < n_chunks) {
+              const uint32_t j = e >> 4;
+              w[u] = *reinterpret_cast<const uint4*>(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u +
+                                                      (e & 7u) * 16u);
+              const int t = (c_begin + it) * C + (int)j;
+              f[u] = (t <= seg_last) ? (t == seg_last ? 1.f : exp2f((float)(seg_last - t) * l2g)) : 0.f;
+            }
+          }
+#pragma unroll
+          for (uint32_t u = 0; u < 8; ++u) {
+            const uint32_t e = e0 + u * 128u;
+            if (e < n_chunks) {
+              const uint32_t j = e >> 4;
+              const float g = f[u];
+              uint4 x = w[u];
+              x.x = pack_bf16x2(bf16lo_to_f32(x.x) * g, bf16hi_to_f32(x.x) * g);
+              x.y = pack_bf16x2(bf16lo_to_f32(x.y) * g, bf16hi_to_f32(x.y) * g);
+              x.z = pack_bf16x2(bf16lo_to_f32(x.z) * g, bf16hi_to_f32(x.z) * g);
+              x.w = pack_bf16x2(bf16lo_to_f32(x.w) * g, bf16hi_to_f32(x.w) * g);
+              *reinterpret_cast<uint4*>(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u + (e & 7u) * 16u) = x;
+            }
           }
         }
       }
