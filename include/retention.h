@@ -180,8 +180,8 @@ RET_API size_t retention_chunkwise_state_workspace_bytes(int chunk, ret_shape s,
  * The same page and section: the state after a run is the decayed state before
  * it plus the run's own sum.  On a sequence cut across ranks, rank r folds the
  * parts of ranks 0 .. r-1 to get the state its own run starts from.
- * parts : device fp32 [n][B][H][dk][dv] (the D_i), 16-byte aligned; must not
- *         alias state_out.
+ * parts : device fp32 [n][B][H][dk][dv] (the D_i), 16-byte aligned; a
+ *         state_out that overlaps them is RET_EINVAL.
  * lens  : host int [n], each >= 0.  n in [0, 256].
  * state_in : device fp32 [B][H][dk][dv] or NULL (zero); state_out : device fp32,
  *         may alias state_in.  s.L is ignored.  Runs on `stream`.

@@ -791,6 +791,11 @@ ret_status retention_state_fold(const float* parts, const int* lens, int n, cons
   if ((parts && !aligned16(parts)) || !aligned16(state_out) || (state_in && !aligned16(state_in)))
     return RET_EINVAL;
   const long long per = (long long)s.B * s.H * s.dk * s.dv;
+  if (n > 0) {  // state_out must not overlap the parts (state_in may be state_out)
+    const uintptr_t p0 = reinterpret_cast<uintptr_t>(parts), p1 = p0 + (uintptr_t)n * per * sizeof(float);
+    const uintptr_t o0 = reinterpret_cast<uintptr_t>(state_out), o1 = o0 + (uintptr_t)per * sizeof(float);
+    if (o0 < p1 && p0 < o1) return RET_EINVAL;
+  }
   return launch_state_fold(state_in, parts, state_out, s, gamma, n, lens, per, (long long)s.dk * s.dv,
                            static_cast<cudaStream_t>(stream));
 }

@@ -239,3 +239,13 @@ def test_chunkwise_state_and_fold_validation(lib):
     assert fold(ln=(ctypes.c_int * 3)(10, -1, 30)) == _abi.RET_EINVAL
     assert fold(out=None) == _abi.RET_EINVAL
     assert fold(parts=ctypes.c_void_p(0x10004)) == _abi.RET_EINVAL
+
+
+def test_state_fold_rejects_out_inside_parts(lib):
+    s = _abi.RetShape(1, 2, 0, 16, 16)
+    lens = (ctypes.c_int * 2)(5, 7)
+    per = 2 * 16 * 16 * 4
+    parts = 0x100000
+    for out in (parts, parts + per, parts + per - 16, parts - per + 16):
+        assert lib.retention_state_fold(ctypes.c_void_p(parts), lens, 2, _g(0.5, 0.9), None, ctypes.c_void_p(out), s,
+                                        None) == _abi.RET_EINVAL, hex(out)
