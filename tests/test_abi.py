@@ -7,6 +7,7 @@
 import ctypes
 import os
 import re
+import tempfile
 
 import pytest
 
@@ -249,3 +250,22 @@ def test_state_fold_rejects_out_inside_parts(lib):
     for out in (parts, parts + per, parts + per - 16, parts - per + 16):
         assert lib.retention_state_fold(ctypes.c_void_p(parts), lens, 2, _g(0.5, 0.9), None, ctypes.c_void_p(out), s,
                                         None) == _abi.RET_EINVAL, hex(out)
+
+
+def test_plain_c_caller():
+    # the header compiles as C99 and the library links and answers from C
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.join(root, "retnet_retention_chunkwise_b200")
+    with tempfile.TemporaryDirectory() as tmp:
+        exe = os.path.join(tmp, "c_caller")
+        subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                        os.path.join(root, "tests", "c_caller.c"), "-o", exe, "-L", libdir, "-lretention",
+                        f"-Wl,-rpath,{libdir}"], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stdout + out.stderr
+    assert out.stdout.startswith("ok ")
