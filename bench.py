@@ -597,6 +597,20 @@ def run_profile_case(args):
         gam = inputs.multiscale_gammas(H)
         st = torch.zeros((B, H, dk, dv), dtype=torch.float32, device="cuda")
         fn = lambda: ret.recurrent_step(q, k, v, gam, st)  # noqa: E731
+    elif kind in ("groupnorm", "groupnorm_gated"):
+        B, H, L, dv = d
+        g = torch.Generator("cuda").manual_seed(0)
+        y = torch.randn((B, H, L, dv), generator=g, device="cuda").to(torch.bfloat16)
+        gate = torch.randn((B, H, L, dv), generator=g, device="cuda").to(torch.bfloat16)
+        if kind == "groupnorm":
+            fn = lambda: ret.groupnorm(y, 1e-5, out=y)  # noqa: E731
+        else:
+            fn = lambda: ret.groupnorm(y, 1e-5, out=y, gate=gate, act="swish")  # noqa: E731
+    elif kind == "state":
+        B, H, L, dk, dv, C = d
+        _, k, v = gpu_qkv(B, H, L, dk, dv, seed=0)
+        gam = inputs.multiscale_gammas(H)
+        fn = lambda: ret.chunkwise_state(k, v, gam, C)  # noqa: E731
     else:
         raise SystemExit(f"unknown profile kind {kind}")
     for _ in range(args.warmup):
@@ -622,7 +636,8 @@ def main():
     ap.add_argument("--no-forms", action="store_true", help="headline only")
     ap.add_argument("--profile", default=None,
                     help="run only one kind of call for a profiler, no JSON: "
-                         "chunkwise:B,H,L,dk,dv,C | parallel:B,H,L,dk,dv | decode:B,H,dk,dv")
+                         "chunkwise:B,H,L,dk,dv,C | parallel:B,H,L,dk,dv | decode:B,H,dk,dv | "
+                         "groupnorm:B,H,L,dv | groupnorm_gated:B,H,L,dv | state:B,H,L,dk,dv,C")
     args = ap.parse_args()
     if args.warmup < 3 and args.profile is None:
         args.warmup = 3
