@@ -193,6 +193,27 @@ def parallel_backward(q, k, v, gamma, dy, lib=None):
     return dq, dkk, dvv
 
 
+def state_backward(q, k, v, gamma, dy, state_in=None, dstate_out=None, lib=None):
+    """Only the terms a carried state adds to (dq, dk, dv), and dstate_in, in
+    fp64 (oracle_state_backward; linear in L, for long sequences)."""
+    lib = lib or load()
+    q, k, v, dy = _f64(q), _f64(k), _f64(v), _f64(dy)
+    gamma = _f64(gamma).reshape(-1)
+    B, H, L, dk = q.shape
+    dv = v.shape[-1]
+    s0 = None if state_in is None else _f64(state_in)
+    dso = None if dstate_out is None else _f64(dstate_out)
+    for t in (s0, dso):
+        if t is not None and t.shape != (B, H, dk, dv):
+            raise ValueError("oracle: state shape mismatch")
+    dq, dkk, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    ds0 = np.zeros((B, H, dk, dv))
+    if lib.oracle_state_backward(B, H, L, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(gamma), _ptr(dy), _ptr(s0),
+                                 _ptr(dso), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(ds0)) != 0:
+        raise ValueError("oracle_state_backward: invalid arguments")
+    return dq, dkk, dvv, ds0
+
+
 def backward(q, k, v, gamma, dy, state_in=None, dstate_out=None, lib=None):
     """Gradients (dq, dk, dv, dstate_in) of y and state_out with respect to q,
     k, v and state_in, for upstream dy and dstate_out (None: zero), in fp64.
