@@ -10,6 +10,8 @@ Also measured in the same run (same timing rules, reported under "forms"):
                 after a 512-token chunkwise prefill (6.7B-shaped heads);
   parallel   -- parallel form, B=2, H=8, L=2048, dk=64, dv=128 (MSR core);
   parallel_backward -- its gradients dq, dk, dv on the same shape;
+  decode_batch1_graph -- decode at batch 1, eager calls against the same
+                steps replayed from a CUDA graph;
   chunkwise_backward_long_context -- the gradients through the chunkwise form,
                 one 16384-token call of the long-context layout;
   chunkwise_backward_state_long_context -- the same with a carried state
@@ -377,6 +379,39 @@ def bench_decode(ret, args, dist, peaks):
             "gpu_launches": steps}
 
 
+def bench_decode_graph(ret, args, dist, peaks):
+    """Decode at batch 1 (one sequence, 6.7B-shaped heads): a step moves 16.8 MB
+    of state, a few microseconds of HBM time, so eager calls are bound by the
+    host.  The same steps captured once as a CUDA graph (graphs.DecodeGraph)
+    and replayed."""
+    from retnet_retention_chunkwise_b200.graphs import DecodeGraph
+    B, H, dk, dv, n = 1, 16, 256, 512, 64
+    gam = inputs.multiscale_gammas(H)
+    state = torch.zeros((B, H, dk, dv), dtype=torch.float32, device="cuda")
+    tq, tk, tv = gpu_qkv(n, B * H, 1, dk, dv, seed=1)
+    tq, tk, tv = (t.view(n, B, H, 1, -1) for t in (tq, tk, tv))
+    y = torch.empty((B, H, 1, dv), dtype=torch.bfloat16, device="cuda")
+
+    def eager():
+        for i in range(n):
+            ret.recurrent_step(tq[i], tk[i], tv[i], gam, state, out=y)
+
+    _, t_eager = time_calls(eager, 10, max(args.warmup, 3), dist)
+    g = DecodeGraph(state, gam, n)
+    g.q.copy_(tq)
+    g.k.copy_(tk)
+    g.v.copy_(tv)
+    _, t_graph = time_calls(g.replay, 10, max(args.warmup, 3), dist)
+    assert ret.device_status() == 0
+    e = dist.max(t_eager) / (10 * n)
+    gr = dist.max(t_graph) / (10 * n)
+    nbytes = B * H * (2 * dk * dv * 4 + (2 * dk + 2 * dv) * 2)
+    return {"workload": "decode at batch 1: B=1 H=16 dk=256 dv=512, 64 steps per graph",
+            "eager_ms_per_step": round(e, 4), "graph_ms_per_step": round(gr, 4),
+            "tokens_per_s_graph": dist.sum(B) / (gr * 1e-3),
+            "hbm_frac_graph": round(nbytes / (gr * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+
+
 def _shape_of(w):
     from retnet_retention_chunkwise_b200 import _abi
     return _abi.RetShape(w.B, w.H, w.L, w.dk, w.dv)
@@ -656,6 +691,7 @@ def main():
     forms = {}
     if not args.no_forms:
         forms["decode"] = bench_decode(ret, args, dist, peaks)
+        forms["decode_batch1_graph"] = bench_decode_graph(ret, args, dist, peaks)
         forms.update(bench_small(ret, args, dist, peaks))
     cpu = cpu_baseline() if (dist.rank == 0 and dist.world == 1) else None
     w = HEADLINE

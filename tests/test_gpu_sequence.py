@@ -140,3 +140,34 @@ def test_sequence_sharded_one_rank_nccl():
     finally:
         dist.destroy_process_group()
     assert ret.device_status() == 0
+
+
+def test_decode_graph_matches_eager_steps():
+    from retnet_retention_chunkwise_b200.graphs import DecodeGraph
+    B, H, dk, dv, n = 2, 4, 128, 256, 16
+    gam = inputs.multiscale_gammas(H)
+    s0 = inputs.state(B, H, dk, dv, seed=3, scale=0.5).cuda()
+    tq, tk, tv = inputs.qkv(2 * n, B * H, 1, dk, dv, torch.bfloat16, seed=21)
+    tq, tk, tv = (t.view(2 * n, B, H, 1, -1).cuda() for t in (tq, tk, tv))
+    # eager: 2n steps
+    s_eager = s0.clone()
+    y_eager = torch.stack([ret.recurrent_step(tq[i], tk[i], tv[i], gam, s_eager) for i in range(2 * n)])
+    # graph: n steps captured once, replayed twice with new inputs
+    s_graph = s0.clone()
+    g = DecodeGraph(s_graph, gam, n)
+    ys = []
+    for r in range(2):
+        g.q.copy_(tq[r * n:(r + 1) * n])
+        g.k.copy_(tk[r * n:(r + 1) * n])
+        g.v.copy_(tv[r * n:(r + 1) * n])
+        ys.append(g.replay().clone())
+    torch.cuda.synchronize()
+    assert ret.device_status() == 0
+    assert torch.equal(torch.cat(ys), y_eager) and torch.equal(s_graph, s_eager)
+    # and the oracle on the whole run of 2n tokens
+    q_all = tq.reshape(2 * n, B, H, -1).permute(1, 2, 0, 3).cpu()
+    k_all = tk.reshape(2 * n, B, H, -1).permute(1, 2, 0, 3).cpu()
+    v_all = tv.reshape(2 * n, B, H, -1).permute(1, 2, 0, 3).cpu()
+    y_ref, s_ref = oracle.recurrent(q_all, k_all, v_all, gam, s0.cpu())
+    assert rel(torch.cat(ys).reshape(2 * n, B, H, dv).permute(1, 2, 0, 3), y_ref) <= 2e-2
+    assert rel(s_graph, s_ref) <= 2e-2
