@@ -220,6 +220,25 @@ def test_recurrent_step_odd_dv():
     assert rel(y, y_ref) <= 1e-4 and rel(state, s_ref) <= 1e-4
 
 
+@pytest.mark.parametrize("dt,B,H,dk,dv", [
+    (torch.bfloat16, 1, 40, 128, 512),   # two CTAs per column block (cluster of 2)
+    (torch.bfloat16, 1, 24, 128, 512),   # cluster of 4
+    (torch.float32, 1, 1, 256, 512),     # cluster of 8
+    (torch.float32, 1, 2, 64, 30),       # cluster of 4, scalar columns
+])
+def test_recurrent_steps_small_batch_clusters(dt, B, H, dk, dv):
+    steps = 4
+    qs, ks, vs = inputs.decode_tokens(steps, B, H, dk, dv, dt, seed=5)
+    s0 = inputs.state(B, H, dk, dv, seed=6, scale=0.3)
+    gam = inputs.multiscale_gammas(H)
+    y_ref, s_ref = oracle.recurrent(torch.cat(list(qs), dim=2), torch.cat(list(ks), dim=2),
+                                    torch.cat(list(vs), dim=2), gam, s0)
+    state = s0.cuda()
+    ys = [ret.recurrent_step(qs[n].cuda(), ks[n].cuda(), vs[n].cuda(), gam, state) for n in range(steps)]
+    assert ret.device_status() == 0
+    assert rel(torch.cat(ys, dim=2), y_ref) <= TOL[dt] and rel(state, s_ref) <= TOL[dt]
+
+
 # ------------------------------------------------- host-buffer entry point
 def test_chunkwise_host_matches_device_call_and_oracle():
     B, H, L, dk, dv, C = 2, 3, 700, 128, 256, 128
