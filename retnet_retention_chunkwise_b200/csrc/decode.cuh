@@ -11,11 +11,8 @@
 //    (coalesced), rows d = warp, warp+8, ... are walked with 4 rows in flight;
 //  * q and k are staged in shared memory as fp32 (broadcast reads);
 //  * the readout y = q S sums each warp's rows in registers and the 8 warp
-//    partials through shared memory;
-//  * small batches, whose (b, h, column block) count would leave SMs idle, split
-//    the rows of each block over a cluster of 2..8 CTAs (see the kernel).
+//    partials through shared memory.
 #pragma once
-#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -34,13 +31,7 @@ __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162flo
 __device__ __forceinline__ void from_f32(float* p, float x) { *p = x; }
 __device__ __forceinline__ void from_f32(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
-// SPLIT > 1: a thread-block cluster of SPLIT CTAs shares one (b, h, column
-// block); CTA r of the cluster takes the state rows d = 8 r + warp (mod 8 SPLIT),
-// and the partial readouts meet in the first CTA's shared memory through
-// distributed shared memory.  Used when the (b, h, column block) count alone
-// would leave SMs idle (small batches).  Every thread of every CTA reaches both
-// cluster barriers: no thread leaves the kernel early.
-template <typename T, bool kVec, int SPLIT>
+template <typename T, bool kVec>
 __global__ void __launch_bounds__(kDecodeThreads)
 recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                       T* __restrict__ y, float* __restrict__ S, int H, int dk, int dv,
@@ -48,14 +39,11 @@ recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   __shared__ float sq[kDecodeMaxDk];
   __shared__ float sk[kDecodeMaxDk];
   __shared__ float4 red[kDecodeThreads / 32][32];
-  __shared__ float4 part[32];
 
   const int bh = blockIdx.y;
   const float g = hg.g[bh % H];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rank = (SPLIT > 1) ? (int)(blockIdx.x % SPLIT) : 0;
-  const int col = (int)(blockIdx.x / SPLIT) * kDecodeCols + lane * 4;
-  constexpr int R = 8 * SPLIT;  // row stride of one warp
+  const int col = blockIdx.x * kDecodeCols + lane * 4;
 
   for (int i = threadIdx.x; i < dk; i += kDecodeThreads) {
     sq[i] = to_f32(q[(size_t)bh * dk + i]);
@@ -72,27 +60,27 @@ recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   if (kVec) {
     // dv % 4 == 0 and S 16-byte aligned: whole float4 columns, col < dv or not at all.
     if (col < dv) {
-      int d = 8 * rank + warp;
-      for (; d + 3 * R < dk; d += 4 * R) {
+      int d = warp;
+      for (; d + 24 < dk; d += 32) {
         float4 s[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          s[u] = *reinterpret_cast<const float4*>(Sh + (size_t)(d + R * u) * dv + col);
+          s[u] = *reinterpret_cast<const float4*>(Sh + (size_t)(d + 8 * u) * dv + col);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const float kd = sk[d + R * u], qd = sq[d + R * u];
+          const float kd = sk[d + 8 * u], qd = sq[d + 8 * u];
           s[u].x = fmaf(g, s[u].x, kd * vv[0]);
           s[u].y = fmaf(g, s[u].y, kd * vv[1]);
           s[u].z = fmaf(g, s[u].z, kd * vv[2]);
           s[u].w = fmaf(g, s[u].w, kd * vv[3]);
-          *reinterpret_cast<float4*>(Sh + (size_t)(d + R * u) * dv + col) = s[u];
+          *reinterpret_cast<float4*>(Sh + (size_t)(d + 8 * u) * dv + col) = s[u];
           acc[0] = fmaf(qd, s[u].x, acc[0]);
           acc[1] = fmaf(qd, s[u].y, acc[1]);
           acc[2] = fmaf(qd, s[u].z, acc[2]);
           acc[3] = fmaf(qd, s[u].w, acc[3]);
         }
       }
-      for (; d < dk; d += R) {
+      for (; d < dk; d += 8) {
         float4 s = *reinterpret_cast<const float4*>(Sh + (size_t)d * dv + col);
         const float kd = sk[d], qd = sq[d];
         s.x = fmaf(g, s.x, kd * vv[0]);
@@ -107,7 +95,7 @@ recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
       }
     }
   } else {
-    for (int d = 8 * rank + warp; d < dk; d += R) {
+    for (int d = warp; d < dk; d += 8) {
       const float kd = sk[d], qd = sq[d];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -122,9 +110,8 @@ recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   }
   red[warp][lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
   __syncthreads();
-  float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
   if (warp == 0) {
-    t = red[0][lane];
+    float4 t = red[0][lane];
 #pragma unroll
     for (int w = 1; w < kDecodeThreads / 32; ++w) {
       const float4 o = red[w][lane];
@@ -133,29 +120,10 @@ recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
       t.z += o.z;
       t.w += o.w;
     }
-  }
-  if constexpr (SPLIT > 1) {
-    namespace cg = cooperative_groups;
-    cg::cluster_group cluster = cg::this_cluster();
-    if (warp == 0) part[lane] = t;
-    cluster.sync();  // every CTA's partial readout is in its shared memory
-    if (rank == 0 && warp == 0) {
-#pragma unroll
-      for (int r = 1; r < SPLIT; ++r) {
-        const float4 o = cluster.map_shared_rank(part, r)[lane];
-        t.x += o.x;
-        t.y += o.y;
-        t.z += o.z;
-        t.w += o.w;
-      }
-    }
-    cluster.sync();  // the other CTAs keep their shared memory until it is read
-  }
-  if (rank == 0 && warp == 0) {
-    const float r4[4] = {t.x, t.y, t.z, t.w};
+    const float r[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-      if (col + u < dv) from_f32(y + (size_t)bh * dv + col + u, r4[u]);
+      if (col + u < dv) from_f32(y + (size_t)bh * dv + col + u, r[u]);
   }
 }
 

@@ -593,63 +593,6 @@ ret_status retention_get_device_status(void* stream) {
   return RET_OK;
 }
 
-}  // extern "C"
-
-namespace {
-
-// CTAs per (b, h, column block) of a decode step: doubled (up to a cluster of
-// 8) while the grid would fill fewer than two CTAs per SM and every warp still
-// gets two rows or more.
-int decode_split(const ret_shape& s) {
-  const long long base = (long long)((s.dv + kDecodeCols - 1) / kDecodeCols) * s.B * s.H;
-  int split = 1;
-  while (split < 8 && base * split < 2LL * sm_count() && 16 * (2 * split) <= s.dk) split *= 2;
-  return split;
-}
-
-template <typename T, bool kVec, int SPLIT>
-cudaError_t launch_decode(dim3 grid, cudaStream_t st, const T* q, const T* k, const T* v, T* y, float* state,
-                          const ret_shape& s, const HeadGamma& hg) {
-  grid.x *= SPLIT;
-  if constexpr (SPLIT == 1) {
-    recurrent_step_kernel<T, kVec, 1><<<grid, kDecodeThreads, 0, st>>>(q, k, v, y, state, s.H, s.dk, s.dv, hg);
-    return cudaGetLastError();
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(kDecodeThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = SPLIT;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, recurrent_step_kernel<T, kVec, SPLIT>, q, k, v, y, state, s.H, s.dk, s.dv, hg);
-  }
-}
-
-template <typename T, bool kVec>
-cudaError_t launch_decode_split(int split, dim3 grid, cudaStream_t st, const void* q, const void* k, const void* v,
-                                void* y, float* state, const ret_shape& s, const HeadGamma& hg) {
-  auto* qt = static_cast<const T*>(q);
-  auto* kt = static_cast<const T*>(k);
-  auto* vt = static_cast<const T*>(v);
-  auto* yt = static_cast<T*>(y);
-  switch (split) {
-    case 8: return launch_decode<T, kVec, 8>(grid, st, qt, kt, vt, yt, state, s, hg);
-    case 4: return launch_decode<T, kVec, 4>(grid, st, qt, kt, vt, yt, state, s, hg);
-    case 2: return launch_decode<T, kVec, 2>(grid, st, qt, kt, vt, yt, state, s, hg);
-    default: return launch_decode<T, kVec, 1>(grid, st, qt, kt, vt, yt, state, s, hg);
-  }
-}
-
-}  // namespace
-
-extern "C" {
-
 ret_status retention_recurrent_step(const void* q, const void* k, const void* v, const float* gamma,
                                     void* y, float* state, ret_shape s, ret_dtype dt, void* stream) {
   ret_status rc = check_shape(s, false);
@@ -664,17 +607,23 @@ ret_status retention_recurrent_step(const void* q, const void* k, const void* v,
   std::lock_guard<std::mutex> lock(mu);
   for (int h = 0; h < s.H; ++h) hg.g[h] = gamma[h];
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const dim3 grid((s.dv + kDecodeCols - 1) / kDecodeCols, s.B * s.H);
+  dim3 grid((s.dv + kDecodeCols - 1) / kDecodeCols, s.B * s.H);
   const bool vec = (s.dv % 4) == 0;
-  const int split = decode_split(s);
-  cudaError_t e;
-  if (dt == RET_F32)
-    e = vec ? launch_decode_split<float, true>(split, grid, st, q, k, v, y, state, s, hg)
-            : launch_decode_split<float, false>(split, grid, st, q, k, v, y, state, s, hg);
-  else
-    e = vec ? launch_decode_split<__nv_bfloat16, true>(split, grid, st, q, k, v, y, state, s, hg)
-            : launch_decode_split<__nv_bfloat16, false>(split, grid, st, q, k, v, y, state, s, hg);
-  if (e != cudaSuccess) return RET_ECUDA;
+  if (dt == RET_F32) {
+    auto* qf = static_cast<const float*>(q);
+    auto* kf = static_cast<const float*>(k);
+    auto* vf = static_cast<const float*>(v);
+    auto* yf = static_cast<float*>(y);
+    if (vec) recurrent_step_kernel<float, true><<<grid, kDecodeThreads, 0, st>>>(qf, kf, vf, yf, state, s.H, s.dk, s.dv, hg);
+    else recurrent_step_kernel<float, false><<<grid, kDecodeThreads, 0, st>>>(qf, kf, vf, yf, state, s.H, s.dk, s.dv, hg);
+  } else {
+    auto* qb = static_cast<const __nv_bfloat16*>(q);
+    auto* kb = static_cast<const __nv_bfloat16*>(k);
+    auto* vb = static_cast<const __nv_bfloat16*>(v);
+    auto* yb = static_cast<__nv_bfloat16*>(y);
+    if (vec) recurrent_step_kernel<__nv_bfloat16, true><<<grid, kDecodeThreads, 0, st>>>(qb, kb, vb, yb, state, s.H, s.dk, s.dv, hg);
+    else recurrent_step_kernel<__nv_bfloat16, false><<<grid, kDecodeThreads, 0, st>>>(qb, kb, vb, yb, state, s.H, s.dk, s.dv, hg);
+  }
   return launch_status();
 }
 

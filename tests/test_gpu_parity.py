@@ -221,12 +221,12 @@ def test_recurrent_step_odd_dv():
 
 
 @pytest.mark.parametrize("dt,B,H,dk,dv", [
-    (torch.bfloat16, 1, 40, 128, 512),   # two CTAs per column block (cluster of 2)
-    (torch.bfloat16, 1, 24, 128, 512),   # cluster of 4
-    (torch.float32, 1, 1, 256, 512),     # cluster of 8
-    (torch.float32, 1, 2, 64, 30),       # cluster of 4, scalar columns
+    (torch.bfloat16, 1, 40, 128, 512),
+    (torch.bfloat16, 1, 24, 128, 512),
+    (torch.float32, 1, 1, 256, 512),     # one head
+    (torch.float32, 1, 2, 64, 30),       # scalar columns
 ])
-def test_recurrent_steps_small_batch_clusters(dt, B, H, dk, dv):
+def test_recurrent_steps_small_batch(dt, B, H, dk, dv):
     steps = 4
     qs, ks, vs = inputs.decode_tokens(steps, B, H, dk, dv, dt, seed=5)
     s0 = inputs.state(B, H, dk, dv, seed=6, scale=0.3)
