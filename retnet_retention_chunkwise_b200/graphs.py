@@ -45,7 +45,9 @@ class DecodeGraph:
         torch.cuda.current_stream(dev).wait_stream(side)
         torch.cuda.synchronize(dev)
         self.graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph):
+        # thread-local capture: CUDA calls made meanwhile by other threads of the
+        # process (a collective library's watchdog, a sampler) do not end it
+        with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
             for n in range(n_steps):
                 self._step(self.q[n], self.k[n], self.v[n], gamma, self.state, out=self.y[n])
 
