@@ -45,14 +45,6 @@ recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int col = blockIdx.x * kDecodeCols + lane * 4;
 
-  // Launched with programmatic dependent launch: this grid may start while the
-  // previous kernel on the stream (usually the previous step) is finishing.
-  // Nothing above reads memory another kernel writes; wait for the previous
-  // grid's completion and memory here, then let the next step's grid start its
-  // own launch.  Without the launch attribute both instructions do nothing.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
   for (int i = threadIdx.x; i < dk; i += kDecodeThreads) {
     sq[i] = to_f32(q[(size_t)bh * dk + i]);
     sk[i] = to_f32(k[(size_t)bh * dk + i]);

@@ -607,40 +607,23 @@ ret_status retention_recurrent_step(const void* q, const void* k, const void* v,
   std::lock_guard<std::mutex> lock(mu);
   for (int h = 0; h < s.H; ++h) hg.g[h] = gamma[h];
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const dim3 grid((s.dv + kDecodeCols - 1) / kDecodeCols, s.B * s.H);
+  dim3 grid((s.dv + kDecodeCols - 1) / kDecodeCols, s.B * s.H);
   const bool vec = (s.dv % 4) == 0;
-  // programmatic dependent launch: the step's grid may be scheduled while the
-  // previous kernel drains (the kernel waits for it before touching memory)
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(kDecodeThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e;
   if (dt == RET_F32) {
     auto* qf = static_cast<const float*>(q);
     auto* kf = static_cast<const float*>(k);
     auto* vf = static_cast<const float*>(v);
     auto* yf = static_cast<float*>(y);
-    e = vec ? cudaLaunchKernelEx(&cfg, recurrent_step_kernel<float, true>, qf, kf, vf, yf, state, s.H, s.dk, s.dv, hg)
-            : cudaLaunchKernelEx(&cfg, recurrent_step_kernel<float, false>, qf, kf, vf, yf, state, s.H, s.dk, s.dv,
-                                 hg);
+    if (vec) recurrent_step_kernel<float, true><<<grid, kDecodeThreads, 0, st>>>(qf, kf, vf, yf, state, s.H, s.dk, s.dv, hg);
+    else recurrent_step_kernel<float, false><<<grid, kDecodeThreads, 0, st>>>(qf, kf, vf, yf, state, s.H, s.dk, s.dv, hg);
   } else {
     auto* qb = static_cast<const __nv_bfloat16*>(q);
     auto* kb = static_cast<const __nv_bfloat16*>(k);
     auto* vb = static_cast<const __nv_bfloat16*>(v);
     auto* yb = static_cast<__nv_bfloat16*>(y);
-    e = vec ? cudaLaunchKernelEx(&cfg, recurrent_step_kernel<__nv_bfloat16, true>, qb, kb, vb, yb, state, s.H, s.dk,
-                                 s.dv, hg)
-            : cudaLaunchKernelEx(&cfg, recurrent_step_kernel<__nv_bfloat16, false>, qb, kb, vb, yb, state, s.H,
-                                 s.dk, s.dv, hg);
+    if (vec) recurrent_step_kernel<__nv_bfloat16, true><<<grid, kDecodeThreads, 0, st>>>(qb, kb, vb, yb, state, s.H, s.dk, s.dv, hg);
+    else recurrent_step_kernel<__nv_bfloat16, false><<<grid, kDecodeThreads, 0, st>>>(qb, kb, vb, yb, state, s.H, s.dk, s.dv, hg);
   }
-  if (e != cudaSuccess) return RET_ECUDA;
   return launch_status();
 }
 
