@@ -1,0 +1,40 @@
+"""Host-side pieces of bench.py (no GPU): the algorithmic counts behind the
+roofline fractions, and the reading of the committed ncu summary."""
+import os
+import tempfile
+
+import bench
+
+
+def test_headline_algorithmic_counts():
+    # B4 H8 L8192 dk256 dv512 C128: q, k, v read once, y written once (bf16),
+    # fp32 state out; causal intra-block pairs, cross-block term, state update
+    assert bench.chunk_bytes(4, 8, 8192, 256, 512) == 805_306_368 + 16_777_216
+    per_token = bench.chunk_flops_per_head_token(128, 256, 512)
+    assert per_token == 129 * 768 + 4 * 256 * 512 == 623_360
+    assert 4 * 8 * 8192 * per_token == 163_410_083_840
+
+
+def test_parallel_flops_counts_causal_pairs():
+    # L(L+1)/2 pairs per head, 2 (dk + dv) flops each
+    assert bench.parallel_flops(1, 1, 4, 2, 3) == 10 * 2 * 5
+    assert bench.parallel_flops(2, 8, 2048, 64, 128) == 12_891_193_344
+
+
+def test_traffic_is_read_only_for_the_current_kernel_source():
+    digest = bench.kernel_source_digest()
+    assert len(digest) == 16
+    text = ("# summary\n\n- dram_bytes_per_launch: `123456`\n"
+            f"- kernel_source_sha256_16: `{digest}` (the kernel's source)\n")
+    stale = text.replace(digest, "0" * 16)
+    orig = bench.TRAFFIC_FILE
+    try:
+        with tempfile.TemporaryDirectory() as d:
+            for body, want in ((text, 123456.0), (stale, None)):
+                p = os.path.join(d, "s.md")
+                with open(p, "w") as f:
+                    f.write(body)
+                bench.TRAFFIC_FILE = p
+                assert bench.measured_traffic() == want
+    finally:
+        bench.TRAFFIC_FILE = orig
