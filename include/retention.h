@@ -275,6 +275,18 @@ RET_API ret_status retention_chunkwise_gn(const void* q, const void* k, const vo
 RET_API size_t retention_chunkwise_gn_workspace_bytes(int chunk, ret_shape s, ret_dtype dt);
 
 /*
+ * retention_chunkwise_gn with the output gate: y receives
+ * GroupNorm(y) * act(gate) (see retention_groupnorm_gated), in place.  gate:
+ * device [B][H][L][dv] in the call's dtype, 16-byte aligned, not y; NULL for no
+ * gate.  act: a ret_gate_act.  Workspace: retention_chunkwise_gn_workspace_bytes().
+ */
+RET_API ret_status retention_chunkwise_gn_gated(const void* q, const void* k, const void* v, const float* gamma,
+                                                void* y, const float* state_in, float* state_out, int chunk,
+                                                ret_shape s, ret_dtype dt, float eps, const float* weight,
+                                                const float* bias, const void* gate, int act, void* workspace,
+                                                size_t workspace_bytes, void* stream);
+
+/*
  * Backward pass of retention_parallel: for the upstream gradient dy of
  * y = retention_parallel(q, k, v), writes
  *     dq_n = sum_{m<=n} gamma^(n-m) (dy_n . v_m) k_m

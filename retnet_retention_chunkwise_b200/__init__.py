@@ -261,10 +261,12 @@ def groupnorm(y, eps: float = 1e-5, *, weight=None, bias=None, out=None, gate=No
 
 
 def chunkwise_groupnorm(q, k, v, gamma, chunk: int, eps: float = 1e-5, *, weight=None, bias=None,
-                        state_in=None, state_out=None, return_state=True, out=None, workspace="auto"):
+                        state_in=None, state_out=None, return_state=True, out=None, workspace="auto",
+                        gate=None, act: str = "swish"):
     """Chunkwise form followed by the per-head group normalisation of its output
-    (see :func:`groupnorm`, a second kernel on the stream).  Returns
-    (normalised y, state_out)."""
+    (see :func:`groupnorm`, a second kernel on the stream), and with ``gate``
+    (v's shape and dtype) the output gate act(gate).  Returns (normalised y,
+    state_out)."""
     dt = _qkv(q, k, v)
     s = _shape(q, v)
     y = out if out is not None else torch.empty(v.shape, dtype=v.dtype, device=v.device)
@@ -281,10 +283,22 @@ def chunkwise_groupnorm(q, k, v, gamma, chunk: int, eps: float = 1e-5, *, weight
     if isinstance(workspace, str):
         workspace = _workspace(int(library().retention_chunkwise_gn_workspace_bytes(chunk, s, dt)), q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(library().retention_chunkwise_gn(_ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(y),
-                                            _ptr(state_in), _ptr(state_out), int(chunk), s, dt, float(eps),
-                                            _ptr(weight), _ptr(bias), _ptr(workspace), wbytes, _stream()),
-           "retention_chunkwise_gn")
+    if gate is None:
+        _check(library().retention_chunkwise_gn(_ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(y),
+                                                _ptr(state_in), _ptr(state_out), int(chunk), s, dt, float(eps),
+                                                _ptr(weight), _ptr(bias), _ptr(workspace), wbytes, _stream()),
+               "retention_chunkwise_gn")
+        return y, state_out
+    _cuda(gate, "gate")
+    if gate.shape != v.shape or gate.dtype != v.dtype:
+        raise ValueError("retention: gate must match v")
+    if act not in _abi.GATE_ACTS:
+        raise ValueError(f"retention: act must be one of {sorted(_abi.GATE_ACTS)}")
+    _check(library().retention_chunkwise_gn_gated(_ptr(q), _ptr(k), _ptr(v), _gamma(gamma, s.H), _ptr(y),
+                                                  _ptr(state_in), _ptr(state_out), int(chunk), s, dt, float(eps),
+                                                  _ptr(weight), _ptr(bias), _ptr(gate), _abi.GATE_ACTS[act],
+                                                  _ptr(workspace), wbytes, _stream()),
+           "retention_chunkwise_gn_gated")
     return y, state_out
 
 

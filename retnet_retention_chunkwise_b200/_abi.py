@@ -30,6 +30,7 @@ EXPORTS = (
     "retention_chunkwise_host_workspace_bytes",
     "retention_groupnorm",
     "retention_groupnorm_gated",
+    "retention_chunkwise_gn_gated",
     "retention_chunkwise_gn",
     "retention_chunkwise_gn_workspace_bytes",
     "retention_parallel_backward",
@@ -79,6 +80,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.retention_groupnorm.restype = ctypes.c_int
     lib.retention_groupnorm_gated.argtypes = [vp, vp, vp, f32, vp, vp, i, RetShape, i, vp]
     lib.retention_groupnorm_gated.restype = ctypes.c_int
+    lib.retention_chunkwise_gn_gated.argtypes = [vp, vp, vp, fp, vp, vp, vp, i, RetShape, i, f32, vp, vp, vp, i,
+                                                 vp, sz, vp]
+    lib.retention_chunkwise_gn_gated.restype = ctypes.c_int
     lib.retention_chunkwise_gn.argtypes = [vp, vp, vp, fp, vp, vp, vp, i, RetShape, i, f32, vp, vp, vp, sz, vp]
     lib.retention_chunkwise_gn.restype = ctypes.c_int
     lib.retention_chunkwise_gn_workspace_bytes.argtypes = [i, RetShape, i]

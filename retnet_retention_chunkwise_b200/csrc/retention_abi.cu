@@ -949,12 +949,23 @@ ret_status retention_chunkwise_gn(const void* q, const void* k, const void* v, c
                                   const float* state_in, float* state_out, int chunk, ret_shape s, ret_dtype dt,
                                   float eps, const float* weight, const float* bias, void* workspace,
                                   size_t workspace_bytes, void* stream) {
+  return retention_chunkwise_gn_gated(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, eps, weight, bias,
+                                      nullptr, RET_GATE_NONE, workspace, workspace_bytes, stream);
+}
+
+ret_status retention_chunkwise_gn_gated(const void* q, const void* k, const void* v, const float* gamma, void* y,
+                                        const float* state_in, float* state_out, int chunk, ret_shape s,
+                                        ret_dtype dt, float eps, const float* weight, const float* bias,
+                                        const void* gate, int act, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
   if (!(eps >= 0.f) || !std::isfinite(eps)) return RET_EINVAL;
+  if (act < kGateNone || act > kGateSigmoid) return RET_EINVAL;
   if (s.dv > kGN_MaxDv) return RET_EUNSUPPORTED;
+  if (gate && s.L > 0 && (!aligned16(gate) || gate == y)) return RET_EINVAL;
   ret_status rc = retention_chunkwise(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, workspace,
                                       workspace_bytes, stream);
   if (rc != RET_OK || s.L == 0) return rc;
-  return retention_groupnorm(y, y, eps, weight, bias, s, dt, stream);
+  return retention_groupnorm_gated(y, gate, y, eps, weight, bias, act, s, dt, stream);
 }
 
 size_t retention_parallel_backward_workspace_bytes(ret_shape s, ret_dtype dt) {

@@ -269,3 +269,14 @@ def test_plain_c_caller():
         out = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0, out.stdout + out.stderr
     assert out.stdout.startswith("ok ")
+
+
+def test_chunkwise_gn_gated_validation(lib):
+    s = _abi.RetShape(1, 2, 64, 128, 128)
+    g = _g(0.5, 0.9)
+    call = lambda gate, act, eps=1e-5, y=ctypes.c_void_p(0x20000): lib.retention_chunkwise_gn_gated(  # noqa: E731
+        FAKE, FAKE, FAKE, g, y, None, None, 64, s, _abi.RET_BF16, eps, None, None, gate, act, None, 0, None)
+    assert call(FAKE, 5) == _abi.RET_EINVAL                       # unknown activation
+    assert call(FAKE, 1, eps=-1.0) == _abi.RET_EINVAL             # eps < 0
+    assert call(ctypes.c_void_p(0x10008), 1) == _abi.RET_EINVAL   # gate not 16-byte aligned
+    assert call(ctypes.c_void_p(0x20000), 1) == _abi.RET_EINVAL   # gate is y

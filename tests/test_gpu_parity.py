@@ -282,6 +282,23 @@ def test_groupnorm_standalone(dt, dv, affine):
     assert torch.equal(yd, out)
 
 
+@pytest.mark.parametrize("act", ["swish", "sigmoid"])
+def test_chunkwise_groupnorm_gated(act):
+    B, H, L, dk, dv, C = 1, 2, 300, 128, 256, 128
+    q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed=L + 11)
+    gam = inputs.multiscale_gammas(H)
+    s_in = inputs.state(B, H, dk, dv, seed=12, scale=0.5)
+    g = torch.Generator("cpu").manual_seed(13)
+    gate = (torch.randn((B, H, L, dv), generator=g) * 2.0).to(torch.bfloat16)
+    w = torch.rand(H * dv, generator=g) + 0.5
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam, s_in)
+    z_ref = oracle.gate(oracle.groupnorm(y_ref, eps=1e-5, weight=w), gate, act)
+    qd, kd, vd, sd = dev(q, k, v, s_in)
+    z, s = ret.chunkwise_groupnorm(qd, kd, vd, gam, C, 1e-5, weight=w.cuda(), state_in=sd, gate=gate.cuda(), act=act)
+    assert ret.device_status() == 0
+    assert rel(z, z_ref) <= 2e-2 and rel(s, s_ref) <= 2e-2
+
+
 @pytest.mark.parametrize("dt,dv", [(torch.bfloat16, 512), (torch.bfloat16, 128), (torch.bfloat16, 96),
                                    (torch.float32, 128), (torch.float32, 48)])
 @pytest.mark.parametrize("act", ["swish", "sigmoid", "none"])
