@@ -567,7 +567,7 @@ RET_API int retention_debug_trace(void* buf, int blocks, int events) {
 }
 #endif
 
-int retention_abi_version(void) { return 102; }
+int retention_abi_version(void) { return 103; }
 
 const char* retention_status_str(ret_status st) {
   switch (st) {

@@ -50,7 +50,7 @@ def test_status_strings_and_version(lib):
     names = [lib.retention_status_str(i).decode() for i in range(5)]
     assert names == ["RET_OK", "RET_EINVAL", "RET_EUNSUPPORTED", "RET_ECUDA", "RET_ETIMEOUT"]
     assert lib.retention_status_str(99).decode() == "RET_UNKNOWN"
-    assert lib.retention_abi_version() == 102
+    assert lib.retention_abi_version() == 103
 
 
 def _g(*vals):
