@@ -280,3 +280,24 @@ def test_chunkwise_gn_gated_validation(lib):
     assert call(FAKE, 1, eps=-1.0) == _abi.RET_EINVAL             # eps < 0
     assert call(ctypes.c_void_p(0x10008), 1) == _abi.RET_EINVAL   # gate not 16-byte aligned
     assert call(ctypes.c_void_p(0x20000), 1) == _abi.RET_EINVAL   # gate is y
+
+
+def test_missing_library_fails_loudly():
+    # no fallback: without the built library the binding raises, naming the build step
+    with pytest.raises(ImportError, match="build"):
+        _abi.load("/nonexistent/libretention.so")
+
+
+def test_calls_fail_without_cuda_tensors():
+    # the binding never computes on the host: CPU tensors are refused
+    import torch
+
+    import retnet_retention_chunkwise_b200 as ret
+    q = torch.zeros((1, 1, 4, 64), dtype=torch.bfloat16)
+    v = torch.zeros((1, 1, 4, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        ret.chunkwise(q, q, v, torch.tensor([0.5]), 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        ret.parallel(q, q, v, torch.tensor([0.5]))
+    with pytest.raises(ValueError, match="CUDA"):
+        ret.chunkwise_state(q, v, torch.tensor([0.5]), 64)
