@@ -81,7 +81,8 @@ def _free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("world,L,chunk,uneven", [(2, 40, 8, False), (3, 37, 4, False), (3, 23, 4, True)])
+@pytest.mark.parametrize("world,L,chunk,uneven", [(2, 40, 8, False), (3, 37, 4, False), (3, 23, 4, True),
+                                                  (4, 50, 4, True)])
 def test_sequence_sharded_exchange_gloo(world, L, chunk, uneven):
     with tempfile.TemporaryDirectory() as out_dir:
         mp.start_processes(_worker, args=(world, _free_port(), out_dir, L, chunk, uneven), nprocs=world,
