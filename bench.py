@@ -55,7 +55,9 @@ METRIC = "retention tokens/sec (chunkwise fwd, decode) and % of tensor/HBM roofl
 HEADLINE = inputs.WORKLOADS["retnet1p3b_layer_bf16"]
 L2_BYTES = 126 * 1024 * 1024
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "chunkwise_tc256_retnet1p3b_layer.md")
+# ncu DRAM traffic of one headline launch, with the digest of the kernel source
+# it was captured on (written next to the ncu summary of that capture)
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "chunkwise_tc256_retnet1p3b_layer.traffic.json")
 
 
 # --------------------------------------------------------------- accounting
@@ -110,21 +112,14 @@ def kernel_source_digest():
 
 
 def measured_traffic():
-    """dram bytes per launch of the headline kernel from the committed ncu summary,
-    or None if absent or taken on a different kernel source."""
+    """dram bytes per launch of the headline kernel from the ncu capture's JSON
+    record, or None if absent or captured on a different kernel source."""
     try:
-        kv = {}
         with open(TRAFFIC_FILE) as f:
-            for ln in f:
-                if ":" in ln and ln.strip().startswith("- "):
-                    k, v = ln.strip()[2:].split(":", 1)
-                    v = v.strip()
-                    if v.startswith("`") and "`" in v[1:]:
-                        v = v[1:v.index("`", 1)]  # the first quoted token
-                    kv[k.strip()] = v
-        if kv.get("kernel_source_sha256_16") != kernel_source_digest():
+            rec = json.load(f)
+        if rec.get("kernel_source_sha256_16") != kernel_source_digest():
             return None
-        return float(kv["dram_bytes_per_launch"])
+        return float(rec["dram_bytes_per_launch"])
     except Exception:
         return None
 
@@ -322,11 +317,13 @@ def bench_e2e(ret, args, dist):
     gam = w.gammas()
     dev = tuple(torch.empty_like(t, device="cuda") for t in (qh, kh, vh, yh))
     sd = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device="cuda")
+    sh = torch.empty(sd.shape, dtype=torch.float32).pin_memory()
 
     def step():
         # retention_chunkwise_host: q, k, v host -> device, the kernels, y device -> host,
-        # overlapped across groups of heads inside the library
+        # overlapped across groups of heads inside the library; then state_out to the host
         ret.chunkwise_host(qh, kh, vh, gam, w.chunk, dev=dev, out=yh, state_out=sd)
+        sh.copy_(sd, non_blocking=True)
 
     steps = 10
     _, total = time_calls(step, steps, max(args.warmup, 3), dist)
@@ -334,7 +331,7 @@ def bench_e2e(ret, args, dist):
     value = dist.sum(w.B * w.L * steps) / (t_ms * 1e-3 * steps)
     return {"value": value, "unit": "tokens/s", "ms_per_step": round(t_ms, 3), "steps": steps,
             "h2d_bytes_per_step": sum(t.numel() * 2 for t in (qh, kh, vh)),
-            "d2h_bytes_per_step": yh.numel() * 2}
+            "d2h_bytes_per_step": yh.numel() * 2 + sh.numel() * 4}
 
 
 def bench_decode(ret, args, dist, peaks):
@@ -370,7 +367,7 @@ def bench_decode(ret, args, dist, peaks):
     kern = dist.max(statistics.mean(a.elapsed_time(b) for a, b in ev))
     nbytes = w.B * w.H * (2 * w.dk * w.dv * 4 + (2 * w.dk + 2 * w.dv) * 2)
     gbs = nbytes / (kern * 1e-3) / 1e9
-    return {"workload": "decode_6p7b: B=64 H=16 dk=256 dv=512, 1024 steps after a 512-token prefill",
+    return {"workload": "B64 H16 dk256 dv512, 1024 steps after a 512-token prefill",
             "tokens_per_s": dist.sum(w.B * steps) / (total * 1e-3),
             "ms_per_token_step": round(total / steps, 4), "kernel_ms": round(kern, 4),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -406,7 +403,7 @@ def bench_decode_graph(ret, args, dist, peaks):
     e = dist.max(t_eager) / (10 * n)
     gr = dist.max(t_graph) / (10 * n)
     nbytes = B * H * (2 * dk * dv * 4 + (2 * dk + 2 * dv) * 2)
-    return {"workload": "decode at batch 1: B=1 H=16 dk=256 dv=512, 64 steps per graph",
+    return {"workload": "B1 H16 dk256 dv512, 64 steps per graph",
             "eager_ms_per_step": round(e, 4), "graph_ms_per_step": round(gr, 4),
             "tokens_per_s_graph": dist.sum(B) / (gr * 1e-3),
             "hbm_frac_graph": round(nbytes / (gr * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
@@ -427,7 +424,7 @@ def bench_small(ret, args, dist, peaks):
     per, _ = time_calls(lambda: ret.parallel(q, k, v, gam, out=y), n, max(args.warmup, 3), dist, flush=True)
     t = dist.max(statistics.median(per))
     fl = parallel_flops(w.B, w.H, w.L, w.dk, w.dv)
-    out["parallel"] = {"workload": "msr_core: B=2 H=8 L=2048 dk=64 dv=128 (L2 flushed per call)",
+    out["parallel"] = {"workload": "B2 H8 L2048 dk64 dv128, L2 flushed",
                        "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3), "kernel_ms": round(t, 4),
                        "roofline": {"bound": "tensor", "achieved": round(fl / (t * 1e-3) / 1e12, 1),
                                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -439,8 +436,7 @@ def bench_small(ret, args, dist, peaks):
     per, _ = time_calls(lambda: ret.parallel_backward(q, k, v, gam, dy, workspace=ws), n, max(args.warmup, 3),
                         dist, flush=True)
     t = dist.max(statistics.median(per))
-    out["parallel_backward"] = {"workload": "msr_core: B=2 H=8 L=2048 dk=64 dv=128, dq dk dv for an upstream dy "
-                                            "(L2 flushed per call)",
+    out["parallel_backward"] = {"workload": "B2 H8 L2048 dk64 dv128, L2 flushed",
                                 "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3), "call_ms": round(t, 4),
                                 "tensor": {"achieved_tflops": round(3 * fl / (t * 1e-3) / 1e12, 1),
                                            "frac": round(3 * fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
@@ -450,7 +446,7 @@ def bench_small(ret, args, dist, peaks):
                         max(args.warmup, 3), dist, flush=True)
     t = dist.max(statistics.median(per))
     nb = chunk_bytes(w.B, w.H, w.L, w.dk, w.dv, state_out=False)
-    out["chunkwise_msr_core"] = {"workload": "msr_core: B=2 H=8 L=2048 dk=64 dv=128 C=64 (L2 flushed per call)",
+    out["chunkwise_msr_core"] = {"workload": "B2 H8 L2048 dk64 dv128 C64, L2 flushed",
                                  "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3), "call_ms": round(t, 4),
                                  "hbm_frac": round(nb / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
     del q, k, v, y
@@ -473,7 +469,7 @@ def bench_small(ret, args, dist, peaks):
         fl = w.B * w.H * w.L * chunk_flops_per_head_token(C, w.dk, w.dv)
         nb = chunk_bytes(w.B, w.H, w.L, w.dk, w.dv) + 2 * inputs.LONG_CONTEXT_CALLS * w.B * w.H * w.dk * w.dv * 4
         out[f"long_context_C{C}"] = {
-            "workload": "long_context: B=1 H=16 L=65536 dk=128 dv=256, 4 x 16384-token calls, state carried",
+            "workload": "B1 H16 L65536 dk128 dv256, 4 calls, state carried",
             "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3), "ms_per_65536_tokens": round(t, 4),
             "hbm_frac": round(nb / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
             "tensor_frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
@@ -484,7 +480,7 @@ def bench_small(ret, args, dist, peaks):
     t = dist.max(statistics.median(per))
     fl = 3 * w.B * w.H * seg * chunk_flops_per_head_token(128, w.dk, w.dv)
     out["chunkwise_backward_long_context"] = {
-        "workload": "long_context layout, one 16384-token call: dq dk dv through the chunkwise form, C=128",
+        "workload": "B1 H16 L16384 dk128 dv256 C128",
         "tokens_per_s": dist.sum(w.B * seg) / (t * 1e-3), "call_ms": round(t, 4),
         "tensor_frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
     # the same call carrying a state: state_in, dstate_out in, dstate_in out
@@ -495,7 +491,7 @@ def bench_small(ret, args, dist, peaks):
                         max(args.warmup, 3), dist)
     t = dist.max(statistics.median(per))
     out["chunkwise_backward_state_long_context"] = {
-        "workload": "as chunkwise_backward_long_context, with state_in, dstate_out and dstate_in (fp32 states)",
+        "workload": "B1 H16 L16384 dk128 dv256 C128, with states",
         "tokens_per_s": dist.sum(w.B * seg) / (t * 1e-3), "call_ms": round(t, 4),
         "tensor_frac": round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
     del parts, y, dy, s0, dso, ds0
@@ -512,7 +508,7 @@ def bench_small(ret, args, dist, peaks):
     nb = (k.numel() + v.numel()) * 2 + s_out.numel() * 4
     fl = 2 * w.B * w.H * w.L * w.dk * w.dv
     out["chunkwise_state_headline"] = {
-        "workload": "state only (no y): B=4 H=8 L=8192 dk=256 dv=512 C=128, k and v read, fp32 state out",
+        "workload": "B4 H8 L8192 dk256 dv512, k v in, fp32 state out",
         "call_ms": round(t, 4), "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3),
         "roofline": {"bound": "hbm", "achieved": round(nb / (t * 1e-3) / 1e9, 1), "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": round(nb / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
@@ -524,7 +520,7 @@ def bench_small(ret, args, dist, peaks):
     per, _ = time_calls(lambda: ret.groupnorm(y, 1e-5, out=y), 20, max(args.warmup, 3), dist)
     t = dist.max(statistics.median(per))
     nb = 2 * y.numel() * y.element_size()
-    out["groupnorm"] = {"workload": "per-head group normalisation of y: B=4 H=8 L=8192 dv=512 bf16, in place",
+    out["groupnorm"] = {"workload": "B4 H8 L8192 dv512, in place",
                         "kernel_ms": round(t, 4), "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3),
                         "roofline": {"bound": "hbm", "achieved": round(nb / (t * 1e-3) / 1e9, 1),
                                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -535,7 +531,7 @@ def bench_small(ret, args, dist, peaks):
     per, _ = time_calls(lambda: ret.groupnorm(y, 1e-5, out=y, gate=gate, act="swish"), 20, max(args.warmup, 3), dist)
     t = dist.max(statistics.median(per))
     nb = 3 * y.numel() * y.element_size()
-    out["groupnorm_gated"] = {"workload": "GroupNorm then swish gate: B=4 H=8 L=8192 dv=512 bf16, in place",
+    out["groupnorm_gated"] = {"workload": "B4 H8 L8192 dv512, swish gate, in place",
                               "kernel_ms": round(t, 4), "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3),
                               "roofline": {"bound": "hbm", "achieved": round(nb / (t * 1e-3) / 1e9, 1),
                                            "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -543,6 +539,30 @@ def bench_small(ret, args, dist, peaks):
                                            "algorithmic_bytes": nb, "kernel": "groupnorm_rows_kernel<bf16>"}}
     del y, gate
     return out
+
+
+def bench_headline_sustained(ret, args, dist, peaks, seconds=1.5):
+    """The headline call repeated for about `seconds` (the power cap and the
+    clock it settles at show up here, unlike in a short burst), with the SM
+    clock sampled during the run."""
+    w = HEADLINE
+    q, k, v = gpu_qkv(w.B, w.H, w.L, w.dk, w.dv, seed=w.seed)
+    gam = w.gammas()
+    y = torch.empty_like(v)
+    s_out = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device="cuda")
+    step = lambda: ret.chunkwise(q, k, v, gam, w.chunk, state_out=s_out, out=y)  # noqa: E731
+    n = max(20, int(seconds / 0.25e-3))
+    with ClockSampler(dist.local) as clk:
+        per, _ = time_calls(step, n, 5, dist)
+    assert ret.device_status() == 0
+    kern = dist.max(statistics.mean(per))
+    flops = w.B * w.H * w.L * chunk_flops_per_head_token(w.chunk, w.dk, w.dv)
+    nbytes = chunk_bytes(w.B, w.H, w.L, w.dk, w.dv, state_in=False, state_out=True)
+    tf = flops / (kern * 1e-3) / 1e12
+    return {"steps": n, "kernel_ms": round(kern, 4), "clocks": clk.summary(),
+            "hbm_frac": round(nbytes / (kern * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "tensor_frac": round(tf / peaks["bf16_tflops"], 4),
+            "tensor_frac_of_sustained": round(tf / peaks["bf16_tflops_sustained"], 4)}
 
 
 # ------------------------------------------------------------ CPU / oracle
@@ -573,6 +593,52 @@ def cpu_baseline():
     return {"value": tokens / dt, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
             "sample": f"fp64 recurrent oracle on {nthreads} of {HEADLINE.B * HEADLINE.H} heads x {L} positions "
                       f"of the headline workload ({dt:.1f} s), tokens scaled by heads/H"}
+
+
+def oracle_timings():
+    """The fp64 oracle (oracle_recurrent) timed on this host for every
+    configuration: T = all cores over (b, h), plus one thread for the two small
+    ones.  Bounded samples of the large ones (T heads; tokens scaled by T/H).
+    A CPU baseline, not the target."""
+    import oracle
+    lib = oracle.load()
+    T = os.cpu_count() or 1
+
+    def timed(q, k, v, gam, threads, reps=1):
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            oracle.recurrent(q, k, v, gam, nthreads=threads, lib=lib)
+        return (time.perf_counter() - t0) / reps
+
+    def heads(w, n, L, seed):
+        q, k, v = inputs.qkv(1, n, L, w.dk, w.dv, w.dtype, seed)
+        g = w.gammas()
+        return q, k, v, torch.stack([g[i % w.H] for i in range(n)])
+
+    out = {"threads": T}
+    w = inputs.WORKLOADS["single_head_f32"]
+    q, k, v = inputs.qkv(w.B, w.H, w.L, w.dk, w.dv, w.dtype, w.seed)
+    t1 = timed(q, k, v, w.gammas(), 1, reps=200)
+    out["single_head_f32"] = {"tokens_per_s_1thread": round(w.B * w.L / t1), "sample": "whole workload"}
+    w = inputs.WORKLOADS["msr_core_bf16"]
+    q, k, v = inputs.qkv(w.B, w.H, w.L, w.dk, w.dv, w.dtype, w.seed)
+    t1, tT = timed(q, k, v, w.gammas(), 1), timed(q, k, v, w.gammas(), T)
+    out["msr_core_bf16"] = {"tokens_per_s_1thread": round(w.B * w.L / t1), "tokens_per_s": round(w.B * w.L / tT),
+                            "sample": "whole workload"}
+    w = inputs.WORKLOADS["retnet1p3b_layer_bf16"]
+    n, L = min(T, w.B * w.H), 2048
+    tT = timed(*heads(w, n, L, 0), T)
+    out["retnet1p3b_layer_bf16"] = {"tokens_per_s": round(n / w.H * L / tT), "sample": f"{n} heads x {L} tokens"}
+    w = inputs.WORKLOADS["decode_6p7b_bf16"]
+    n, steps = min(T, w.B * w.H), inputs.DECODE_STEPS
+    tT = timed(*heads(w, n, steps, 1), T)
+    out["decode_6p7b_bf16"] = {"tokens_per_s": round(n / w.H * steps / tT),
+                               "sample": f"{n} heads x {steps} steps from a zero state"}
+    w = inputs.WORKLOADS["long_context_bf16"]
+    n, L = min(T, w.B * w.H), 4096
+    tT = timed(*heads(w, n, L, 0), T)
+    out["long_context_bf16"] = {"tokens_per_s": round(n / w.H * L / tT), "sample": f"{n} heads x {L} tokens"}
+    return out
 
 
 def headline_config(world: int) -> dict:
@@ -661,6 +727,61 @@ def run_profile_case(args):
     assert ret.device_status() == 0
 
 
+def run_sequence(args):
+    """--mode sequence: one sequence of the long-context layout (B=1, H=16,
+    dk=128, dv=256, C=128) cut across the ranks, each rank holding a run of
+    65536 tokens (weak scaling: the sequence is 65536 * N tokens).  A step is
+    chunkwise_sequence_sharded on every rank: the run's state-only sum, one
+    NCCL all-gather of the sums, the fold, the chunkwise call from the folded
+    state.  value = tokens of the whole sequence / max-over-ranks time."""
+    import datetime
+    import socket
+
+    import torch.distributed as tdist
+
+    import retnet_retention_chunkwise_b200 as ret
+    from retnet_retention_chunkwise_b200 import sequence
+    ret.library()
+    dist = Dist(args.gpus)
+    own_group = False
+    if not tdist.is_initialized():  # one rank: a one-rank NCCL group of its own
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        store = tdist.TCPStore("127.0.0.1", port, 1, True, timeout=datetime.timedelta(seconds=60))
+        tdist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                                 device_id=torch.device("cuda", torch.cuda.current_device()))
+        own_group = True
+    w = inputs.WORKLOADS["long_context_bf16"]
+    C, L_run = 128, w.L
+    q, k, v = gpu_qkv(w.B, w.H, L_run, w.dk, w.dv, seed=dist.rank)
+    gam = w.gammas()
+    lens = [L_run] * dist.world
+
+    def step():
+        sequence.chunkwise_sequence_sharded(q, k, v, gam, C, lens=lens)
+
+    steps = min(args.steps, 200)
+    with ClockSampler(dist.local) as clk:
+        _, total = time_calls(step, steps, args.warmup, dist)
+    assert ret.device_status() == 0
+    t_ms = dist.max(total / steps)
+    value = dist.sum(w.B * L_run * steps) / (t_ms * 1e-3 * steps)
+    line = {"metric": METRIC, "mode": "sequence", "value": value, "unit": "tokens/s", "n_gpus": dist.world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "long_context_bf16 sequence cut across ranks: B=1 H=16 dk=128 dv=256 C=128, "
+                                   f"{L_run} tokens per rank", "seq_len": L_run * dist.world,
+                       "parallelism": f"sequence-sharded over {dist.world} ranks, one all-gather of "
+                                      "B*H*dk*dv fp32 run sums per step"},
+            "clocks": clk.summary(), "gpu_launches": None}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    if own_group:
+        tdist.destroy_process_group()
+    dist.close()
+
+
 # ----------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -669,6 +790,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-forms", action="store_true", help="headline only")
+    ap.add_argument("--mode", default="headline", choices=["headline", "sequence"],
+                    help="sequence: time one long-context sequence cut across the ranks instead")
     ap.add_argument("--profile", default=None,
                     help="run only one kind of call for a profiler, no JSON: "
                          "chunkwise:B,H,L,dk,dv,C | parallel:B,H,L,dk,dv | decode:B,H,dk,dv | "
@@ -682,6 +805,9 @@ def main():
     if args.profile:
         run_profile_case(args)
         return
+    if args.mode == "sequence":
+        run_sequence(args)
+        return
     import retnet_retention_chunkwise_b200 as ret
     ret.library()
     dist = Dist(args.gpus)
@@ -690,10 +816,16 @@ def main():
     e2e = bench_e2e(ret, args, dist)
     forms = {}
     if not args.no_forms:
-        forms["decode"] = bench_decode(ret, args, dist, peaks)
-        forms["decode_batch1_graph"] = bench_decode_graph(ret, args, dist, peaks)
+        # the line is long: decode goes last, so a reader of its tail sees it
         forms.update(bench_small(ret, args, dist, peaks))
-    cpu = cpu_baseline() if (dist.rank == 0 and dist.world == 1) else None
+        forms["headline_sustained"] = bench_headline_sustained(ret, args, dist, peaks)
+        forms["decode_batch1_graph"] = bench_decode_graph(ret, args, dist, peaks)
+        forms["decode"] = bench_decode(ret, args, dist, peaks)
+    cpu = None
+    if dist.rank == 0 and dist.world == 1:
+        cpu = cpu_baseline()
+        if not args.no_forms:
+            cpu["per_config"] = oracle_timings()
     w = HEADLINE
     line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": dist.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],

@@ -133,9 +133,9 @@ RET_API ret_status retention_recurrent_step(const void* q, const void* k, const 
  *     (retention_chunkwise_workspace_bytes() > 16 MiB) return
  *     RET_EUNSUPPORTED before anything is launched; shapes that need no split
  *     never touch the array.
- *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any
- *     stream capture.
+ *   - The first call on a device, whatever its shape, looks up the array's
+ *     device address (once per device, with that device current); make that
+ *     first call before any stream capture.
  *   - Every call uses the same array and leaves its contents behind.  Nothing
  *     in it has to start at zero (each call writes every slot it reads), but
  *     calls that can run at the same time on the GPU -- different streams, or
@@ -277,8 +277,10 @@ RET_API size_t retention_chunkwise_gn_workspace_bytes(int chunk, ret_shape s, re
 /*
  * retention_chunkwise_gn with the output gate: y receives
  * GroupNorm(y) * act(gate) (see retention_groupnorm_gated), in place.  gate:
- * device [B][H][L][dv] in the call's dtype, 16-byte aligned, not y; NULL for no
- * gate.  act: a ret_gate_act.  Workspace: retention_chunkwise_gn_workspace_bytes().
+ * device [B][H][L][dv] in the call's dtype, 16-byte aligned, sharing no byte
+ * with y (RET_EINVAL otherwise: y is normalised in place while the gate is
+ * read); NULL for no gate.  act: a ret_gate_act.  Workspace:
+ * retention_chunkwise_gn_workspace_bytes().
  */
 RET_API ret_status retention_chunkwise_gn_gated(const void* q, const void* k, const void* v, const float* gamma,
                                                 void* y, const float* state_in, float* state_out, int chunk,

@@ -14,6 +14,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/retention.h"
 #include "chunkwise_tc.cuh"
 #include "chunkwise_wide.cuh"
@@ -28,6 +30,16 @@
 namespace {
 
 using namespace ret;
+
+// An NVTX range around each compute call of the C ABI, named after the call,
+// so a profiler's timeline shows which library call launched which kernels.
+// Without a profiler attached the push and pop return at once.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Wall-clock budget of any single wait inside a kernel.  A healthy wait is
 // microseconds; this only bounds a kernel whose pipeline broke.
@@ -595,6 +607,7 @@ ret_status retention_get_device_status(void* stream) {
 
 ret_status retention_recurrent_step(const void* q, const void* k, const void* v, const float* gamma,
                                     void* y, float* state, ret_shape s, ret_dtype dt, void* stream) {
+  NvtxRange nvtx_range("retention_recurrent_step");
   ret_status rc = check_shape(s, false);
   if (rc != RET_OK) return rc;
   if (!q || !k || !v || !y || !state) return RET_EINVAL;
@@ -629,6 +642,7 @@ ret_status retention_recurrent_step(const void* q, const void* k, const void* v,
 
 ret_status retention_parallel(const void* q, const void* k, const void* v, const float* gamma, void* y,
                               ret_shape s, ret_dtype dt, void* stream) {
+  NvtxRange nvtx_range("retention_parallel");
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
@@ -675,6 +689,7 @@ size_t retention_chunkwise_workspace_bytes(int chunk, ret_shape s, ret_dtype dt)
 ret_status retention_chunkwise(const void* q, const void* k, const void* v, const float* gamma, void* y,
                                const float* state_in, float* state_out, int chunk, ret_shape s,
                                ret_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("retention_chunkwise");
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
@@ -733,6 +748,7 @@ size_t retention_chunkwise_state_workspace_bytes(int chunk, ret_shape s, ret_dty
 ret_status retention_chunkwise_state(const void* k, const void* v, const float* gamma, const float* state_in,
                                      float* state_out, int chunk, ret_shape s, ret_dtype dt, void* workspace,
                                      size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("retention_chunkwise_state");
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
@@ -781,6 +797,7 @@ ret_status retention_chunkwise_state(const void* k, const void* v, const float* 
 
 ret_status retention_state_fold(const float* parts, const int* lens, int n, const float* gamma,
                                 const float* state_in, float* state_out, ret_shape s, void* stream) {
+  NvtxRange nvtx_range("retention_state_fold");
   ret_status rc = check_shape(s, false);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
@@ -805,18 +822,18 @@ ret_status retention_state_fold(const float* parts, const int* lens, int n, cons
 ret_status retention_chunkwise_static_ws(const void* q, const void* k, const void* v, const float* gamma,
                                          void* y, const float* state_in, float* state_out, int chunk,
                                          ret_shape s, ret_dtype dt, void* stream) {
+  NvtxRange nvtx_range("retention_chunkwise_static_ws");
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
   if (chunk < 1) return RET_EINVAL;
+  // The address is looked up on every call (cached per device after the
+  // first), so the first call on a device does the lookup whatever its shape.
+  void* ws = static_ws_address(&rc);
+  if (rc != RET_OK) return rc;
   const size_t need = retention_chunkwise_workspace_bytes(chunk, s, dt);
   if (need > kStaticWsBytes) return RET_EUNSUPPORTED;  // beyond the fixed scratch
-  void* ws = nullptr;
-  if (need > 0) {
-    ws = static_ws_address(&rc);
-    if (rc != RET_OK) return rc;
-  }
-  return retention_chunkwise(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, ws,
+  return retention_chunkwise(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, need > 0 ? ws : nullptr,
                              need > 0 ? kStaticWsBytes : 0, stream);
 }
 
@@ -834,6 +851,7 @@ ret_status retention_chunkwise_host(const void* q_host, const void* k_host, cons
                                     void* y_dev, const float* state_in, float* state_out, int chunk,
                                     ret_shape s, ret_dtype dt, void* workspace, size_t workspace_bytes,
                                     int n_groups, void* stream) {
+  NvtxRange nvtx_range("retention_chunkwise_host");
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
@@ -921,6 +939,7 @@ ret_status retention_chunkwise_host(const void* q_host, const void* k_host, cons
 
 ret_status retention_groupnorm_gated(const void* y, const void* gate, void* out, float eps, const float* weight,
                                      const float* bias, int act, ret_shape s, ret_dtype dt, void* stream) {
+  NvtxRange nvtx_range("retention_groupnorm_gated");
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
@@ -958,10 +977,17 @@ ret_status retention_chunkwise_gn_gated(const void* q, const void* k, const void
                                         ret_dtype dt, float eps, const float* weight, const float* bias,
                                         const void* gate, int act, void* workspace, size_t workspace_bytes,
                                         void* stream) {
+  NvtxRange nvtx_range("retention_chunkwise_gn_gated");
   if (!(eps >= 0.f) || !std::isfinite(eps)) return RET_EINVAL;
   if (act < kGateNone || act > kGateSigmoid) return RET_EINVAL;
   if (s.dv > kGN_MaxDv) return RET_EUNSUPPORTED;
-  if (gate && s.L > 0 && (!aligned16(gate) || gate == y)) return RET_EINVAL;
+  if (gate && s.L > 0) {
+    // y is normalised in place while the gate is read: the two must not share
+    // a byte (an offset view of y would be read after rows of it were written)
+    const size_t bytes = (size_t)s.B * s.H * s.L * s.dv * (dt == RET_BF16 ? 2 : 4);
+    const uintptr_t g0 = reinterpret_cast<uintptr_t>(gate), y0 = reinterpret_cast<uintptr_t>(y);
+    if (!aligned16(gate) || (g0 < y0 + bytes && y0 < g0 + bytes)) return RET_EINVAL;
+  }
   ret_status rc = retention_chunkwise(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, workspace,
                                       workspace_bytes, stream);
   if (rc != RET_OK || s.L == 0) return rc;
@@ -976,6 +1002,7 @@ size_t retention_parallel_backward_workspace_bytes(ret_shape s, ret_dtype dt) {
 ret_status retention_parallel_backward(const void* q, const void* k, const void* v, const float* gamma,
                                        const void* dy, void* dq, void* dk, void* dv, ret_shape s, ret_dtype dt,
                                        void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("retention_parallel_backward");
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
@@ -1052,6 +1079,7 @@ ret_status retention_chunkwise_backward_state(const void* q, const void* k, cons
                                               void* dq, void* dk, void* dv, float* dstate_in, int chunk,
                                               ret_shape s, ret_dtype dt, void* workspace, size_t workspace_bytes,
                                               void* stream) {
+  NvtxRange nvtx_range("retention_chunkwise_backward_state");
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;

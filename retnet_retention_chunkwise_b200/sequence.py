@@ -52,24 +52,34 @@ class CudaOps:
         return self._chunkwise(q, k, v, gamma, chunk, state_in=state_in)
 
 
-def chunkwise_sequence_sharded(q, k, v, gamma, chunk: int, *, state_in=None, group=None, ops=None):
+def chunkwise_sequence_sharded(q, k, v, gamma, chunk: int, *, state_in=None, group=None, ops=None, lens=None):
     """This rank's run of a sequence cut across the ranks of `group`.
 
     q, k, v: the run, [B,H,L_r,d] on this rank's device (runs in rank order make
     the sequence; lengths may differ).  state_in: the state before the whole
     sequence, fp32 [B,H,dk,dv], the same on every rank, or None (zero).
+    lens: the run length of every rank, in rank order, when the caller knows
+    them (e.g. from split_runs); then they are not exchanged and nothing waits
+    on the device between the collective and the fold.  None: they are
+    all-gathered with the sums and read back to the host.
     Returns (y_r, state after this run); on the last rank the latter is the
     state after the whole sequence."""
     import torch.distributed as dist
     ops = ops or CudaOps()
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
+    if lens is not None:
+        lens = [int(n) for n in lens]
+        if len(lens) != world or lens[rank] != q.shape[2] or min(lens) < 0:
+            raise ValueError("lens must hold every rank's run length, this rank's equal to q.shape[2]")
     d = ops.run_state(k, v, gamma, chunk)                      # 1. the run's own sum
     # 2. the exchange: rank i's sum lands in rows [i*B, (i+1)*B) of one tensor
     parts = torch.empty((world * d.shape[0],) + tuple(d.shape[1:]), dtype=d.dtype, device=d.device)
     dist.all_gather_into_tensor(parts, d.contiguous(), group=group)
     parts = parts.view((world,) + tuple(d.shape))
-    lens = torch.empty(world, dtype=torch.int64, device=d.device)
-    dist.all_gather_into_tensor(lens, torch.tensor([q.shape[2]], dtype=torch.int64, device=d.device), group=group)
-    s_r = ops.fold(parts[:rank], lens[:rank].tolist(), gamma, state_in)  # 3. the state at begin_r
+    if lens is None:
+        n = torch.empty(world, dtype=torch.int64, device=d.device)
+        dist.all_gather_into_tensor(n, torch.tensor([q.shape[2]], dtype=torch.int64, device=d.device), group=group)
+        lens = n.tolist()
+    s_r = ops.fold(parts[:rank], lens[:rank], gamma, state_in)  # 3. the state at begin_r
     return ops.chunkwise(q, k, v, gamma, chunk, s_r)           # 4. the run itself

@@ -59,8 +59,20 @@ def _g(*vals):
 
 FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
 
+# The validation tests pass made-up device addresses that the library must
+# refuse before any launch.  Were a check ever to regress on a machine with a
+# GPU, the call would launch kernels on those addresses and fault the device,
+# so these tests run only where no CUDA device is visible.
+try:
+    import torch as _torch
+    _DEVICE_VISIBLE = _torch.cuda.is_available()
+except Exception:  # pragma: no cover
+    _DEVICE_VISIBLE = False
+NO_DEVICE = pytest.mark.skipif(_DEVICE_VISIBLE, reason="made-up device addresses: host-only validation test")
+
 
 @pytest.mark.parametrize("gamma", [-0.01, 1.0001, float("nan"), float("inf")])
+@NO_DEVICE
 def test_bad_gamma_is_einval(lib, gamma):
     s = _abi.RetShape(1, 1, 8, 64, 128)
     assert lib.retention_parallel(FAKE, FAKE, FAKE, _g(gamma), FAKE, s, _abi.RET_BF16, None) == _abi.RET_EINVAL
@@ -70,6 +82,7 @@ def test_bad_gamma_is_einval(lib, gamma):
                                         None) == _abi.RET_EINVAL
 
 
+@NO_DEVICE
 def test_null_gamma_and_pointers_are_einval(lib):
     s = _abi.RetShape(1, 1, 8, 64, 128)
     assert lib.retention_parallel(FAKE, FAKE, FAKE, None, FAKE, s, _abi.RET_BF16, None) == _abi.RET_EINVAL
@@ -82,6 +95,7 @@ def test_null_gamma_and_pointers_are_einval(lib):
 
 @pytest.mark.parametrize("shape", [(0, 1, 8, 64, 128), (1, 0, 8, 64, 128), (1, 1, -1, 64, 128),
                                    (1, 1, 8, 0, 128), (1, 1, 8, 64, 0)])
+@NO_DEVICE
 def test_bad_shapes_are_einval(lib, shape):
     s = _abi.RetShape(*shape)
     g = _g(*([0.5] * max(shape[1], 1)))
@@ -89,6 +103,7 @@ def test_bad_shapes_are_einval(lib, shape):
                                    None, 0, None) == _abi.RET_EINVAL
 
 
+@NO_DEVICE
 def test_too_many_heads_is_unsupported(lib):
     H = _abi.RET_MAX_HEADS + 1
     s = _abi.RetShape(1, H, 8, 64, 128)
@@ -96,6 +111,7 @@ def test_too_many_heads_is_unsupported(lib):
                                   None) == _abi.RET_EUNSUPPORTED
 
 
+@NO_DEVICE
 def test_misaligned_pointers_are_einval(lib):
     s = _abi.RetShape(1, 1, 8, 64, 128)
     odd = ctypes.c_void_p(0x10008)
@@ -106,12 +122,14 @@ def test_misaligned_pointers_are_einval(lib):
 
 @pytest.mark.parametrize("chunk,dk,dv", [(8, 64, 128), (24, 64, 128), (272, 64, 128), (144, 256, 128),
                                          (256, 256, 512), (64, 96, 128), (64, 64, 192), (64, 512, 128)])
+@NO_DEVICE
 def test_unsupported_bf16_shapes(lib, chunk, dk, dv):
     s = _abi.RetShape(1, 1, 256, dk, dv)
     assert lib.retention_chunkwise(FAKE, FAKE, FAKE, _g(0.5), FAKE, None, None, chunk, s, _abi.RET_BF16,
                                    None, 0, None) == _abi.RET_EUNSUPPORTED
 
 
+@NO_DEVICE
 def test_zero_chunk_is_einval(lib):
     s = _abi.RetShape(1, 1, 8, 64, 128)
     assert lib.retention_chunkwise(FAKE, FAKE, FAKE, _g(0.5), FAKE, None, None, 0, s, _abi.RET_F32,
@@ -135,6 +153,7 @@ def test_workspace_query(lib):
     assert lib.retention_chunkwise_workspace_bytes(256, _abi.RetShape(1, 2, 8192, 256, 128), _abi.RET_BF16) == 0
 
 
+@NO_DEVICE
 def test_host_entry_validation(lib):
     s = _abi.RetShape(1, 2, 256, 64, 128)
     g = _g(0.5, 0.9)
@@ -157,6 +176,7 @@ def test_host_entry_workspace_query(lib):
     assert n > 0
 
 
+@NO_DEVICE
 def test_parallel_backward_validation(lib):
     s = _abi.RetShape(1, 2, 64, 64, 128)
     g = _g(0.5, 0.9)
@@ -171,6 +191,7 @@ def test_parallel_backward_validation(lib):
                 _abi.RetShape(1, 2, 64, 96, 128)) == _abi.RET_EUNSUPPORTED
 
 
+@NO_DEVICE
 def test_chunkwise_backward_state_validation(lib):
     # every case below returns before any launch
     s = _abi.RetShape(1, 2, 64, 64, 128)
@@ -197,6 +218,7 @@ def test_chunkwise_backward_state_validation(lib):
                                                   None) == _abi.RET_EINVAL  # gamma outside [0, 1]
 
 
+@NO_DEVICE
 def test_groupnorm_gated_validation(lib):
     s = _abi.RetShape(1, 2, 8, 1, 128)
     call = lambda gate, act, y=FAKE: lib.retention_groupnorm_gated(  # noqa: E731
@@ -211,6 +233,7 @@ def test_groupnorm_gated_validation(lib):
                                          _abi.RET_BF16, None) == _abi.RET_EUNSUPPORTED
 
 
+@NO_DEVICE
 def test_chunkwise_state_and_fold_validation(lib):
     # every case below returns before any launch
     s = _abi.RetShape(1, 2, 256, 128, 128)
@@ -242,6 +265,7 @@ def test_chunkwise_state_and_fold_validation(lib):
     assert fold(parts=ctypes.c_void_p(0x10004)) == _abi.RET_EINVAL
 
 
+@NO_DEVICE
 def test_state_fold_rejects_out_inside_parts(lib):
     s = _abi.RetShape(1, 2, 0, 16, 16)
     lens = (ctypes.c_int * 2)(5, 7)
@@ -271,6 +295,7 @@ def test_plain_c_caller():
     assert out.stdout.startswith("ok ")
 
 
+@NO_DEVICE
 def test_chunkwise_gn_gated_validation(lib):
     s = _abi.RetShape(1, 2, 64, 128, 128)
     g = _g(0.5, 0.9)
@@ -280,6 +305,10 @@ def test_chunkwise_gn_gated_validation(lib):
     assert call(FAKE, 1, eps=-1.0) == _abi.RET_EINVAL             # eps < 0
     assert call(ctypes.c_void_p(0x10008), 1) == _abi.RET_EINVAL   # gate not 16-byte aligned
     assert call(ctypes.c_void_p(0x20000), 1) == _abi.RET_EINVAL   # gate is y
+    # a gate that shares any byte with y (y is 2*64*128 bf16 = 0x8000 bytes at 0x20000)
+    assert call(ctypes.c_void_p(0x20010), 1) == _abi.RET_EINVAL   # a few rows into y
+    assert call(ctypes.c_void_p(0x27ff0), 1) == _abi.RET_EINVAL   # its last 16 bytes
+    assert call(ctypes.c_void_p(0x18010), 1) == _abi.RET_EINVAL   # ends inside y
 
 
 def test_missing_library_fails_loudly():

@@ -1,5 +1,6 @@
 """Host-side pieces of bench.py (no GPU): the algorithmic counts behind the
-roofline fractions, and the reading of the committed ncu summary."""
+roofline fractions, and the reading of the committed ncu traffic record."""
+import json
 import os
 import tempfile
 
@@ -24,17 +25,18 @@ def test_parallel_flops_counts_causal_pairs():
 def test_traffic_is_read_only_for_the_current_kernel_source():
     digest = bench.kernel_source_digest()
     assert len(digest) == 16
-    text = ("# summary\n\n- dram_bytes_per_launch: `123456`\n"
-            f"- kernel_source_sha256_16: `{digest}` (the kernel's source)\n")
-    stale = text.replace(digest, "0" * 16)
+    rec = {"kernel_source_sha256_16": digest, "dram_bytes_per_launch": 123456}
+    stale = dict(rec, kernel_source_sha256_16="0" * 16)
     orig = bench.TRAFFIC_FILE
     try:
         with tempfile.TemporaryDirectory() as d:
-            for body, want in ((text, 123456.0), (stale, None)):
-                p = os.path.join(d, "s.md")
+            for body, want in ((rec, 123456.0), (stale, None), ({}, None)):
+                p = os.path.join(d, "s.json")
                 with open(p, "w") as f:
-                    f.write(body)
+                    json.dump(body, f)
                 bench.TRAFFIC_FILE = p
                 assert bench.measured_traffic() == want
+            bench.TRAFFIC_FILE = os.path.join(d, "missing.json")
+            assert bench.measured_traffic() is None
     finally:
         bench.TRAFFIC_FILE = orig

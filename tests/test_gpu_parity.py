@@ -1,7 +1,8 @@
 """GPU parity: every kernel, through the C ABI, against the fp64 oracle.
 
-Metric (per tensor): max |gpu - oracle| / max |oracle|.  Bounds: 1e-4 for fp32
-inputs, 2e-2 for bf16 inputs (fp32 accumulation and state).  Both sides read the
+Metric: max |gpu - oracle| / max |oracle|, over each tensor and over each of
+its (b, h) slices on its own (tests/parity.py).  Bounds: 1e-4 for fp32 inputs,
+2e-2 for bf16 inputs (fp32 accumulation and state).  Both sides read the
 same seeded bytes; the oracle widens them to fp64 exactly.
 """
 import math
@@ -13,17 +14,13 @@ import torch
 import oracle
 import retnet_retention_chunkwise_b200 as ret
 from retnet_retention_chunkwise_b200 import inputs
+from tests.parity import rel
 
 pytestmark = pytest.mark.gpu
 
 TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
 
 
-def rel(gpu, ref):
-    g = gpu.detach().double().cpu().numpy() if isinstance(gpu, torch.Tensor) else np.asarray(gpu)
-    ref = np.asarray(ref, dtype=np.float64)
-    assert np.all(np.isfinite(g)), "non-finite GPU output"
-    return float(np.max(np.abs(g - ref)) / max(np.max(np.abs(ref)), 1e-30))
 
 
 def dev(*ts):

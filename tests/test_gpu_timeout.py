@@ -8,14 +8,11 @@ import torch
 import oracle
 import retnet_retention_chunkwise_b200 as ret
 from retnet_retention_chunkwise_b200 import _abi, inputs
+from tests.parity import rel
 
 pytestmark = pytest.mark.gpu
 
 
-def _rel(a, b):
-    import numpy as np
-    a = a.double().cpu().numpy()
-    return float(np.max(np.abs(a - b)) / np.max(np.abs(b)))
 
 
 @pytest.mark.parametrize("dk,dv,C", [(128, 128, 128), (256, 256, 128), (128, 128, 256)])
@@ -34,4 +31,4 @@ def test_dropped_load_times_out_then_recovers(monkeypatch, dk, dv, C):
     y, s = ret.chunkwise(qd, kd, vd, gam, C, workspace=None)
     assert ret.device_status() == _abi.RET_OK
     y_ref, s_ref = oracle.recurrent(q, k, v, gam)
-    assert _rel(y, y_ref) <= 2e-2 and _rel(s, s_ref) <= 2e-2
+    assert rel(y, y_ref) <= 2e-2 and rel(s, s_ref) <= 2e-2

@@ -55,7 +55,7 @@ def _inputs(B, H, L, dk, dv, seed):
     return q, k, v, s_in
 
 
-def _worker(rank, world, port, out_dir, L, chunk, uneven):
+def _worker(rank, world, port, out_dir, L, chunk, uneven, known_lens=False):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
@@ -64,12 +64,14 @@ def _worker(rank, world, port, out_dir, L, chunk, uneven):
         gamma = np.array([0.9, 0.6])
         if uneven:  # runs of arbitrary lengths, not block-aligned
             cuts = [0, 5, 6, 17, L][: world] + [L]
-            b, e = cuts[rank], cuts[rank + 1]
         else:
-            b, e = sequence.split_runs(L, chunk, rank, world)
+            cuts = [sequence.split_runs(L, chunk, r, world)[0] for r in range(world)] + [L]
+        b, e = cuts[rank], cuts[rank + 1]
+        # the caller's own run lengths (no length exchange), or None (exchanged)
+        lens = [cuts[r + 1] - cuts[r] for r in range(world)] if known_lens else None
         run = lambda t: t[:, :, b:e].contiguous()  # noqa: E731
         y, s = sequence.chunkwise_sequence_sharded(run(q), run(k), run(v), gamma, chunk, state_in=s_in,
-                                                   ops=OracleOps())
+                                                   ops=OracleOps(), lens=lens)
         torch.save({"y": y, "s": s, "b": b, "e": e}, os.path.join(out_dir, f"r{rank}.pt"))
     finally:
         dist.destroy_process_group()
@@ -81,11 +83,12 @@ def _free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("world,L,chunk,uneven", [(2, 40, 8, False), (3, 37, 4, False), (3, 23, 4, True),
-                                                  (4, 50, 4, True)])
-def test_sequence_sharded_exchange_gloo(world, L, chunk, uneven):
+@pytest.mark.parametrize("world,L,chunk,uneven,known_lens", [(2, 40, 8, False, False), (3, 37, 4, False, False),
+                                                             (3, 23, 4, True, False), (4, 50, 4, True, False),
+                                                             (2, 40, 8, False, True), (3, 23, 4, True, True)])
+def test_sequence_sharded_exchange_gloo(world, L, chunk, uneven, known_lens):
     with tempfile.TemporaryDirectory() as out_dir:
-        mp.start_processes(_worker, args=(world, _free_port(), out_dir, L, chunk, uneven), nprocs=world,
+        mp.start_processes(_worker, args=(world, _free_port(), out_dir, L, chunk, uneven, known_lens), nprocs=world,
                            join=True, start_method="spawn")
         res = [torch.load(os.path.join(out_dir, f"r{r}.pt")) for r in range(world)]
     q, k, v, s_in = _inputs(1, 2, L, 3, 4, 5)
