@@ -57,7 +57,9 @@ typedef enum {
   RET_EINVAL = 1,        /* null pointer, bad size, gamma outside [0,1], misalignment */
   RET_EUNSUPPORTED = 2,  /* valid request that this library does not implement */
   RET_ECUDA = 3,         /* a CUDA runtime call failed (launch, attribute, copy) */
-  RET_ETIMEOUT = 4       /* a kernel's bounded wait expired (device status) */
+  RET_ETIMEOUT = 4,      /* a kernel's bounded wait expired (device status) */
+  RET_EBOUNDS = 5        /* bounds-checked builds only (-DRET_BOUNDS_CHECK): an index
+                            check in a kernel failed and its access was skipped */
 } ret_status;
 
 typedef enum { RET_F32 = 0, RET_BF16 = 1 } ret_dtype;
@@ -296,20 +298,22 @@ RET_API ret_status retention_chunkwise_gn_gated(const void* q, const void* k, co
  *     dv_m = sum_{n>=m} gamma^(n-m) (q_n . k_m) dy_n
  * (the derivative of the retention sum of the page "Retentive Networks --
  * Microsoft ...", section "Il meccanismo"; the pages give no backward pass).
- * Each is a retention sum itself: dq on (dy, v, k), and dk, dv on the
- * time-reversed sequences; the call runs three parallel-form launches and the
- * reversals on `stream`.
+ * Each is a retention sum itself: dq on (dy, v, k), and dk, dv the
+ * anti-causal sums (n >= m) on (v, dy, q) and (k, q, dy), which the kernels
+ * walk from the end of the sequence; the call runs three parallel-form
+ * launches on `stream` and copies nothing.
  * q, k, dq, dk : device [B][H][L][dk]; v, dy, dv : device [B][H][L][dv]; all in
  *             the call's dtype, 16-byte aligned.
- * workspace : device scratch of retention_parallel_backward_workspace_bytes()
- *             bytes, 256-byte aligned (reversed inputs and results).
+ * workspace : not used (retention_parallel_backward_workspace_bytes() is 0);
+ *             NULL is accepted.
  * Supported: bf16 with dk and dv in {64, 128, 256}; fp32 with dk, dv <= 256.
  */
 RET_API ret_status retention_parallel_backward(const void* q, const void* k, const void* v, const float* gamma,
                                                const void* dy, void* dq, void* dk, void* dv, ret_shape s,
                                                ret_dtype dt, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Workspace size of retention_parallel_backward. */
+/* Workspace size of retention_parallel_backward: 0 (kept for callers that size
+ * a workspace before the call). */
 RET_API size_t retention_parallel_backward_workspace_bytes(ret_shape s, ret_dtype dt);
 
 /*
@@ -318,11 +322,14 @@ RET_API size_t retention_parallel_backward_workspace_bytes(ret_shape s, ret_dtyp
  * computed by retention_chunkwise, so the cost grows linearly with L.  No
  * state gradient: the forward call it differentiates starts from a zero state
  * and its state_out is not used.
+ * dk and dv are the anti-causal sums, walked from the end of the sequence
+ * (their blocks are of min(chunk, 128) rows; the result does not depend on the
+ * block length beyond rounding).  Nothing is copied.
  * Supported: bf16 with dk and dv in {128, 256} (each is the value width of one
  * of the three calls) and a chunk the chunkwise path takes for both; fp32 with
- * dk, dv <= 256 and chunk <= 128.  Workspace: the reversal buffers plus the
- * chunkwise calls' sequence-split scratch,
- * retention_chunkwise_backward_workspace_bytes() bytes, 256-byte aligned.
+ * dk, dv <= 256 and chunk <= 128.  Workspace: the chunkwise calls'
+ * sequence-split scratch, retention_chunkwise_backward_workspace_bytes() bytes
+ * (0 when no call splits; NULL is then accepted), 256-byte aligned.
  */
 RET_API ret_status retention_chunkwise_backward(const void* q, const void* k, const void* v, const float* gamma,
                                                 const void* dy, void* dq, void* dk, void* dv, int chunk, ret_shape s,
@@ -360,7 +367,7 @@ RET_API size_t retention_chunkwise_backward_workspace_bytes(int chunk, ret_shape
  * Supported shapes, dtypes and chunks: those of retention_chunkwise_backward.
  * workspace : retention_chunkwise_backward_state_workspace_bytes() bytes,
  *             256-byte aligned (that of retention_chunkwise_backward plus
- *             three fp32 states when any state pointer is given).
+ *             three fp32 states, needed when any state pointer is given).
  */
 RET_API ret_status retention_chunkwise_backward_state(const void* q, const void* k, const void* v,
                                                       const float* gamma, const void* dy, const float* state_in,
@@ -373,7 +380,8 @@ RET_API size_t retention_chunkwise_backward_state_workspace_bytes(int chunk, ret
 
 /* Synchronises `stream`, then returns and clears the device status word:
  * RET_OK, RET_ETIMEOUT if a kernel's bounded wait expired since the last
- * query, or RET_ECUDA if the stream reported an error. */
+ * query, RET_EBOUNDS if a bounds-checked build found an index out of range,
+ * or RET_ECUDA if the stream reported an error. */
 RET_API ret_status retention_get_device_status(void* stream);
 
 /* Static, NUL-terminated name of a status code. */

@@ -10,9 +10,11 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libretention.so")
+# RETENTION_LIBRARY selects another build of the same library (the
+# bounds-checked one for tests); by default the in-tree libretention.so.
+LIB_PATH = os.environ.get("RETENTION_LIBRARY") or os.path.join(HERE, "libretention.so")
 
-RET_OK, RET_EINVAL, RET_EUNSUPPORTED, RET_ECUDA, RET_ETIMEOUT = 0, 1, 2, 3, 4
+RET_OK, RET_EINVAL, RET_EUNSUPPORTED, RET_ECUDA, RET_ETIMEOUT, RET_EBOUNDS = 0, 1, 2, 3, 4, 5
 RET_F32, RET_BF16 = 0, 1
 RET_MAX_HEADS = 1024
 

@@ -14,6 +14,10 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libretention.so")
+# The same library with index checks in the kernels (-DRET_BOUNDS_CHECK): a
+# failed check skips its access and the device status reads RET_EBOUNDS.  For
+# tests only; select it with RETENTION_LIBRARY=<path>.
+LIB_BOUNDS_CHECK = os.path.join(HERE, "libretention_bc.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -41,6 +45,13 @@ def build(out: str = LIB, extra=(), verbose: bool = False) -> str:
     return out
 
 
+def build_bounds_check(out: str = LIB_BOUNDS_CHECK, verbose: bool = False) -> str:
+    return build(out, extra=("-DRET_BOUNDS_CHECK",), verbose=verbose)
+
+
 if __name__ == "__main__":
     build(verbose="-v" in sys.argv)
     print(LIB)
+    if "--bounds-check" in sys.argv:
+        build_bounds_check()
+        print(LIB_BOUNDS_CHECK)

@@ -1,15 +1,15 @@
-// backward.cuh -- pieces of the backward pass of the parallel form.
+// backward.cuh -- pieces of the backward passes around the three retention sums.
 //
 // With y_n = sum_{m<=n} gamma^(n-m) (q_n . k_m) v_m (page "Retentive Networks
 // -- Microsoft ...", section "Il meccanismo: Multi-Scale Retention") and an
 // upstream gradient dy, the chain rule gives three sums of the same kind:
 //     dq_n = sum_{m<=n} gamma^(n-m) (dy_n . v_m) k_m     = retention(dy, v, k)_n
-//     dk_m = sum_{n>=m} gamma^(n-m) (dy_n . v_m) q_n
-//     dv_m = sum_{n>=m} gamma^(n-m) (q_n . k_m) dy_n
-// The last two run backwards in time: with R the reversal of the sequence
-// axis, dk = R(retention(R v, R dy, R q)) and dv = R(retention(R k, R q, R dy)).
-// So the backward pass is three launches of the forward parallel kernel plus
-// the reversals below.
+//     dk_m = sum_{n>=m} gamma^(n-m) (v_m . dy_n) q_n     = retention_rev(v, dy, q)_m
+//     dv_m = sum_{n>=m} gamma^(n-m) (k_m . q_n) dy_n     = retention_rev(k, q, dy)_m
+// The last two run backwards in time (anti-causal); the parallel and chunkwise
+// kernels take them directly (their REV instantiations walk the key tiles or
+// blocks from the end), so the backward pass is three launches of the forward
+// kernels with no copy of the inputs.
 //
 // A carried state (state_in S0, state_out S_out with upstream gradient dS_out)
 // adds, from y_n += gamma^(n+1) q_n S0 and S_out = gamma^L S0 +
@@ -17,11 +17,12 @@
 //     dq_n += gamma^(n+1) dy_n S0^T
 //     dk_m += gamma^(L-1-m) v_m dS_out^T,   dv_m += gamma^(L-1-m) k_m dS_out
 //     dS0   = gamma^L dS_out + sum_n gamma^(n+1) q_n^T dy_n
-// Each is the initial-state term of one of the three sums: in reversed time
-// m' = L-1-m the factor gamma^(L-1-m) = gamma^(m'+1) / gamma, so
-//     dq = retention(dy, v, k;          state_in S0^T)
-//     dk = R retention(R v, R dy, R q;  state_in (dS_out / gamma)^T)
-//     dv = R retention(R k, R q, R dy;  state_in dS_out / gamma)
+// Each is the initial-state term of one of the three sums: the anti-causal sum
+// started from S_in adds gamma^(L-m) a_m S_in, and gamma^(L-1-m) =
+// gamma^(L-m) / gamma, so
+//     dq = retention(dy, v, k;         state_in S0^T)
+//     dk = retention_rev(v, dy, q;     state_in (dS_out / gamma)^T)
+//     dv = retention_rev(k, q, dy;     state_in dS_out / gamma)
 // and the last sum's state_out T = sum_n gamma^n q_n^T dy_n + gamma^(L-1)
 // dS_out gives dS0 = gamma T.  Heads whose gamma is below kBwdMinGamma take a
 // zero initial state in the dk and dv sums instead (1 / gamma would overflow):
@@ -36,22 +37,6 @@
 #include "decode.cuh"  // HeadGamma
 
 namespace ret {
-
-// out[bh][L-1-n][:] = in[bh][n][:] for rows of `row_bytes` bytes, copied in
-// units of U (uint4 when row_bytes % 16 == 0, else uint32_t or uint16_t).
-template <typename U>
-__global__ void __launch_bounds__(256) reverse_rows_kernel(const U* __restrict__ in, U* __restrict__ out,
-                                                           long long BH, int L, int units_per_row) {
-  const long long total = BH * L * (long long)units_per_row;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const long long row = e / units_per_row;
-    const int u = (int)(e % units_per_row);
-    const long long bh = row / L;
-    const int n = (int)(row % L);
-    out[(bh * L + (L - 1 - n)) * units_per_row + u] = in[e];
-  }
-}
 
 constexpr float kBwdMinGamma = 8.673617379884035e-19f;  // 2^-60
 

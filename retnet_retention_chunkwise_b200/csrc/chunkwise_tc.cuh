@@ -219,7 +219,7 @@ __device__ __forceinline__ float cw_rho_first(bool rescaled, float g0) {
   return (rescaled && g0 >= 0x1p-64f) ? g0 : 1.f;
 }
 
-template <int DK>
+template <int DK, bool REV>
 __global__ void __launch_bounds__(kCW_MainThreads, 1)
 chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapY,
@@ -268,6 +268,12 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   const int c_begin = seg * a.seg_chunks;
   const int c_end = min(c_begin + a.seg_chunks, n_total);
   const int nck = max(c_end - c_begin, 0);
+  // Step it of the walk takes block blk_idx(it): forward from the segment's
+  // first block, REV (the anti-causal sum) from its last block down.
+  auto blk_idx = [&](int it) { return REV ? c_end - 1 - it : c_begin + it; };
+  auto blk_t0 = [&](int it) { return blk_idx(it) * C; };
+  auto blk_len = [&](int it) { return min(C, a.L - blk_t0(it)); };
+  const int l_first = nck > 0 ? blk_len(0) : 0;
   const int cta_id = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
   (void)cta_id;
   RET_TRACE_INIT();
@@ -331,7 +337,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       const uint32_t qk_bytes = (uint32_t)DK * (uint32_t)C * 2u;
       const uint32_t v_bytes = (uint32_t)kCW_DVT * (uint32_t)C * 2u;
       for (int it = 0; it < min(NS, nck); ++it) {
-        const int t0 = (c_begin + it) * C;
+        const int t0 = blk_t0(it);
         for (int b = 0; b < DK / 64; ++b) {
           tma_prefetch_l2_3d(&mapK, b * 64, t0, bh);
           tma_prefetch_l2_3d(&mapQ, b * 64, t0, bh);
@@ -342,10 +348,10 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       for (int it = 0; it < nck; ++it) {
         const int s = it % NS;
         const uint32_t par = ((it / NS) - 1) & 1;
-        const int t0 = (c_begin + it) * C;
+        const int t0 = blk_t0(it);
         if (it >= NS && !mbar_wait(&emptyK[s], par, abort_flag, a.lim)) break;
         RET_TRACE_STAMP(cta_id, it, 0);
-        if (c_begin + it != a.debug_drop_block) {  // fault injection: a load that never lands
+        if (blk_idx(it) != a.debug_drop_block) {  // fault injection: a load that never lands
           mbar_arrive_expect_tx(&fullK[s], qk_bytes);
           for (int b = 0; b < DK / 64; ++b)
             tma_load_3d(sK + s * sp.k_stage + b * C * 128, &mapK, &fullK[s], b * 64, t0, bh);
@@ -360,7 +366,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           tma_load_3d(sV + s * sp.v_stage + b * C * 128, &mapV, &fullV[s], vt * kCW_DVT + b * 64, t0, bh);
         issued = it + 1;
         if (it + NS < nck) {
-          const int tp = t0 + NS * C;
+          const int tp = blk_t0(it + NS);
           for (int b = 0; b < DK / 64; ++b) {
             tma_prefetch_l2_3d(&mapK, b * 64, tp, bh);
             tma_prefetch_l2_3d(&mapQ, b * 64, tp, bh);
@@ -450,7 +456,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   } else if (warp >= kWarpZBase) {
     // ---------------------------------------------------- V group (4 warps)
     const uint32_t t = threadIdx.x - kWarpZBase * 32;
-    float rho = cw_rho_first(rescaled, pw[max(min(C, a.L - c_begin * C), 0)]);
+    float rho = cw_rho_first(rescaled, pw[l_first]);
     for (int it = 0; it < nck; ++it) {
       const int s = it % NS;
       if (!mbar_wait(&fullV[s], (it / NS) & 1, abort_flag, a.lim)) break;
@@ -458,12 +464,12 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       // block's O was drained.
       if (!rescaled && !mbar_wait(ofree, it & 1, abort_flag, a.lim)) break;
       tc_fence_after();
-      const int l = min(C, a.L - (c_begin + it) * C);
+      const int l = min(C, a.L - blk_t0(it));
       uint8_t* vs = sV + s * sp.v_stage;
       if (rescaled) {
         // row j of the V tile scaled in place by zeta_j = gamma^(l-1-j) (0 past the end)
-        if ((int)t < C) {
-          const float zs = (((int)t < l) ? pw[l - 1 - (int)t] : 0.f) * __frcp_rn(rho);  // zeta / rho
+        if ((int)t < C && RET_BC(s < NS, 105)) {
+          const float zs = (((int)t < l) ? pw[REV ? (int)t : l - 1 - (int)t] : 0.f) * __frcp_rn(rho);  // zeta / rho
           scale_row_sw128(vs, t, zs);
           scale_row_sw128(vs + C * 128, t, zs);
         }
@@ -484,12 +490,13 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const uint32_t j = (uint32_t)j0 + 2u * u;
+            if (!RET_BC(j + 1 < (uint32_t)C + 16u, 106)) break;
             const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vt_s + j * 128 + ((vchunk ^ (j & 7)) << 4) + vbyte);
             const uint32_t w1 =
                 *reinterpret_cast<const uint32_t*>(vt_s + (j + 1) * 128 + ((vchunk ^ ((j + 1) & 7)) << 4) + vbyte);
             const uint32_t pr = __byte_perm(w0, w1, sel);
-            const float z0 = ((int)j < l) ? pw[l - 1 - (int)j] : 0.f;
-            const float z1 = ((int)j + 1 < l) ? pw[l - 2 - (int)j] : 0.f;
+            const float z0 = ((int)j < l) ? pw[REV ? (int)j : l - 1 - (int)j] : 0.f;
+            const float z1 = ((int)j + 1 < l) ? pw[REV ? (int)j + 1 : l - 2 - (int)j] : 0.f;
             w[u] = pack_bf16x2(bf16lo_to_f32(pr) * z0, bf16hi_to_f32(pr) * z1);
           }
           // When C % 32 == 16 the last piece covers 16 rows past C (zeta = 0
@@ -502,7 +509,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       }
       mbar_arrive(&zready[s]);
       if (t == 0) RET_TRACE_STAMP(cta_id, it, 3);
-      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[min(C, a.L - (c_begin + it) * C - C)]);
+      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[blk_len(it + 1)]);
     }
   } else if (warp >= kWarpSBase) {
     // ---------------------------------------------------- S group (4 warps)
@@ -513,7 +520,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     const uint32_t lane_off = (uint32_t)((warp - kWarpSBase) * 32) << 16;
     const int v = vt * kCW_DVT + (int)v_loc;
     const size_t dkdv = (size_t)DK * a.dv;
-    const float g0 = pw[max(min(C, a.L - c_begin * C), 0)];
+    const float g0 = pw[l_first];
     float rho = cw_rho_first(rescaled, g0);
     {
       const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
@@ -527,7 +534,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         uint32_t w[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          const float sv = src ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
+          const float sv = (src && RET_BC(d0 + u < DK && v < a.dv, 104)) ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
           x[u] = gc * sv;
           w[u] = __float_as_uint(gu * sv);
         }
@@ -544,9 +551,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       if (!mbar_wait(ocross, it & 1, abort_flag, a.lim)) break;
       if (v_loc == 0) RET_TRACE_STAMP(cta_id, it, 10);
       tc_fence_after();
-      const int t0 = (c_begin + it) * C;
+      const int t0 = blk_t0(it);
       if (it < nck - 1) {
-        const float gn = pw[min(C, a.L - t0 - C)];
+        const float gn = pw[blk_len(it + 1)];
         const float rho_n = rescaled ? cw_rho_next(rho, gn) : 1.f;
         const bool write_back = !rescaled || rho_n == 1.f;
         const float mult = rescaled ? gn * rho : gn;
@@ -576,12 +583,13 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         tc_fence_before();
         mbar_arrive(sready);
         if (v_loc == 0) RET_TRACE_STAMP(cta_id, it, 8);
-      } else if (a.state_out && seg == a.n_seg - 1) {
+      } else if (a.state_out && seg == (REV ? 0 : a.n_seg - 1)) {
         float* so = a.state_out + (size_t)bh * dkdv;
         for (int d0 = 0; d0 < DK; d0 += 32) {
           uint32_t sr[32];
           tmem_ld32(tm + lane_off + TM_S + d0, sr);
           tmem_ld_wait();
+          if (!RET_BC(d0 + 32 <= DK && v < a.dv, 103)) continue;
 #pragma unroll
           for (int u = 0; u < 32; ++u) so[(size_t)(d0 + u) * a.dv + v] = rho * __uint_as_float(sr[u]);
         }
@@ -593,13 +601,14 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     const int r = (int)threadIdx.x;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int row_lo = warp * 32;  // rows of this warp: [row_lo, row_lo + 32)
-    float rho = cw_rho_first(rescaled, pw[max(min(C, a.L - c_begin * C), 0)]);
+    float rho = cw_rho_first(rescaled, pw[l_first]);
     mbar_arrive(ofree);            // O starts free
     for (int it = 0; it < nck; ++it) {
       const int pb = it % NP;
-      const int t0 = (c_begin + it) * C;
+      const int t0 = blk_t0(it);
       const int l = min(C, a.L - t0);
       if (!mbar_wait(&pfull[pb], (it / NP) & 1, abort_flag, a.lim)) break;
+      (void)RET_BC(l >= 1 && l <= C && t0 >= 0 && t0 < a.L, 107);
       tc_fence_after();
       // P -> P~ in place (two bf16 per column).  Rows past the block end read
       // zero Q rows and columns past it zero K rows, so P is already 0 there.
@@ -611,34 +620,34 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         tmem_ld32(tp + j0, pr);
         tmem_ld_wait();
         uint32_t w[16];
-        if (j0 >= row_lo + 32) {
+        if (REV ? j0 + 32 <= row_lo : j0 >= row_lo + 32) {
 #pragma unroll
           for (int u = 0; u < 16; ++u) w[u] = 0u;
         } else if (rescaled) {
-          if (j0 + 31 <= row_lo) {
+          if ((REV ? j0 >= row_lo + 31 : j0 + 31 <= row_lo)) {
 #pragma unroll
             for (int u = 0; u < 32; u += 2) w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]), __uint_as_float(pr[u + 1]));
           } else {
 #pragma unroll
             for (int u = 0; u < 32; u += 2) {
               const int j = j0 + u;
-              w[u / 2] = pack_bf16x2((j <= r) ? __uint_as_float(pr[u]) : 0.f,
-                                     (j + 1 <= r) ? __uint_as_float(pr[u + 1]) : 0.f);
+              w[u / 2] = pack_bf16x2((REV ? (j >= r && j < C) : j <= r) ? __uint_as_float(pr[u]) : 0.f,
+                                     (REV ? (j + 1 >= r && j + 1 < C) : j + 1 <= r) ? __uint_as_float(pr[u + 1]) : 0.f);
             }
           }
-        } else if (j0 + 31 <= row_lo) {
+        } else if ((REV ? j0 >= row_lo + 31 : j0 + 31 <= row_lo)) {
           // whole 32x32 block below the diagonal: gamma^(r-j) = gamma^(r-j0-31) * gamma^(31-u)
-          const float ar = pw[r - j0 - 31];
+          const float ar = pw[REV ? j0 - r : r - j0 - 31];
 #pragma unroll
           for (int u = 0; u < 32; u += 2)
-            w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * ar * pw[31 - u],
-                                   __uint_as_float(pr[u + 1]) * ar * pw[30 - u]);
+            w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * ar * pw[REV ? u : 31 - u],
+                                   __uint_as_float(pr[u + 1]) * ar * pw[REV ? u + 1 : 30 - u]);
         } else {
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
             const int j = j0 + u;
-            const float f0 = (j <= r) ? pw[r - j] : 0.f;
-            const float f1 = (j + 1 <= r) ? pw[r - j - 1] : 0.f;
+            const float f0 = (REV ? (j >= r && j < C) : j <= r) ? pw[REV ? j - r : r - j] : 0.f;
+            const float f1 = (REV ? (j + 1 >= r && j + 1 < C) : j + 1 <= r) ? pw[REV ? j + 1 - r : r - j - 1] : 0.f;
             w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * f0, __uint_as_float(pr[u + 1]) * f1);
           }
         }
@@ -651,7 +660,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         // O *= xi_r = gamma^(r+1) once MMA4 wrote Q S_prev into O
         if (!mbar_wait(ocross, it & 1, abort_flag, a.lim)) break;
         tc_fence_after();
-        const float xi = pw[r + 1];
+        const float xi = pw[REV ? max(l - r, 0) : r + 1];
         for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(tm + lane_off + TM_O + c0, o);
@@ -670,8 +679,8 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 9);
       tc_fence_after();
       const int s = it % NS;
-      const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) * rho : 1.f;
-      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[min(C, a.L - t0 - C)]);
+      const float yf = rescaled ? exp2f((float)(REV ? -r : r + 1 - l) * l2g) * rho : 1.f;
+      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[blk_len(it + 1)]);
       if (NS >= 2) {
         // The V tile is dead after MMA3 and its buffer is not needed again for
         // NS-1 blocks: stage y there (bf16, 128B-swizzled) for two TMA tensor
@@ -712,7 +721,8 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           // the factor differs per row: scale before the transpose
 #pragma unroll
           for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(yf * __uint_as_float(o[u]));
-          store_rows_bf16_quad(wrow0 + c0, (size_t)a.dv, lane, o, 1.f, l - row_lo);
+          if (RET_BC(t0 + l <= a.L && vt * kCW_DVT + c0 + 32 <= a.dv, 102))
+            store_rows_bf16_quad(wrow0 + c0, (size_t)a.dv, lane, o, 1.f, l - row_lo);
         }
         tc_fence_before();
         mbar_arrive(ofree);
@@ -754,6 +764,7 @@ __host__ __device__ inline Cw256Smem cw256_smem_plan(int C) {
   return s;
 }
 
+template <bool REV>
 __global__ void __launch_bounds__(kCW_MainThreads, 1)
 chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                        const __grid_constant__ CUtensorMap mapV, const CwArgs a,
@@ -795,6 +806,12 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
   const int c_begin = seg * a.seg_chunks;
   const int c_end = min(c_begin + a.seg_chunks, n_total);
   const int nck = max(c_end - c_begin, 0);
+  // Step it of the walk takes block blk_idx(it): forward from the segment's
+  // first block, REV (the anti-causal sum) from its last block down.
+  auto blk_idx = [&](int it) { return REV ? c_end - 1 - it : c_begin + it; };
+  auto blk_t0 = [&](int it) { return blk_idx(it) * C; };
+  auto blk_len = [&](int it) { return min(C, a.L - blk_t0(it)); };
+  const int l_first = nck > 0 ? blk_len(0) : 0;
   const int cta_id = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
   (void)cta_id;
   RET_TRACE_INIT();
@@ -841,13 +858,13 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       int issued = 0;
       for (int it = 0; it < nck; ++it) {
         const uint32_t par = (it - 1) & 1;
-        const int t0 = (c_begin + it) * C;
+        const int t0 = blk_t0(it);
         if (it >= 1 && !mbar_wait(emptyQ, par, abort_flag, a.lim)) break;
         mbar_arrive_expect_tx(fullQ, qk_bytes);
         for (int b = 0; b < 4; ++b) tma_load_3d(sQ + b * 16384, &mapQ, fullQ, b * 64, t0, bh);
         if (it >= 1 && !mbar_wait(emptyK, par, abort_flag, a.lim)) break;
         RET_TRACE_STAMP(cta_id, it, 0);
-        if (c_begin + it != a.debug_drop_block) {  // fault injection: a load that never lands
+        if (blk_idx(it) != a.debug_drop_block) {  // fault injection: a load that never lands
           mbar_arrive_expect_tx(fullK, qk_bytes);
           for (int b = 0; b < 4; ++b) tma_load_3d(sKS + b * sp.ks_box, &mapK, fullK, b * 64, t0, bh);
         }
@@ -856,7 +873,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         for (int b = 0; b < 2; ++b) tma_load_3d(sV + b * C * 128, &mapV, fullV, vt * kCW_DVT + b * 64, t0, bh);
         issued = it + 1;
         if (it + 1 < nck) {  // next block's tiles into L2 while this one runs
-          const int tp = t0 + C;
+          const int tp = blk_t0(it + 1);
           for (int b = 0; b < 4; ++b) {
             tma_prefetch_l2_3d(&mapQ, b * 64, tp, bh);
             tma_prefetch_l2_3d(&mapK, b * 64, tp, bh);
@@ -935,7 +952,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
     const int v = vt * kCW_DVT + (int)v_loc;
     const size_t dkdv = (size_t)DK * a.dv;
     uint8_t* sSb = sKS + (uint32_t)C * 128u;  // first Sb row of box 0; box stride ks_box
-    const float g0 = pw[max(min(C, a.L - c_begin * C), 0)];
+    const float g0 = pw[l_first];
     float rho = cw_rho_first(rescaled, g0);
     {
       const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
@@ -950,7 +967,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         uint32_t w[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          const float sv = src ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
+          const float sv = (src && RET_BC(d0 + u < DK && v < a.dv, 104)) ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
           x[u] = gc * sv;
           w[u] = __float_as_uint(gu * sv);
         }
@@ -964,7 +981,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
     }
     for (int it = 0; it < nck; ++it) {
       const uint32_t par = it & 1;
-      const int t0 = (c_begin + it) * C;
+      const int t0 = blk_t0(it);
       {
         // zeta (rescaled: zeta / rho) on row v_loc of V (rescaled form, as soon
         // as V lands) or of K (direct form, once MMA14 has read it); the S group
@@ -977,7 +994,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         }
         const int l = min(C, a.L - t0);
         if ((int)v_loc < C) {
-          const float zeta = ((int)v_loc < l) ? pw[l - 1 - (int)v_loc] : 0.f;
+          const float zeta = ((int)v_loc < l) ? pw[REV ? (int)v_loc : l - 1 - (int)v_loc] : 0.f;
           if (rescaled) {
             scale_row_sw128(sV + half * C * 128, v_loc, zeta * __frcp_rn(rho));
           } else {
@@ -993,7 +1010,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       if (v_loc == 0 && !vgrp) RET_TRACE_STAMP(cta_id, it, 5);
       tc_fence_after();
       if (it < nck - 1) {
-        const float gn = pw[min(C, a.L - t0 - C)];
+        const float gn = pw[blk_len(it + 1)];
         // direct form: decay the state in TMEM, Sb = S.  Rescaled form: Sb = U,
         // and U is multiplied through only when rho is reset.
         const float rho_n = rescaled ? cw_rho_next(rho, gn) : 1.f;
@@ -1025,12 +1042,13 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         tc_fence_before();
         mbar_arrive(sready);
         if (v_loc == 0 && !vgrp) RET_TRACE_STAMP(cta_id, it, 8);
-      } else if (a.state_out && seg == a.n_seg - 1) {
+      } else if (a.state_out && seg == (REV ? 0 : a.n_seg - 1)) {
         float* so = a.state_out + (size_t)bh * dkdv;
         for (int d0 = d_lo; d0 < d_lo + 128; d0 += 32) {
           uint32_t sr[32];
           tmem_ld32(tm + lane_off + TM_S + d0, sr);
           tmem_ld_wait();
+          if (!RET_BC(d0 + 32 <= DK && v < a.dv, 103)) continue;
 #pragma unroll
           for (int u = 0; u < 32; ++u) so[(size_t)(d0 + u) * a.dv + v] = rho * __uint_as_float(sr[u]);
         }
@@ -1041,14 +1059,15 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
     const int r = (int)threadIdx.x;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int row_lo = warp * 32;
-    float rho = cw_rho_first(rescaled, pw[max(min(C, a.L - c_begin * C), 0)]);
+    float rho = cw_rho_first(rescaled, pw[l_first]);
     mbar_arrive(ofree);  // X starts free
     for (int it = 0; it < nck; ++it) {
       const uint32_t par = it & 1;
-      const int t0 = (c_begin + it) * C;
+      const int t0 = blk_t0(it);
       const int l = min(C, a.L - t0);
       if (!mbar_wait(pxfull, par, abort_flag, a.lim)) break;
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 10);
+      (void)RET_BC(l >= 1 && l <= C && t0 >= 0 && t0 < a.L, 207);
       tc_fence_after();
       // P -> P~ in place (see the main kernel for the two forms)
       const uint32_t tp = tm + lane_off + TM_P;
@@ -1057,33 +1076,33 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         tmem_ld32(tp + j0, pr);
         tmem_ld_wait();
         uint32_t w[16];
-        if (j0 >= row_lo + 32) {
+        if (REV ? j0 + 32 <= row_lo : j0 >= row_lo + 32) {
 #pragma unroll
           for (int u = 0; u < 16; ++u) w[u] = 0u;
         } else if (rescaled) {
-          if (j0 + 31 <= row_lo) {
+          if ((REV ? j0 >= row_lo + 31 : j0 + 31 <= row_lo)) {
 #pragma unroll
             for (int u = 0; u < 32; u += 2) w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]), __uint_as_float(pr[u + 1]));
           } else {
 #pragma unroll
             for (int u = 0; u < 32; u += 2) {
               const int j = j0 + u;
-              w[u / 2] = pack_bf16x2((j <= r) ? __uint_as_float(pr[u]) : 0.f,
-                                     (j + 1 <= r) ? __uint_as_float(pr[u + 1]) : 0.f);
+              w[u / 2] = pack_bf16x2((REV ? (j >= r && j < C) : j <= r) ? __uint_as_float(pr[u]) : 0.f,
+                                     (REV ? (j + 1 >= r && j + 1 < C) : j + 1 <= r) ? __uint_as_float(pr[u + 1]) : 0.f);
             }
           }
-        } else if (j0 + 31 <= row_lo) {
-          const float ar = pw[r - j0 - 31];
+        } else if ((REV ? j0 >= row_lo + 31 : j0 + 31 <= row_lo)) {
+          const float ar = pw[REV ? j0 - r : r - j0 - 31];
 #pragma unroll
           for (int u = 0; u < 32; u += 2)
-            w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * ar * pw[31 - u],
-                                   __uint_as_float(pr[u + 1]) * ar * pw[30 - u]);
+            w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * ar * pw[REV ? u : 31 - u],
+                                   __uint_as_float(pr[u + 1]) * ar * pw[REV ? u + 1 : 30 - u]);
         } else {
 #pragma unroll
           for (int u = 0; u < 32; u += 2) {
             const int j = j0 + u;
-            const float f0 = (j <= r) ? pw[r - j] : 0.f;
-            const float f1 = (j + 1 <= r) ? pw[r - j - 1] : 0.f;
+            const float f0 = (REV ? (j >= r && j < C) : j <= r) ? pw[REV ? j - r : r - j] : 0.f;
+            const float f1 = (REV ? (j + 1 >= r && j + 1 < C) : j + 1 <= r) ? pw[REV ? j + 1 - r : r - j - 1] : 0.f;
             w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * f0, __uint_as_float(pr[u + 1]) * f1);
           }
         }
@@ -1094,7 +1113,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       }
       if (!rescaled) {
         // X *= xi_r = gamma^(r+1): X holds Q S_prev from MMA14
-        const float xi = pw[r + 1];
+        const float xi = pw[REV ? max(l - r, 0) : r + 1];
         for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(tm + lane_off + TM_X + c0, o);
@@ -1115,7 +1134,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       {
         // X -> registers as bf16 pairs, release X to the next block's MMA14,
         // then the global stores.
-        const float yf = rescaled ? exp2f((float)(r + 1 - l) * l2g) * rho : 1.f;
+        const float yf = rescaled ? exp2f((float)(REV ? -r : r + 1 - l) * l2g) * rho : 1.f;
         __nv_bfloat16* wrow0 = a.y + ((size_t)bh * a.L + t0 + row_lo) * a.dv + vt * kCW_DVT;
         uint32_t yb[4][16];
 #pragma unroll
@@ -1129,11 +1148,13 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         }
         tc_fence_before();
         mbar_arrive(ofree);
+        if (RET_BC(t0 + l <= a.L && vt * kCW_DVT + 128 <= a.dv, 202)) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) store_rows_packed_quad(wrow0 + 32 * c, (size_t)a.dv, lane, yb[c], l - row_lo);
+          for (int c = 0; c < 4; ++c) store_rows_packed_quad(wrow0 + 32 * c, (size_t)a.dv, lane, yb[c], l - row_lo);
+        }
       }
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 7);
-      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[min(C, a.L - t0 - C)]);
+      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[blk_len(it + 1)]);
     }
   }
   tc_fence_before();
@@ -1152,7 +1173,10 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
 // the workspace [BH][n_seg][dk][dv].  Rows of K (DK <= 128) or of V (DK = 256)
 // are scaled by the decay to the segment end in shared memory, then
 // accumulated by tcgen05 into TMEM.
-template <int DK>
+// REV (the anti-causal sum): the sum of segment g = 1..n_seg-1 decays to the
+// segment's FIRST token s_g, D_g^T = sum_{t in g} gamma^(t - s_g) v_t^T k_t,
+// and goes to slot g-1.
+template <int DK, bool REV>
 __global__ void __launch_bounds__(kCW_Threads)
 chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                    const CwArgs a, const __grid_constant__ CwDecay dec, float* ws) {
@@ -1172,13 +1196,15 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13) + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int vt = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;  // seg < n_seg - 1
+  const int vt = blockIdx.x, bh = blockIdx.y;
+  const int seg = REV ? (int)blockIdx.z + 1 : (int)blockIdx.z;  // forward: seg < n_seg - 1; REV: seg >= 1
   const float l2g = dec.l2g[bh % a.H];
   const int n_total = (a.L + C - 1) / C;
   const int c_begin = seg * a.seg_chunks;
   const int c_end = min(c_begin + a.seg_chunks, n_total);
   const int nck = max(c_end - c_begin, 0);
   const int seg_last = min(c_end * C, a.L) - 1;  // e_g
+  const int seg_first = c_begin * C;              // s_g
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) {
@@ -1249,7 +1275,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
       if constexpr (DK <= kCW_DVT) {
         for (uint32_t j = r; j < (uint32_t)C; j += 128) {  // rows j and j + 128 (blocks up to 256)
           const int t = (c_begin + it) * C + (int)j;
-          const float f = (t <= seg_last) ? (t == seg_last ? 1.f : exp2f((float)(seg_last - t) * l2g)) : 0.f;
+          const int ex = REV ? t - seg_first : seg_last - t;
+          const float f = (t <= seg_last) ? (ex == 0 ? 1.f : exp2f((float)ex * l2g)) : 0.f;
           for (int b = 0; b < DK / 64; ++b) scale_row_sw128(sK + s * k_stage + b * C * 128, j, f);
         }
       } else {
@@ -1266,7 +1293,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
               w[u] = *reinterpret_cast<const uint4*>(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u +
                                                       (e & 7u) * 16u);
               const int t = (c_begin + it) * C + (int)j;
-              f[u] = (t <= seg_last) ? (t == seg_last ? 1.f : exp2f((float)(seg_last - t) * l2g)) : 0.f;
+              const int ex = REV ? t - seg_first : seg_last - t;
+              f[u] = (t <= seg_last) ? (ex == 0 ? 1.f : exp2f((float)ex * l2g)) : 0.f;
             }
           }
 #pragma unroll
@@ -1292,9 +1320,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
       tc_fence_after();
       const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
       const size_t dkdv = (size_t)DK * a.dv;
-      float* dst = ws + ((size_t)bh * a.n_seg + seg + 1) * dkdv;
+      const int slot = REV ? seg - 1 : seg + 1;
+      float* dst = ws + ((size_t)bh * a.n_seg + slot) * dkdv;
       const int v = vt * kCW_DVT + (int)r;
-      for (int d0 = 0; d0 < DK; d0 += 32) {
+      for (int d0 = 0; d0 < DK && RET_BC(slot >= 0 && slot < a.n_seg && v < a.dv, 401); d0 += 32) {
         uint32_t sr[32];
         tmem_ld32(tm + lane_off + d0, sr);
         tmem_ld_wait();
@@ -1320,8 +1349,12 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
 // g = 1..n_seg-1, slot g <- gamma^len * slot(g-1) + D_(g-1) (D_(g-1) was stored in
 // slot g by chunk_state_kernel).  len = tokens per segment (all but the last
 // segment are full).
+// REV: slot n_seg-1 <- S_in (the state after the sequence), and for
+// g = n_seg-2..0, slot g <- gamma^len(g+1) * slot(g+1) + D_(g+1) (stored in
+// slot g); the last segment has last_len tokens.
+template <bool REV>
 __global__ void state_scan_kernel(const float* __restrict__ state_in, float* __restrict__ ws,
-                                  int BH, int H, int dkdv, int n_seg, int seg_len,
+                                  int BH, int H, int dkdv, int n_seg, int seg_len, int last_len,
                                   const __grid_constant__ CwDecay dec) {
   const size_t total = (size_t)BH * dkdv;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
@@ -1331,10 +1364,19 @@ __global__ void state_scan_kernel(const float* __restrict__ state_in, float* __r
     const float gl = exp2f((float)seg_len * dec.l2g[bh % H]);
     float S = state_in ? state_in[e] : 0.f;
     float* slot = ws + (size_t)bh * n_seg * dkdv + off;
-    slot[0] = S;
-    for (int g = 1; g < n_seg; ++g) {
-      S = fmaf(gl, S, slot[(size_t)g * dkdv]);
-      slot[(size_t)g * dkdv] = S;
+    if (!REV) {
+      slot[0] = S;
+      for (int g = 1; g < n_seg; ++g) {
+        S = fmaf(gl, S, slot[(size_t)g * dkdv]);
+        slot[(size_t)g * dkdv] = S;
+      }
+    } else {
+      const float gl_last = exp2f((float)last_len * dec.l2g[bh % H]);
+      slot[(size_t)(n_seg - 1) * dkdv] = S;
+      for (int g = n_seg - 2; g >= 0; --g) {
+        S = fmaf(g + 1 == n_seg - 1 ? gl_last : gl, S, slot[(size_t)g * dkdv]);
+        slot[(size_t)g * dkdv] = S;
+      }
     }
   }
 }

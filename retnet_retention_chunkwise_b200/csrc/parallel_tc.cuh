@@ -22,6 +22,12 @@
 // n = 128 (qt - kt) + i - j splits as  i + (128 (qt - kt) - 127) + (127 - j), all
 // three parts >= 0, so  gamma^n = pw[i] * T * pw[127 - j]  with one exp2 per tile
 // (T) and a 128-entry table; the diagonal tile uses pw[i - j] and the mask.
+//
+// REV computes the anti-causal sum y_n = sum_{m>=n} gamma^(m-n) (q_n . k_m) v_m
+// (the form the backward pass needs for dk and dv, without reversing the
+// sequence in memory): key tiles kt >= qt, walked from the last down to the
+// diagonal, exponent 128 (kt - qt) + j - i = (127 - i) + (128 (kt - qt) - 127) + j,
+// so gamma^n = pw[127 - i] * T * pw[j], and the diagonal tile keeps j >= i.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -62,7 +68,7 @@ __host__ __device__ inline PaSmem pa_smem_plan(int DK, int DVT, int ns) {
   return s;
 }
 
-template <int DK, int DVT>
+template <int DK, int DVT, bool REV>
 __global__ void __launch_bounds__(kPA_Threads, 1)
 parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, const PaArgs a,
@@ -94,11 +100,14 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int vt = blockIdx.x, bh = blockIdx.z;
-  const int qt0 = a.n_qt - 1 - (int)blockIdx.y;  // heavy tile first
-  const int qt1 = (int)blockIdx.y;               // then the light one
-  const int ntile = (qt1 < qt0) ? 2 : 1;
-  const int nk0 = qt0 + 1;
-  const int nitems = nk0 + (ntile == 2 ? qt1 + 1 : 0);
+  // the pair (n-1-y, y): the heavy tile first (forward: the later tile, REV:
+  // the earlier one, which has the most key tiles)
+  const int qt0 = REV ? (int)blockIdx.y : a.n_qt - 1 - (int)blockIdx.y;
+  const int qt1 = REV ? a.n_qt - 1 - (int)blockIdx.y : (int)blockIdx.y;
+  const int ntile = (qt0 != qt1) ? 2 : 1;
+  auto nkeys = [&](int qt) { return REV ? a.n_qt - qt : qt + 1; };  // key tiles of query tile qt
+  const int nk0 = nkeys(qt0);
+  const int nitems = nk0 + (ntile == 2 ? nkeys(qt1) : 0);
   const float l2g = dec.l2g[bh % a.H];
   const int cta_id = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
   (void)cta_id;
@@ -129,11 +138,15 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
 
-  // item i -> (query tile index t in {0,1}, its tile qt, key tile kt)
+  // item i -> (query tile index t in {0,1}, its tile qt, key tile kt); the key
+  // tiles of a query tile end with the diagonal one (REV walks them downwards)
   auto item = [&](int i, int& t, int& qt, int& kt) {
-    if (i < nk0) { t = 0; qt = qt0; kt = i; }
-    else { t = 1; qt = qt1; kt = i - nk0; }
+    const int k = (i < nk0) ? i : i - nk0;
+    t = (i < nk0) ? 0 : 1;
+    qt = t ? qt1 : qt0;
+    kt = REV ? a.n_qt - 1 - k : k;
   };
+  auto first_key = [&](int kt) { return REV ? kt == a.n_qt - 1 : kt == 0; };
 
   if (warp == kPA_WarpProducer) {
     if (lane == 0) {
@@ -185,7 +198,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bd = sdesc_sw128(v_s + kk * 2048, 16384, 1024);
           mma_ts(tm + TM_O + t * 128, tm + TM_P + pb * 128 + (kk / 4) * 64 + (kk % 4) * 8, bd, id3,
-                 (kt > 0 || kk > 0) ? 1u : 0u);
+                 (!first_key(kt) || kk > 0) ? 1u : 0u);
         }
         mma_commit(&empty[s]);
         if (kt == qt) mma_commit(ofull);  // last key tile of this query tile
@@ -195,7 +208,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
         int t, qt, kt;
         item(i, t, qt, kt);
         const int s = i % NS, pb = i & 1;
-        if (kt == 0 && !mbar_wait(&qfull[t], 0, abort_flag, a.lim)) { ok = false; break; }
+        if (first_key(kt) && !mbar_wait(&qfull[t], 0, abort_flag, a.lim)) { ok = false; break; }
         if (!mbar_wait(&full[s], (i / NS) & 1, abort_flag, a.lim)) { ok = false; break; }
         RET_TRACE_STAMP(cta_id, i, 1);
         // P buffer pb was last read by MMA3(i-2), issued before this MMA1 by
@@ -235,7 +248,7 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
     const int row_lo = (warp & 3) * 32;
     const int cbase = (warp >> 2) * 64;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const float rowf = pw[r];
+    const float rowf = pw[REV ? 127 - r : r];
     bool ok = true;
     for (int i = 0; i < nitems; ++i) {
       int t, qt, kt;
@@ -246,31 +259,44 @@ parallel_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_consta
       tc_fence_after();
       const uint32_t tp = tm + lane_off + TM_P + pb * 128;
       const bool diag = (kt == qt);
-      const float rs = diag ? 0.f : rowf * exp2f((float)(128 * (qt - kt) - 127) * l2g);
+      const float rs = diag ? 0.f : rowf * exp2f((float)(128 * (REV ? kt - qt : qt - kt) - 127) * l2g);
       for (int j0 = cbase; j0 < cbase + 64; j0 += 32) {
-        uint32_t pr[32];
-        tmem_ld32(tp + j0, pr);
-        tmem_ld_wait();
         uint32_t w[16];
-        if (!diag) {
-          const float4* cf = reinterpret_cast<const float4*>(pw + 96 - j0);  // pw[127-j] for j = j0+31 .. j0
-#pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 f = cf[7 - q4];  // pw[127-j0-4q4-3 .. 127-j0-4q4]
-            w[2 * q4] = pack_bf16x2(__uint_as_float(pr[4 * q4]) * rs * f.w, __uint_as_float(pr[4 * q4 + 1]) * rs * f.z);
-            w[2 * q4 + 1] =
-                pack_bf16x2(__uint_as_float(pr[4 * q4 + 2]) * rs * f.y, __uint_as_float(pr[4 * q4 + 3]) * rs * f.x);
-          }
-        } else if (j0 >= row_lo + 32) {
+        // diagonal tile: the 32 columns lie wholly on the masked side of row r's warp
+        const bool masked = diag && (REV ? j0 + 32 <= row_lo : j0 >= row_lo + 32);
+        if (masked) {
 #pragma unroll
           for (int u = 0; u < 16; ++u) w[u] = 0u;
         } else {
+          uint32_t pr[32];
+          tmem_ld32(tp + j0, pr);
+          tmem_ld_wait();
+          if (!diag && !REV) {
+            const float4* cf = reinterpret_cast<const float4*>(pw + 96 - j0);  // pw[127-j] for j = j0+31 .. j0
 #pragma unroll
-          for (int u = 0; u < 32; u += 2) {
-            const int j = j0 + u;
-            const float f0 = (j <= r) ? pw[r - j] : 0.f;
-            const float f1 = (j + 1 <= r) ? pw[r - j - 1] : 0.f;
-            w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * f0, __uint_as_float(pr[u + 1]) * f1);
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const float4 f = cf[7 - q4];  // pw[127-j0-4q4-3 .. 127-j0-4q4]
+              w[2 * q4] = pack_bf16x2(__uint_as_float(pr[4 * q4]) * rs * f.w, __uint_as_float(pr[4 * q4 + 1]) * rs * f.z);
+              w[2 * q4 + 1] =
+                  pack_bf16x2(__uint_as_float(pr[4 * q4 + 2]) * rs * f.y, __uint_as_float(pr[4 * q4 + 3]) * rs * f.x);
+            }
+          } else if (!diag) {
+            const float4* cf = reinterpret_cast<const float4*>(pw + j0);  // pw[j] for j = j0 .. j0+31
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const float4 f = cf[q4];
+              w[2 * q4] = pack_bf16x2(__uint_as_float(pr[4 * q4]) * rs * f.x, __uint_as_float(pr[4 * q4 + 1]) * rs * f.y);
+              w[2 * q4 + 1] =
+                  pack_bf16x2(__uint_as_float(pr[4 * q4 + 2]) * rs * f.z, __uint_as_float(pr[4 * q4 + 3]) * rs * f.w);
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; u += 2) {
+              const int j = j0 + u;
+              const float f0 = REV ? ((j >= r) ? pw[j - r] : 0.f) : ((j <= r) ? pw[r - j] : 0.f);
+              const float f1 = REV ? ((j + 1 >= r) ? pw[j + 1 - r] : 0.f) : ((j + 1 <= r) ? pw[r - j - 1] : 0.f);
+              w[u / 2] = pack_bf16x2(__uint_as_float(pr[u]) * f0, __uint_as_float(pr[u + 1]) * f1);
+            }
           }
         }
         tmem_st16(tp + cbase + (j0 - cbase) / 2, w);

@@ -179,10 +179,13 @@ size_t seg_workspace_bytes(const ret_shape& s, int n_seg) {
   return (size_t)s.B * s.H * n_seg * (size_t)s.dk * s.dv * sizeof(float);
 }
 
-template <int DK>
+// REV = true runs the anti-causal sum (see chunkwise_dir); blocks longer than
+// 128 rows have no anti-causal kernel.
+template <int DK, bool REV>
 ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, const float* gamma,
                                void* y, const float* state_in, float* state_out, int C,
                                const ret_shape& s, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (REV && C > 128) return RET_EUNSUPPORTED;
   const int BH = s.B * s.H;
   CUtensorMap mq, mk, mv, my;
   if (!make_map(&mq, q, DK, s.L, BH, C) || !make_map(&mk, k, DK, s.L, BH, C) ||
@@ -244,16 +247,16 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
     a2.nstages = ns2;
     a2.debug_drop_block = -1;
     const int smem2 = (int)(ns2 * per + kMiscBytes + kSmemAlign);
-    if (cudaFuncSetAttribute(chunk_state_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) !=
+    if (cudaFuncSetAttribute(chunk_state_kernel<DK, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2) !=
         cudaSuccess)
       return RET_ECUDA;
     dim3 g2(s.dv / kCW_DVT, BH, n_seg - 1);
-    chunk_state_kernel<DK><<<g2, kCW_Threads, smem2, st>>>(mk, mv, a2, dec, static_cast<float*>(ws));
+    chunk_state_kernel<DK, REV><<<g2, kCW_Threads, smem2, st>>>(mk, mv, a2, dec, static_cast<float*>(ws));
     if (launch_status() != RET_OK) return RET_ECUDA;
     const long long total = (long long)BH * DK * s.dv;
     const int blocks = (int)std::min<long long>((total + 255) / 256, 4LL * sm_count());
-    state_scan_kernel<<<blocks, 256, 0, st>>>(state_in, static_cast<float*>(ws), BH, s.H, DK * s.dv,
-                                              n_seg, seg_chunks * C, dec);
+    state_scan_kernel<REV><<<blocks, 256, 0, st>>>(state_in, static_cast<float*>(ws), BH, s.H, DK * s.dv, n_seg,
+                                                   seg_chunks * C, s.L - (n_seg - 1) * seg_chunks * C, dec);
     if (launch_status() != RET_OK) return RET_ECUDA;
   }
   dim3 grid(s.dv / kCW_DVT, BH, n_seg);
@@ -262,10 +265,10 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
     const Cw256Smem p256 = cw256_smem_plan(C);
     if ((int)p256.total > smax) return RET_EUNSUPPORTED;
     a.nstages = 1;
-    if (cudaFuncSetAttribute(chunkwise_tc256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(chunkwise_tc256_kernel<REV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)p256.total) != cudaSuccess)
       return RET_ECUDA;
-    chunkwise_tc256_kernel<<<grid, kCW_MainThreads, p256.total, st>>>(mq, mk, mv, a, dec);
+    chunkwise_tc256_kernel<REV><<<grid, kCW_MainThreads, p256.total, st>>>(mq, mk, mv, a, dec);
     return launch_status();
   } else {
     if (C > 128) {
@@ -276,10 +279,10 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
       chunkwise_wide_kernel<DK><<<grid, kCW_MainThreads, pw.total, st>>>(mq, mk, mv, a, dec);
       return launch_status();
     }
-    if (cudaFuncSetAttribute(chunkwise_tc_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(chunkwise_tc_kernel<DK, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)plan.total) != cudaSuccess)
       return RET_ECUDA;
-    chunkwise_tc_kernel<DK><<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, my, a, dec);
+    chunkwise_tc_kernel<DK, REV><<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, my, a, dec);
     return launch_status();
   }
 }
@@ -358,10 +361,11 @@ ret_status launch_chunk_state(const void* k, const void* v, const float* gamma, 
   a.lim = wait_limit();
   a.debug_drop_block = -1;
   const int smem = (int)(ns * per + kMiscBytes + kSmemAlign);
-  if (cudaFuncSetAttribute(chunk_state_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(chunk_state_kernel<DK, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
     return RET_ECUDA;
   dim3 grid(s.dv / kCW_DVT, BH, n_seg);
-  chunk_state_kernel<DK><<<grid, kCW_Threads, smem, st>>>(mk, mv, a, dec, static_cast<float*>(ws));
+  chunk_state_kernel<DK, false><<<grid, kCW_Threads, smem, st>>>(mk, mv, a, dec, static_cast<float*>(ws));
   if (launch_status() != RET_OK) return RET_ECUDA;
   int lens[kFoldMaxParts];
   for (int g = 0; g < n_seg; ++g) lens[g] = std::min(s.L, (g + 1) * seg_chunks * C) - g * seg_chunks * C;
@@ -370,7 +374,7 @@ ret_status launch_chunk_state(const void* k, const void* v, const float* gamma, 
                            (long long)(n_seg + 1) * dkdv, st);
 }
 
-template <int DK, int DVT>
+template <int DK, int DVT, bool REV>
 ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const float* gamma, void* y,
                               const ret_shape& s, cudaStream_t st) {
   const int BH = s.B * s.H;
@@ -397,12 +401,12 @@ ret_status launch_parallel_tc(const void* q, const void* k, const void* v, const
   a.nstages = ns;
   a.y = static_cast<__nv_bfloat16*>(y);
   a.lim = wait_limit();
-  if (cudaFuncSetAttribute(parallel_tc_kernel<DK, DVT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(parallel_tc_kernel<DK, DVT, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)plan.total) != cudaSuccess)
     return RET_ECUDA;
   // blockIdx.y = y pairs query tiles n_qt-1-y and y (one tile when they meet)
   dim3 grid(s.dv / DVT, (a.n_qt + 1) / 2, BH);
-  parallel_tc_kernel<DK, DVT><<<grid, kPA_Threads, plan.total, st>>>(mq, mk, mv, a, dec);
+  parallel_tc_kernel<DK, DVT, REV><<<grid, kPA_Threads, plan.total, st>>>(mq, mk, mv, a, dec);
   return launch_status();
 }
 
@@ -441,41 +445,102 @@ ret_status launch_groupnorm(const void* y, void* out, float eps, const float* w,
   return launch_status();
 }
 
-// Reverse the sequence axis of a [BH][L][d] tensor (d * es bytes per row).
-ret_status launch_reverse(const void* in, void* out, long long BH, int L, int d, size_t es, cudaStream_t st) {
-  const size_t row = (size_t)d * es;
-  const long long rows = BH * L;
-  if (rows == 0) return RET_OK;
-  auto grid = [&](long long units) {
-    return (unsigned)std::min<long long>((units + 255) / 256, 8LL * sm_count());
-  };
-  if (row % 16 == 0) {
-    const int u = (int)(row / 16);
-    reverse_rows_kernel<uint4><<<grid(rows * u), 256, 0, st>>>(static_cast<const uint4*>(in), static_cast<uint4*>(out),
-                                                               BH, L, u);
-  } else if (row % 4 == 0) {
-    const int u = (int)(row / 4);
-    reverse_rows_kernel<uint32_t><<<grid(rows * u), 256, 0, st>>>(static_cast<const uint32_t*>(in),
-                                                                  static_cast<uint32_t*>(out), BH, L, u);
-  } else {
-    const int u = (int)(row / 2);
-    reverse_rows_kernel<uint16_t><<<grid(rows * u), 256, 0, st>>>(static_cast<const uint16_t*>(in),
-                                                                  static_cast<uint16_t*>(out), BH, L, u);
+// Parallel form in either time direction: REV = false is retention_parallel,
+// REV = true the anti-causal sum y_n = sum_{m>=n} gamma^(m-n) (q_n . k_m) v_m
+// that the backward pass takes for dk and dv.
+template <bool REV>
+ret_status parallel_dir(const void* q, const void* k, const void* v, const float* gamma, void* y, ret_shape s,
+                        ret_dtype dt, cudaStream_t st) {
+  ret_status rc = check_shape(s, true);
+  if (rc != RET_OK) return rc;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (s.L == 0) return RET_OK;
+  if (!q || !k || !v || !y) return RET_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y)) return RET_EINVAL;
+  if (dt == RET_F32) {
+    if (s.dk > 256) return RET_EUNSUPPORTED;
+    static HeadLog2 hl;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int h = 0; h < s.H; ++h) hl.l2g[h] = log2_gamma(gamma[h]);
+    const int smem = (2 * kPF_Rows * (s.dk + 1) + kPF_Rows * kPF_Cols + kPF_Rows * 33) * 4;
+    if (cudaFuncSetAttribute(parallel_f32_kernel<REV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return RET_ECUDA;
+    dim3 grid((s.dv + kPF_Cols - 1) / kPF_Cols, (s.L + kPF_Rows - 1) / kPF_Rows, s.B * s.H);
+    parallel_f32_kernel<REV><<<grid, 256, smem, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
+                                                      static_cast<const float*>(v), static_cast<float*>(y), s.H,
+                                                      s.L, s.dk, s.dv, hl);
+    return launch_status();
   }
-  return launch_status();
+  if (dt != RET_BF16) return RET_EINVAL;
+  if (!parallel_tc_shape_ok(s) || !device_is_sm100()) return RET_EUNSUPPORTED;
+  const bool wide = s.dv % 128 == 0;  // 128-column dv slices, else 64
+  switch (s.dk) {
+    case 64: return wide ? launch_parallel_tc<64, 128, REV>(q, k, v, gamma, y, s, st)
+                         : launch_parallel_tc<64, 64, REV>(q, k, v, gamma, y, s, st);
+    case 128: return wide ? launch_parallel_tc<128, 128, REV>(q, k, v, gamma, y, s, st)
+                          : launch_parallel_tc<128, 64, REV>(q, k, v, gamma, y, s, st);
+    default: return wide ? launch_parallel_tc<256, 128, REV>(q, k, v, gamma, y, s, st)
+                         : launch_parallel_tc<256, 64, REV>(q, k, v, gamma, y, s, st);
+  }
 }
 
-// Workspace of the parallel backward pass: reversed q, k, v, dy and the two
-// reversed results, each region 256-byte aligned.
-size_t parallel_backward_ws(const ret_shape& s, size_t es, size_t* off) {
-  const size_t nk = (size_t)s.B * s.H * s.L * s.dk * es, nv = (size_t)s.B * s.H * s.L * s.dv * es;
-  const size_t sz[6] = {nk, nk, nv, nv, nk, nv};  // Rq, Rk, Rv, Rdy, T (-> dk), T2 (-> dv)
-  size_t o = 0;
-  for (int i = 0; i < 6; ++i) {
-    if (off) off[i] = o;
-    o += (sz[i] + 255) & ~size_t(255);
+// Chunkwise form in either time direction.  REV = false is retention_chunkwise.
+// REV = true is the anti-causal sum, which the backward pass takes for dk and
+// dv without reversing the sequence in memory:
+//     y_n = sum_{m>=n} gamma^(m-n) (q_n . k_m) v_m + gamma^(L-n) q_n S_in,
+// walked from the last block to the first, with state_in the state after the
+// sequence and state_out = gamma^L S_in + sum_m gamma^m k_m^T v_m the state at
+// its start (bf16: blocks of at most 128 rows).
+template <bool REV>
+ret_status chunkwise_dir(const void* q, const void* k, const void* v, const float* gamma, void* y,
+                         const float* state_in, float* state_out, int chunk, ret_shape s, ret_dtype dt,
+                         void* workspace, size_t workspace_bytes, cudaStream_t st) {
+  ret_status rc = check_shape(s, true);
+  if (rc != RET_OK) return rc;
+  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
+  if (chunk < 1) return RET_EINVAL;
+  if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
+  if (s.L > 0 && (!q || !k || !v || !y)) return RET_EINVAL;
+  if (s.L > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y))) return RET_EINVAL;
+  if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out))) return RET_EINVAL;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RET_EINVAL;
+  if (dt == RET_F32) {
+    if (chunk > kCF_MaxC || s.dk > 256) return RET_EUNSUPPORTED;
+  } else {
+    if (!tc_chunk_ok(chunk, s.dk)) return RET_EUNSUPPORTED;
+    if (!tc_shape_ok(s)) return RET_EUNSUPPORTED;
+    if (s.L > 0 && !device_is_sm100()) return RET_EUNSUPPORTED;
   }
-  return o;
+  const size_t sbytes = (size_t)s.B * s.H * s.dk * s.dv * sizeof(float);
+  if (s.L == 0) {  // nothing to compute: the state passes through
+    if (!state_out) return RET_OK;
+    cudaError_t e = state_in ? (state_in == state_out ? cudaSuccess
+                                                      : cudaMemcpyAsync(state_out, state_in, sbytes,
+                                                                        cudaMemcpyDeviceToDevice, st))
+                             : cudaMemsetAsync(state_out, 0, sbytes, st);
+    return e == cudaSuccess ? RET_OK : RET_ECUDA;
+  }
+  if (dt == RET_F32) {
+    static HeadLog2 hl;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int h = 0; h < s.H; ++h) hl.l2g[h] = log2_gamma(gamma[h]);
+    const int smem = (s.dk * kCF_Cols + chunk * (chunk + 1) + chunk + 1) * 4;
+    if (cudaFuncSetAttribute(chunkwise_f32_kernel<REV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return RET_ECUDA;
+    dim3 grid((s.dv + kCF_Cols - 1) / kCF_Cols, s.B * s.H);
+    chunkwise_f32_kernel<REV><<<grid, 256, smem, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
+                                                  static_cast<const float*>(v), static_cast<float*>(y), state_in,
+                                                  state_out, s.H, s.L, s.dk, s.dv, chunk, hl);
+    return launch_status();
+  }
+  switch (s.dk) {
+    case 64: return launch_chunkwise_tc<64, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+    case 128: return launch_chunkwise_tc<128, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+    default: return launch_chunkwise_tc<256, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -579,7 +644,7 @@ RET_API int retention_debug_trace(void* buf, int blocks, int events) {
 }
 #endif
 
-int retention_abi_version(void) { return 103; }
+int retention_abi_version(void) { return 104; }
 
 const char* retention_status_str(ret_status st) {
   switch (st) {
@@ -588,6 +653,7 @@ const char* retention_status_str(ret_status st) {
     case RET_EUNSUPPORTED: return "RET_EUNSUPPORTED";
     case RET_ECUDA: return "RET_ECUDA";
     case RET_ETIMEOUT: return "RET_ETIMEOUT";
+    case RET_EBOUNDS: return "RET_EBOUNDS";
   }
   return "RET_UNKNOWN";
 }
@@ -600,10 +666,21 @@ ret_status retention_get_device_status(void* stream) {
   if (h != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return RET_ECUDA;
-    return RET_ETIMEOUT;
+    return h == 5 ? RET_EBOUNDS : RET_ETIMEOUT;
   }
   return RET_OK;
 }
+
+#ifdef RET_BOUNDS_CHECK
+// Bounds-checked builds only: the site number of the first failed index check
+// since the last call (0: none), cleared by the call.
+RET_API unsigned int retention_debug_bounds_site(void) {
+  unsigned int site = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&site, g_bc_site, sizeof(site)) != cudaSuccess) return ~0u;
+  cudaMemcpyToSymbol(g_bc_site, &zero, sizeof(zero));
+  return site;
+}
+#endif
 
 ret_status retention_recurrent_step(const void* q, const void* k, const void* v, const float* gamma,
                                     void* y, float* state, ret_shape s, ret_dtype dt, void* stream) {
@@ -643,39 +720,7 @@ ret_status retention_recurrent_step(const void* q, const void* k, const void* v,
 ret_status retention_parallel(const void* q, const void* k, const void* v, const float* gamma, void* y,
                               ret_shape s, ret_dtype dt, void* stream) {
   NvtxRange nvtx_range("retention_parallel");
-  ret_status rc = check_shape(s, true);
-  if (rc != RET_OK) return rc;
-  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
-  if (s.L == 0) return RET_OK;
-  if (!q || !k || !v || !y) return RET_EINVAL;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y)) return RET_EINVAL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dt == RET_F32) {
-    if (s.dk > 256) return RET_EUNSUPPORTED;
-    static HeadLog2 hl;
-    static std::mutex mu;
-    std::lock_guard<std::mutex> lock(mu);
-    for (int h = 0; h < s.H; ++h) hl.l2g[h] = log2_gamma(gamma[h]);
-    const int smem = (2 * kPF_Rows * (s.dk + 1) + kPF_Rows * kPF_Cols + kPF_Rows * 33) * 4;
-    if (cudaFuncSetAttribute(parallel_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return RET_ECUDA;
-    dim3 grid((s.dv + kPF_Cols - 1) / kPF_Cols, (s.L + kPF_Rows - 1) / kPF_Rows, s.B * s.H);
-    parallel_f32_kernel<<<grid, 256, smem, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
-                                                 static_cast<const float*>(v), static_cast<float*>(y), s.H, s.L,
-                                                 s.dk, s.dv, hl);
-    return launch_status();
-  }
-  if (dt != RET_BF16) return RET_EINVAL;
-  if (!parallel_tc_shape_ok(s) || !device_is_sm100()) return RET_EUNSUPPORTED;
-  const bool wide = s.dv % 128 == 0;  // 128-column dv slices, else 64
-  switch (s.dk) {
-    case 64: return wide ? launch_parallel_tc<64, 128>(q, k, v, gamma, y, s, st)
-                         : launch_parallel_tc<64, 64>(q, k, v, gamma, y, s, st);
-    case 128: return wide ? launch_parallel_tc<128, 128>(q, k, v, gamma, y, s, st)
-                          : launch_parallel_tc<128, 64>(q, k, v, gamma, y, s, st);
-    default: return wide ? launch_parallel_tc<256, 128>(q, k, v, gamma, y, s, st)
-                         : launch_parallel_tc<256, 64>(q, k, v, gamma, y, s, st);
-  }
+  return parallel_dir<false>(q, k, v, gamma, y, s, dt, static_cast<cudaStream_t>(stream));
 }
 
 size_t retention_chunkwise_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
@@ -690,51 +735,8 @@ ret_status retention_chunkwise(const void* q, const void* k, const void* v, cons
                                const float* state_in, float* state_out, int chunk, ret_shape s,
                                ret_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
   NvtxRange nvtx_range("retention_chunkwise");
-  ret_status rc = check_shape(s, true);
-  if (rc != RET_OK) return rc;
-  if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
-  if (chunk < 1) return RET_EINVAL;
-  if (dt != RET_F32 && dt != RET_BF16) return RET_EINVAL;
-  if (s.L > 0 && (!q || !k || !v || !y)) return RET_EINVAL;
-  if (s.L > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y))) return RET_EINVAL;
-  if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out))) return RET_EINVAL;
-  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RET_EINVAL;
-  if (dt == RET_F32) {
-    if (chunk > kCF_MaxC || s.dk > 256) return RET_EUNSUPPORTED;
-  } else {
-    if (!tc_chunk_ok(chunk, s.dk)) return RET_EUNSUPPORTED;
-    if (!tc_shape_ok(s)) return RET_EUNSUPPORTED;
-    if (s.L > 0 && !device_is_sm100()) return RET_EUNSUPPORTED;
-  }
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t sbytes = (size_t)s.B * s.H * s.dk * s.dv * sizeof(float);
-  if (s.L == 0) {  // nothing to compute: the state passes through
-    if (!state_out) return RET_OK;
-    cudaError_t e = state_in ? (state_in == state_out ? cudaSuccess
-                                                      : cudaMemcpyAsync(state_out, state_in, sbytes,
-                                                                        cudaMemcpyDeviceToDevice, st))
-                             : cudaMemsetAsync(state_out, 0, sbytes, st);
-    return e == cudaSuccess ? RET_OK : RET_ECUDA;
-  }
-  if (dt == RET_F32) {
-    static HeadLog2 hl;
-    static std::mutex mu;
-    std::lock_guard<std::mutex> lock(mu);
-    for (int h = 0; h < s.H; ++h) hl.l2g[h] = log2_gamma(gamma[h]);
-    const int smem = (s.dk * kCF_Cols + chunk * (chunk + 1) + chunk + 1) * 4;
-    if (cudaFuncSetAttribute(chunkwise_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return RET_ECUDA;
-    dim3 grid((s.dv + kCF_Cols - 1) / kCF_Cols, s.B * s.H);
-    chunkwise_f32_kernel<<<grid, 256, smem, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
-                                                  static_cast<const float*>(v), static_cast<float*>(y), state_in,
-                                                  state_out, s.H, s.L, s.dk, s.dv, chunk, hl);
-    return launch_status();
-  }
-  switch (s.dk) {
-    case 64: return launch_chunkwise_tc<64>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
-    case 128: return launch_chunkwise_tc<128>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
-    default: return launch_chunkwise_tc<256>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
-  }
+  return chunkwise_dir<false>(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, workspace, workspace_bytes,
+                              static_cast<cudaStream_t>(stream));
 }
 
 size_t retention_chunkwise_state_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
@@ -780,10 +782,10 @@ ret_status retention_chunkwise_state(const void* k, const void* v, const float* 
     std::lock_guard<std::mutex> lock(mu);
     for (int h = 0; h < s.H; ++h) hl.l2g[h] = log2_gamma(gamma[h]);
     const int smem = (s.dk * kCF_Cols + chunk * (chunk + 1) + chunk + 1) * 4;
-    if (cudaFuncSetAttribute(chunkwise_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(chunkwise_f32_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return RET_ECUDA;
     dim3 grid((s.dv + kCF_Cols - 1) / kCF_Cols, s.B * s.H);
-    chunkwise_f32_kernel<<<grid, 256, smem, st>>>(static_cast<const float*>(k), static_cast<const float*>(k),
+    chunkwise_f32_kernel<false><<<grid, 256, smem, st>>>(static_cast<const float*>(k), static_cast<const float*>(k),
                                                   static_cast<const float*>(v), nullptr, state_in, state_out, s.H,
                                                   s.L, s.dk, s.dv, chunk, hl);
     return launch_status();
@@ -995,14 +997,17 @@ ret_status retention_chunkwise_gn_gated(const void* q, const void* k, const void
 }
 
 size_t retention_parallel_backward_workspace_bytes(ret_shape s, ret_dtype dt) {
-  if (check_shape(s, true) != RET_OK || (dt != RET_F32 && dt != RET_BF16)) return 0;
-  return parallel_backward_ws(s, dt == RET_BF16 ? 2 : 4, nullptr);
+  (void)s;
+  (void)dt;
+  return 0;  // the anti-causal sums read the inputs in place: no scratch
 }
 
 ret_status retention_parallel_backward(const void* q, const void* k, const void* v, const float* gamma,
                                        const void* dy, void* dq, void* dk, void* dv, ret_shape s, ret_dtype dt,
                                        void* workspace, size_t workspace_bytes, void* stream) {
   NvtxRange nvtx_range("retention_parallel_backward");
+  (void)workspace;
+  (void)workspace_bytes;
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
@@ -1012,59 +1017,54 @@ ret_status retention_parallel_backward(const void* q, const void* k, const void*
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) || !aligned16(dk) ||
       !aligned16(dv))
     return RET_EINVAL;
-  // the three forward calls take (dy, v, k), (Rv, Rdy, Rq) and (Rk, Rq, Rdy):
-  // both dk and dv play the role of the key width
+  // the three sums take (dy, v, k), (v, dy, q) and (k, q, dy): both dk and dv
+  // play the role of the key width
   if (dt == RET_BF16) {
     const ret_shape a{s.B, s.H, s.L, s.dv, s.dk}, b{s.B, s.H, s.L, s.dk, s.dv};
     if (!parallel_tc_shape_ok(a) || !parallel_tc_shape_ok(b) || !device_is_sm100()) return RET_EUNSUPPORTED;
   } else if (s.dk > 256 || s.dv > 256) {
     return RET_EUNSUPPORTED;
   }
-  const size_t es = dt == RET_BF16 ? 2 : 4;
-  size_t off[6];
-  const size_t need = parallel_backward_ws(s, es, off);
-  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return RET_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  char* w = static_cast<char*>(workspace);
-  void *rq = w + off[0], *rk = w + off[1], *rv = w + off[2], *rdy = w + off[3], *t1 = w + off[4], *t2 = w + off[5];
-  const long long BH = (long long)s.B * s.H;
   const ret_shape swapped{s.B, s.H, s.L, s.dv, s.dk};  // key width dv, value width dk
-  // dq = retention(dy, v, k)
-  if ((rc = retention_parallel(dy, v, k, gamma, dq, swapped, dt, stream)) != RET_OK) return rc;
-  if ((rc = launch_reverse(q, rq, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
-  if ((rc = launch_reverse(k, rk, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
-  if ((rc = launch_reverse(v, rv, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
-  if ((rc = launch_reverse(dy, rdy, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
-  // dk = R(retention(Rv, Rdy, Rq)),  dv = R(retention(Rk, Rq, Rdy))
-  if ((rc = retention_parallel(rv, rdy, rq, gamma, t1, swapped, dt, stream)) != RET_OK) return rc;
-  if ((rc = launch_reverse(t1, dk, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
-  if ((rc = retention_parallel(rk, rq, rdy, gamma, t2, s, dt, stream)) != RET_OK) return rc;
-  return launch_reverse(t2, dv, BH, s.L, s.dv, es, st);
+  // dq_n = sum_{m<=n} gamma^(n-m) (dy_n . v_m) k_m        (causal)
+  if ((rc = parallel_dir<false>(dy, v, k, gamma, dq, swapped, dt, st)) != RET_OK) return rc;
+  // dk_m = sum_{n>=m} gamma^(n-m) (v_m . dy_n) q_n        (anti-causal)
+  if ((rc = parallel_dir<true>(v, dy, q, gamma, dk, swapped, dt, st)) != RET_OK) return rc;
+  // dv_m = sum_{n>=m} gamma^(n-m) (k_m . q_n) dy_n        (anti-causal)
+  return parallel_dir<true>(k, q, dy, gamma, dv, s, dt, st);
 }
 
-// Chunkwise variant: the same three retention sums through the chunkwise form
-// (zero initial state), after the reversal buffers the workspace holds the
-// scratch of the largest of the three chunkwise calls.
+// Chunkwise variant: the same three retention sums through the chunkwise form,
+// dq causal and dk, dv anti-causal (chunkwise_dir<true>), so nothing is
+// reversed in memory; the workspace holds the sequence-split scratch of the
+// largest of the three calls and, with a carried state, three fp32 states.
 // One fp32 [B][H][dk][dv] state, rounded up to 256 bytes.
 size_t state_region_bytes(const ret_shape& s) {
   return ((size_t)s.B * s.H * s.dk * s.dv * sizeof(float) + 255) & ~size_t(255);
 }
 
+// Block length of the two anti-causal sums: the anti-causal kernels take
+// blocks of at most 128 rows (the result does not depend on it beyond
+// rounding).
+int rev_chunk(int chunk) { return std::min(chunk, 128); }
+
 size_t chunkwise_backward_split_ws(int chunk, const ret_shape& s, ret_dtype dt) {
   const ret_shape swapped{s.B, s.H, s.L, s.dv, s.dk};
-  return std::max(retention_chunkwise_workspace_bytes(chunk, swapped, dt),
-                  retention_chunkwise_workspace_bytes(chunk, s, dt));
+  const int cr = rev_chunk(chunk);
+  return std::max({retention_chunkwise_workspace_bytes(chunk, swapped, dt),
+                   retention_chunkwise_workspace_bytes(cr, swapped, dt),
+                   retention_chunkwise_workspace_bytes(cr, s, dt)});
 }
 
 size_t retention_chunkwise_backward_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
   if (check_shape(s, true) != RET_OK || (dt != RET_F32 && dt != RET_BF16)) return 0;
-  return parallel_backward_ws(s, dt == RET_BF16 ? 2 : 4, nullptr) + chunkwise_backward_split_ws(chunk, s, dt);
+  return chunkwise_backward_split_ws(chunk, s, dt);
 }
 
 size_t retention_chunkwise_backward_state_workspace_bytes(int chunk, ret_shape s, ret_dtype dt) {
-  const size_t base = retention_chunkwise_backward_workspace_bytes(chunk, s, dt);
-  if (!base) return 0;
-  return base + 3 * state_region_bytes(s);
+  if (check_shape(s, true) != RET_OK || (dt != RET_F32 && dt != RET_BF16)) return 0;
+  return chunkwise_backward_split_ws(chunk, s, dt) + 3 * state_region_bytes(s);
 }
 
 ret_status retention_chunkwise_backward(const void* q, const void* k, const void* v, const float* gamma,
@@ -1111,21 +1111,18 @@ ret_status retention_chunkwise_backward_state(const void* q, const void* k, cons
   } else if (s.dk > 256 || s.dv > 256 || chunk > kCF_MaxC) {
     return RET_EUNSUPPORTED;
   }
-  const size_t es = dt == RET_BF16 ? 2 : 4;
-  size_t off[6];
-  const size_t rev = parallel_backward_ws(s, es, off);
   const size_t split = chunkwise_backward_split_ws(chunk, s, dt);
   const size_t sreg = carried ? state_region_bytes(s) : 0;
-  if (!workspace || workspace_bytes < rev + split + 3 * sreg || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  if (split + 3 * sreg > 0 &&
+      (!workspace || workspace_bytes < split + 3 * sreg || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
     return RET_EINVAL;
   char* w = static_cast<char*>(workspace);
-  void *rq = w + off[0], *rk = w + off[1], *rv = w + off[2], *rdy = w + off[3], *t1 = w + off[4], *t2 = w + off[5];
-  void* sw = split ? w + rev : nullptr;
+  void* sw = split ? w : nullptr;
   // initial states of the three sums: S0^T, (dS_out / gamma)^T, dS_out / gamma;
   // the x2 region later takes the dv sum's state_out
-  float* s0t = carried ? reinterpret_cast<float*>(w + rev + split) : nullptr;
-  float* x2 = carried ? reinterpret_cast<float*>(w + rev + split + sreg) : nullptr;
-  float* x3 = carried ? reinterpret_cast<float*>(w + rev + split + 2 * sreg) : nullptr;
+  float* s0t = carried ? reinterpret_cast<float*>(w + split) : nullptr;
+  float* x2 = carried ? reinterpret_cast<float*>(w + split + sreg) : nullptr;
+  float* x3 = carried ? reinterpret_cast<float*>(w + split + 2 * sreg) : nullptr;
   const long long BH = (long long)s.B * s.H;
   HeadGamma hg, gl;
   bool any_small = false;
@@ -1141,23 +1138,20 @@ ret_status retention_chunkwise_backward_state(const void* q, const void* k, cons
     bwd_state_prep_kernel<<<grid, dim3(32, 8), 0, st>>>(state_in, dstate_out, s0t, x2, x3, s.H, s.dk, s.dv, hg);
     if ((rc = launch_status()) != RET_OK) return rc;
   }
-  // dq = retention(dy, v, k; S0^T)
-  if ((rc = retention_chunkwise(dy, v, k, gamma, dq, state_in ? s0t : nullptr, nullptr, chunk, swapped, dt, sw,
-                                split, stream)) != RET_OK)
+  const int cr = rev_chunk(chunk);
+  // dq_n = sum_{m<=n} gamma^(n-m) (dy_n . v_m) k_m + gamma^(n+1) dy_n S0^T:  causal, state_in S0^T
+  if ((rc = chunkwise_dir<false>(dy, v, k, gamma, dq, state_in ? s0t : nullptr, nullptr, chunk, swapped, dt, sw,
+                                 split, st)) != RET_OK)
     return rc;
-  if ((rc = launch_reverse(q, rq, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
-  if ((rc = launch_reverse(k, rk, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
-  if ((rc = launch_reverse(v, rv, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
-  if ((rc = launch_reverse(dy, rdy, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
-  // dk = R(retention(Rv, Rdy, Rq; x2)),  dv = R(retention(Rk, Rq, Rdy; x3)) with state_out T -> x2
-  if ((rc = retention_chunkwise(rv, rdy, rq, gamma, t1, dstate_out ? x2 : nullptr, nullptr, chunk, swapped, dt, sw,
-                                split, stream)) != RET_OK)
+  // dk_m = sum_{n>=m} gamma^(n-m) (v_m . dy_n) q_n + gamma^(L-1-m) v_m dS_out^T:  anti-causal, state_in x2
+  if ((rc = chunkwise_dir<true>(v, dy, q, gamma, dk, dstate_out ? x2 : nullptr, nullptr, cr, swapped, dt, sw, split,
+                                st)) != RET_OK)
     return rc;
-  if ((rc = launch_reverse(t1, dk, BH, s.L, s.dk, es, st)) != RET_OK) return rc;
-  if ((rc = retention_chunkwise(rk, rq, rdy, gamma, t2, dstate_out ? x3 : nullptr, dstate_in ? x2 : nullptr, chunk,
-                                s, dt, sw, split, stream)) != RET_OK)
+  // dv_m = sum_{n>=m} gamma^(n-m) (k_m . q_n) dy_n + gamma^(L-1-m) k_m dS_out:  anti-causal, state_in x3;
+  // its state_out T = sum_n gamma^n q_n^T dy_n + gamma^(L-1) dS_out goes to x2 (dS0 = gamma T)
+  if ((rc = chunkwise_dir<true>(k, q, dy, gamma, dv, dstate_out ? x3 : nullptr, dstate_in ? x2 : nullptr, cr, s, dt,
+                                sw, split, st)) != RET_OK)
     return rc;
-  if ((rc = launch_reverse(t2, dv, BH, s.L, s.dv, es, st)) != RET_OK) return rc;
   if (dstate_out && any_small) {
     if (dt == RET_BF16)
       bwd_last_token_kernel<__nv_bfloat16><<<(unsigned)BH, 256, 0, st>>>(

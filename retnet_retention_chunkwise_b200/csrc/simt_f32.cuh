@@ -26,9 +26,12 @@ __device__ __forceinline__ float decay_pow(float log2g, int n) {
 // Microsoft ...", section "Il meccanismo", parallel form).
 // CTA = (64-column block of y, 32 query rows, (b,h)).  Thread (r, cg):
 // r = tid / 8 owns query row r, cg = tid % 8 owns columns cg, cg+8, ..., cg+56.
+// REV: the anti-causal sum y_n = sum_{m>=n} gamma^(m-n) (q_n . k_m) v_m (key
+// tiles from the query tile to the end).
 constexpr int kPF_Rows = 32;
 constexpr int kPF_Cols = 64;
 
+template <bool REV>
 __global__ void __launch_bounds__(256)
 parallel_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                     const float* __restrict__ v, float* __restrict__ y, int H, int L, int dk,
@@ -56,7 +59,7 @@ parallel_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
 #pragma unroll
   for (int u = 0; u < 8; ++u) acc[u] = 0.f;
 
-  for (int k0 = 0; k0 <= q0 && k0 < L; k0 += kPF_Rows) {
+  for (int k0 = REV ? q0 : 0; REV ? k0 < L : (k0 <= q0 && k0 < L); k0 += kPF_Rows) {
     __syncthreads();
     for (int e = tid; e < kPF_Rows * dk; e += 256) {
       const int j = e / dk, d = e % dk;
@@ -73,7 +76,7 @@ parallel_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
       const int j = cg * 4 + u;
       float s = 0.f;
       for (int d = 0; d < dk; ++d) s = fmaf(Qs[r * ldq + d], Ks[j * ldq + d], s);
-      const int n = (q0 + r) - (k0 + j);
+      const int n = REV ? (k0 + j) - (q0 + r) : (q0 + r) - (k0 + j);
       Ps[r * 33 + j] = (n >= 0 && k0 + j < L) ? s * decay_pow(l2g, n) : 0.f;
     }
     __syncthreads();
@@ -100,9 +103,17 @@ parallel_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
 // CTA = (32-column block of the state / y, (b,h)); the state block [dk][32]
 // stays in shared memory for the whole sequence.  With y null only the state is
 // carried (q is not read).
+// REV: the anti-causal sum y_n = sum_{m>=n} gamma^(m-n) (q_n . k_m) v_m +
+// gamma^(L-n) q_n S_in (S_in: the state after the sequence), walked from the
+// last block to the first: for a block at t0 of length l,
+//   y_{t0+i} = sum_{j>=i} gamma^(j-i) (q_i.k_j) v_j + gamma^(l-i) q_i S
+//   S       <- gamma^l S + sum_{j<l} gamma^j k_j^T v_j
+// and state_out is the state at the sequence start.  The backward pass takes
+// its two sums that run backwards in time this way.
 constexpr int kCF_Cols = 32;
 constexpr int kCF_MaxC = 128;
 
+template <bool REV>
 __global__ void __launch_bounds__(256)
 chunkwise_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                      const float* __restrict__ v, float* __restrict__ y,
@@ -127,17 +138,20 @@ chunkwise_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
   }
   __syncthreads();
 
-  for (int t0 = 0; t0 < L; t0 += C) {
+  const int n_blk = (L + C - 1) / C;
+  for (int bi = 0; bi < n_blk; ++bi) {
+    const int t0 = (REV ? n_blk - 1 - bi : bi) * C;
     const int l = min(C, L - t0);
-    // 1. decayed, masked scores P[i][j] = gamma^(i-j) q_i.k_j (j <= i), for y
+    // 1. decayed, masked scores P[i][j] = gamma^(i-j) q_i.k_j (j <= i; REV:
+    // gamma^(j-i), j >= i), for y
     for (int e = tid; y && e < l * l; e += 256) {
       const int i = e / l, j = e % l;
       float s = 0.f;
-      if (j <= i) {
+      if (REV ? j >= i : j <= i) {
         const float* qi = qh + (size_t)(t0 + i) * dk;
         const float* kj = kh + (size_t)(t0 + j) * dk;
         for (int d = 0; d < dk; ++d) s = fmaf(qi[d], kj[d], s);
-        s *= pw[i - j];
+        s *= pw[REV ? j - i : i - j];
       }
       Ps[i * (C + 1) + j] = s;
     }
@@ -148,11 +162,12 @@ chunkwise_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
       const int i = e / kCF_Cols, c = e % kCF_Cols;
       if (c0 + c >= dv) continue;
       float a = 0.f;
-      for (int j = 0; j <= i; ++j) a = fmaf(Ps[i * (C + 1) + j], vh[(size_t)(t0 + j) * dv + c0 + c], a);
+      const int j_lo = REV ? i : 0, j_hi = REV ? l - 1 : i;
+      for (int j = j_lo; j <= j_hi; ++j) a = fmaf(Ps[i * (C + 1) + j], vh[(size_t)(t0 + j) * dv + c0 + c], a);
       const float* qi = qh + (size_t)(t0 + i) * dk;
       float x = 0.f;
       for (int d = 0; d < dk; ++d) x = fmaf(qi[d], Ss[d * kCF_Cols + c], x);
-      y[((size_t)bh * L + t0 + i) * dv + c0 + c] = fmaf(pw[i + 1], x, a);
+      y[((size_t)bh * L + t0 + i) * dv + c0 + c] = fmaf(pw[REV ? l - i : i + 1], x, a);
     }
     __syncthreads();
     // 3. state update
@@ -161,7 +176,7 @@ chunkwise_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
       if (c0 + c >= dv) continue;
       float a = pw[l] * Ss[e];
       for (int j = 0; j < l; ++j)
-        a = fmaf(pw[l - 1 - j] * kh[(size_t)(t0 + j) * dk + d], vh[(size_t)(t0 + j) * dv + c0 + c], a);
+        a = fmaf(pw[REV ? j : l - 1 - j] * kh[(size_t)(t0 + j) * dk + d], vh[(size_t)(t0 + j) * dv + c0 + c], a);
       Ss[e] = a;
     }
     __syncthreads();

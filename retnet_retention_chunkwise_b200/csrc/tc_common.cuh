@@ -24,6 +24,27 @@ namespace ret {
 // this is the single definition.
 __device__ int g_device_status = 0;
 
+// Bounds-checked builds (-DRET_BOUNDS_CHECK): RET_BC(cond, site) evaluates an
+// index check; when it fails, the first failing site number is kept in
+// g_bc_site, the device status word reads 5 (RET_EBOUNDS on the host) and the
+// caller skips the access the check guards.  In the normal build RET_BC is the
+// constant true and costs nothing.  Site numbers: 1xx chunkwise (dk <= 128),
+// 2xx chunkwise dk = 256, 3xx blocks of 129..256 rows, 4xx segment sums and
+// scan, 5xx parallel form, 6xx decode, 7xx GroupNorm.
+#ifdef RET_BOUNDS_CHECK
+__device__ unsigned int g_bc_site = 0;
+__device__ __forceinline__ bool bc_ok(bool ok, unsigned int site) {
+  if (!ok) {
+    atomicCAS(&g_bc_site, 0u, site);
+    atomicExch(&g_device_status, 5);
+  }
+  return ok;
+}
+#define RET_BC(cond, site) (::ret::bc_ok((cond), (site)))
+#else
+#define RET_BC(cond, site) (true)
+#endif
+
 // Optional event trace (builds with -DRET_TRACE only): %globaltimer stamps per
 // (CTA, block, event) written to a caller-provided buffer.  RET_TRACE_INIT reads
 // the buffer description once into registers; the stamps are plain stores.
@@ -247,6 +268,7 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
 // TMEM -> registers: 32 lanes x 32 consecutive 32-bit columns; thread t of the
 // warp gets lane (taddr.lane + t), r[i] = column (taddr.col + i).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  if (!RET_BC((taddr & 0xFFFFu) + 32u <= 512u && (taddr >> 16) + 32u <= 128u, 901)) return;
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -263,6 +285,7 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 // registers -> TMEM, 32 lanes x 16 columns.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  if (!RET_BC((taddr & 0xFFFFu) + 16u <= 512u && (taddr >> 16) + 32u <= 128u, 902)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
@@ -273,6 +296,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 // registers -> TMEM, 32 lanes x 32 columns.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  if (!RET_BC((taddr & 0xFFFFu) + 32u <= 512u && (taddr >> 16) + 32u <= 128u, 903)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "

@@ -47,10 +47,10 @@ def test_only_abi_symbols_are_exported():
 
 
 def test_status_strings_and_version(lib):
-    names = [lib.retention_status_str(i).decode() for i in range(5)]
-    assert names == ["RET_OK", "RET_EINVAL", "RET_EUNSUPPORTED", "RET_ECUDA", "RET_ETIMEOUT"]
+    names = [lib.retention_status_str(i).decode() for i in range(6)]
+    assert names == ["RET_OK", "RET_EINVAL", "RET_EUNSUPPORTED", "RET_ECUDA", "RET_ETIMEOUT", "RET_EBOUNDS"]
     assert lib.retention_status_str(99).decode() == "RET_UNKNOWN"
-    assert lib.retention_abi_version() == 103
+    assert lib.retention_abi_version() == 104
 
 
 def _g(*vals):
@@ -180,15 +180,14 @@ def test_host_entry_workspace_query(lib):
 def test_parallel_backward_validation(lib):
     s = _abi.RetShape(1, 2, 64, 64, 128)
     g = _g(0.5, 0.9)
-    need = lib.retention_parallel_backward_workspace_bytes(s, _abi.RET_F32)
-    assert need >= 3 * 64 * 64 * 4 * 2 + 3 * 64 * 128 * 4 * 2  # reversed q, k, v, dy and two results
-    call = lambda ws, nbytes, dt=_abi.RET_F32, shape=s, dy=FAKE: lib.retention_parallel_backward(  # noqa: E731
-        FAKE, FAKE, FAKE, g, dy, FAKE, FAKE, FAKE, shape, dt, ws, nbytes, None)
-    assert call(None, 0) == _abi.RET_EINVAL                      # no workspace
-    assert call(ctypes.c_void_p(0x100000), need - 1) == _abi.RET_EINVAL  # too small
-    assert call(ctypes.c_void_p(0x100000), need, dy=None) == _abi.RET_EINVAL
-    assert call(ctypes.c_void_p(0x100000), need, _abi.RET_BF16,
-                _abi.RetShape(1, 2, 64, 96, 128)) == _abi.RET_EUNSUPPORTED
+    # the anti-causal sums read the inputs in place: no workspace
+    assert lib.retention_parallel_backward_workspace_bytes(s, _abi.RET_F32) == 0
+    assert lib.retention_parallel_backward_workspace_bytes(s, _abi.RET_BF16) == 0
+    call = lambda dt=_abi.RET_F32, shape=s, dy=FAKE, gam=g: lib.retention_parallel_backward(  # noqa: E731
+        FAKE, FAKE, FAKE, gam, dy, FAKE, FAKE, FAKE, shape, dt, None, 0, None)
+    assert call(dy=None) == _abi.RET_EINVAL
+    assert call(gam=_g(0.5, 1.5)) == _abi.RET_EINVAL
+    assert call(_abi.RET_BF16, _abi.RetShape(1, 2, 64, 96, 128)) == _abi.RET_EUNSUPPORTED
 
 
 @NO_DEVICE
@@ -198,7 +197,10 @@ def test_chunkwise_backward_state_validation(lib):
     g = _g(0.5, 0.9)
     base = lib.retention_chunkwise_backward_workspace_bytes(64, s, _abi.RET_F32)
     need = lib.retention_chunkwise_backward_state_workspace_bytes(64, s, _abi.RET_F32)
-    assert base > 0 and need == base + 3 * ((2 * 64 * 128 * 4 + 255) // 256 * 256)
+    assert need == base + 3 * ((2 * 64 * 128 * 4 + 255) // 256 * 256)
+    # bf16 on a long sequence: the split scratch of the chunkwise calls
+    long = _abi.RetShape(1, 2, 8192, 128, 128)
+    assert lib.retention_chunkwise_backward_workspace_bytes(128, long, _abi.RET_BF16) > 0
     ws = ctypes.c_void_p(0x100000)
 
     def call(nbytes, s0=FAKE, dso=FAKE, ds0=FAKE, chunk=64, dt=_abi.RET_F32, shape=s, dy=FAKE, w=ws):

@@ -66,8 +66,9 @@ def test_static_scratch_matches_regular_entry_point_twice(lib):
 
 
 def test_static_scratch_shape_without_split(lib):
-    B, H, L, dk, dv, C = 2, 8, 512, 128, 256, 128  # enough (b, h) that no split is planned
+    B, H, L, dk, dv, C = 4, 8, 512, 256, 512, 128  # 128 (b, h, dv-slice) CTAs: no split is planned
     shape = _abi.RetShape(B, H, L, dk, dv)
+    assert lib.retention_chunkwise_workspace_bytes(C, shape, _abi.RET_BF16) == 0
     gam = (ctypes.c_float * H)(*inputs.multiscale_gammas(H).tolist())
     q, k, v, s_in = _case(7, B, H, L, dk, dv)
     y_ref, s_ref, y, s = torch.empty_like(v), torch.empty_like(s_in), torch.empty_like(v), torch.empty_like(s_in)
