@@ -253,10 +253,10 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   uint64_t* mma3done = bars + 36;  // MMA3 done -> P/O group (y)
   uint64_t* ofree = bars + 37;     // P/O group: O read out -> V group, MMA4 of the next block
   uint64_t* fin = bars + 38;       // teardown drain of the MMA pipe
-  uint64_t* ystaged = bars + 34;   // P/O group: y of the block staged in shared memory -> TMA store
+  uint64_t* ystaged = bars + 41;   // [4] P/O group: y of the block staged in its V buffer -> producer (TMA store)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 39);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 39) + 1;
-  float* pw = reinterpret_cast<float*>(bars + 40);  // gamma^0 .. gamma^128
+  float* pw = reinterpret_cast<float*>(bars + 48);  // gamma^0 .. gamma^128
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int vt = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;
@@ -297,7 +297,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     mbar_init(sready, 128);
     mbar_init(mma3done, 1);
     mbar_init(ofree, 128);
-    mbar_init(ystaged, 128);
+    for (int i = 0; i < 4; ++i) mbar_init(&ystaged[i], 128);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -360,7 +360,21 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         mbar_arrive_expect_tx(&fullQ[s], qk_bytes);
         for (int b = 0; b < DK / 64; ++b)
           tma_load_3d(sQ + s * sp.q_stage + b * 16384, &mapQ, &fullQ[s], b * 64, t0, bh);
-        if (it >= NS && !mbar_wait(&emptyV[s], par, abort_flag, a.lim)) break;
+        if (it >= NS) {
+          if (NS >= 2) {
+            // the V buffer holds y of block it - NS (staged there after MMA3):
+            // store it with two TMA tensor stores, and reload the buffer once
+            // they have read it
+            if (!mbar_wait(&ystaged[s], par, abort_flag, a.lim)) break;
+            const int ty = blk_t0(it - NS);
+            tma_store_3d(&mapY, sV + s * sp.v_stage, vt * kCW_DVT, ty, bh);
+            tma_store_3d(&mapY, sV + s * sp.v_stage + C * 128, vt * kCW_DVT + 64, ty, bh);
+            bulk_commit_group();
+            bulk_wait_read_all();
+          } else if (!mbar_wait(&emptyV[s], par, abort_flag, a.lim)) {
+            break;
+          }
+        }
         mbar_arrive_expect_tx(&fullV[s], v_bytes);
         for (int b = 0; b < 2; ++b)
           tma_load_3d(sV + s * sp.v_stage + b * C * 128, &mapV, &fullV[s], vt * kCW_DVT + b * 64, t0, bh);
@@ -374,6 +388,17 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           for (int b = 0; b < 2; ++b) tma_prefetch_l2_3d(&mapV, vt * kCW_DVT + b * 64, tp, bh);
         }
       }
+      // y of the last blocks (those no later load had to wait for)
+      if (NS >= 2 && issued == nck) {
+        for (int j = max(0, nck - NS); j < nck; ++j) {
+          if (!mbar_wait(&ystaged[j % NS], (j / NS) & 1, abort_flag, a.lim)) break;
+          const uint8_t* ys = sV + (j % NS) * sp.v_stage;
+          tma_store_3d(&mapY, ys, vt * kCW_DVT, blk_t0(j), bh);
+          tma_store_3d(&mapY, ys + C * 128, vt * kCW_DVT + 64, blk_t0(j), bh);
+          bulk_commit_group();
+        }
+      }
+      bulk_wait_all();  // the y stores issued by this thread are complete
       // every load issued must land before the CTA may exit
       for (int it = max(0, issued - NS); it < issued; ++it) {
         mbar_drain(&fullQ[it % NS], (it / NS) & 1, a.lim);
@@ -699,15 +724,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         tc_fence_before();
         mbar_arrive(ofree);
         fence_proxy_async_smem();
-        mbar_arrive(ystaged);
-        if (r == 0) {
-          if (!mbar_wait(ystaged, it & 1, abort_flag, a.lim)) break;
-          tma_store_3d(&mapY, ystage, vt * kCW_DVT, t0, bh);
-          tma_store_3d(&mapY, ystage + C * 128, vt * kCW_DVT + 64, t0, bh);
-          bulk_commit_group();
-          bulk_wait_read_all();
-          mbar_arrive(&emptyV[s]);
-        }
+        mbar_arrive(&ystaged[s]);  // the producer stores it
       } else {
         // Single stage: the V buffer is reloaded at once, so y goes straight
         // from registers to global memory (quad-transposed stores).
@@ -730,7 +747,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 7);
     }
   }
-  if (threadIdx.x == 0) bulk_wait_all();  // y stores issued by this thread are complete
+  if (threadIdx.x == 0) bulk_wait_all();  // no store is left in flight (the producer waited for its own)
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma) {
@@ -1356,6 +1373,9 @@ template <bool REV>
 __global__ void state_scan_kernel(const float* __restrict__ state_in, float* __restrict__ ws,
                                   int BH, int H, int dkdv, int n_seg, int seg_len, int last_len,
                                   const __grid_constant__ CwDecay dec) {
+  // One element per thread; the segment sums are loaded eight at a time
+  // ahead of the dependent multiply-adds, so the chain waits on arithmetic,
+  // not on one memory round trip per segment.
   const size_t total = (size_t)BH * dkdv;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (size_t)gridDim.x * blockDim.x) {
@@ -1366,16 +1386,30 @@ __global__ void state_scan_kernel(const float* __restrict__ state_in, float* __r
     float* slot = ws + (size_t)bh * n_seg * dkdv + off;
     if (!REV) {
       slot[0] = S;
-      for (int g = 1; g < n_seg; ++g) {
-        S = fmaf(gl, S, slot[(size_t)g * dkdv]);
-        slot[(size_t)g * dkdv] = S;
+      for (int g0 = 1; g0 < n_seg; g0 += 8) {
+        float d[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) d[u] = (g0 + u < n_seg) ? slot[(size_t)(g0 + u) * dkdv] : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (g0 + u < n_seg) {
+            S = fmaf(gl, S, d[u]);
+            slot[(size_t)(g0 + u) * dkdv] = S;
+          }
       }
     } else {
       const float gl_last = exp2f((float)last_len * dec.l2g[bh % H]);
       slot[(size_t)(n_seg - 1) * dkdv] = S;
-      for (int g = n_seg - 2; g >= 0; --g) {
-        S = fmaf(g + 1 == n_seg - 1 ? gl_last : gl, S, slot[(size_t)g * dkdv]);
-        slot[(size_t)g * dkdv] = S;
+      for (int g0 = n_seg - 2; g0 >= 0; g0 -= 8) {
+        float d[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) d[u] = (g0 - u >= 0) ? slot[(size_t)(g0 - u) * dkdv] : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (g0 - u >= 0) {
+            S = fmaf(g0 - u + 1 == n_seg - 1 ? gl_last : gl, S, d[u]);
+            slot[(size_t)(g0 - u) * dkdv] = S;
+          }
       }
     }
   }

@@ -254,7 +254,7 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
     chunk_state_kernel<DK, REV><<<g2, kCW_Threads, smem2, st>>>(mk, mv, a2, dec, static_cast<float*>(ws));
     if (launch_status() != RET_OK) return RET_ECUDA;
     const long long total = (long long)BH * DK * s.dv;
-    const int blocks = (int)std::min<long long>((total + 255) / 256, 4LL * sm_count());
+    const int blocks = (int)std::min<long long>((total + 255) / 256, 1LL << 20);  // one element per thread
     state_scan_kernel<REV><<<blocks, 256, 0, st>>>(state_in, static_cast<float*>(ws), BH, s.H, DK * s.dv, n_seg,
                                                    seg_chunks * C, s.L - (n_seg - 1) * seg_chunks * C, dec);
     if (launch_status() != RET_OK) return RET_ECUDA;
