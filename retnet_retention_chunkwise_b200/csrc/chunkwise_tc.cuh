@@ -12,12 +12,13 @@
 // held transposed (lanes = the 128 dv columns, columns = dk) so the state
 // update has M = 128 for every dk.  Warp roles (448 threads, both kernels):
 //   warps 0-3    P/O group: TMEM lane r = row r of the block.  P -> P~ in place
-//                (bf16 pairs), xi on O in the direct form, y out.
+//                (bf16 pairs), xi on O in the direct form; y out in the dk = 256
+//                kernel.
 //   warps 4-7    S group: the state copy Sb for the next block's cross term
 //                (and the state rescale when it is due), state_out.
 //   warps 8-11   V group: zeta on the rows of V (rescaled form) or of K, or
-//                (zeta V)^T in TMEM (direct form); in the dk = 256 kernel it
-//                also keeps half of the state.
+//                (zeta V)^T in TMEM (direct form); y out in the dk <= 128
+//                kernel; in the dk = 256 kernel it also keeps half of the state.
 //   warp 12      TMA producer: Q, K, V of each block on their own barriers.
 //   warp 13      TMEM allocator; lane 0 issues every tcgen05.mma.
 //
@@ -29,12 +30,15 @@
 //   direct (smaller gamma): P~_ij = P_ij gamma^(i-j), O scaled by xi after the
 //     cross term, the state decayed by gamma^l in TMEM each block.
 //
-// chunkwise_tc_kernel<DK> (DK 64, 128; NS = 2..4 stages, P double-buffered):
+// chunkwise_tc_kernel<DK> (DK 64, 128; NS = 2..4 stages, O double-buffered):
 //   MMA1  P[pb] = Q K^T            A = Q  (smem, K-major)   B = K  (smem, K-major)
 //   MMA5  S^T  += (zeta V)^T K     A = V  (smem, MN-major, or TMEM)  B = K (smem, MN-major)
 //   MMA4  O     = Q Sb             A = Q  (smem, K-major)   B = Sb (smem, K-major)
 //   MMA3  O    += P~ V             A = P~ (TMEM, bf16)      B = V  (smem, MN-major)
-//   TMEM: S^T [0, DK), P buffers [DK, DK + 256), O [DK + 256, DK + 384).
+//   TMEM: S^T [0, DK), P [DK, DK + 128), O buffers [DK + 128, DK + 384): block
+//   it uses O buffer it % 2, so MMA4 of the next block does not wait for the
+//   read-out of this block's y, which the V group does while the P/O group
+//   turns the next block's P into P~.
 // chunkwise_tc256_kernel (DK = 256, one stage): the scores and the cross term
 // in one N = C + 128 MMA, [P | X] = Q [K ; Sb]^T, then the state update and
 // P~ V (see there).
@@ -225,9 +229,11 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapY,
                     const CwArgs a, const __grid_constant__ CwDecay dec) {
   static_assert(DK == 64 || DK == 128 || DK == 256, "dk must be 64, 128 or 256");
-  constexpr int NP = (DK <= 128) ? 2 : 1;
-  constexpr uint32_t TM_S = 0, TM_P = DK, TM_O = DK + 128 * NP;
+  // TMEM: S^T [0, DK), P [DK, DK + 128), two O buffers of 128 columns after
+  // it, so the next block's MMA4 never waits for this block's y read-out.
+  constexpr uint32_t TM_S = 0, TM_P = DK, TM_O = DK + 128;
   constexpr uint32_t kTmemCols = 512;
+  static_assert(DK + 3 * 128 <= (int)kTmemCols, "TMEM plan");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align_smem(smem_raw);
@@ -243,17 +249,15 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   uint64_t* fullV = bars + 8;      // [4] TMA -> V group, MMA
   uint64_t* emptyQ = bars + 12;    // [4] MMA4 done -> producer
   uint64_t* emptyK = bars + 16;    // [4] MMA5 done -> producer
-  uint64_t* emptyV = bars + 20;    // [4] y of the block stored out of the V buffer -> producer
   uint64_t* zready = bars + 24;    // [4] V group: scaled V of stage s written -> MMA5 (and MMA3)
-  uint64_t* pfull = bars + 28;     // [2] MMA1 done -> P/O group
-  uint64_t* pfree = bars + 30;     // [2] MMA3 done -> MMA1 of block it+NP
+  uint64_t* pfull = bars + 28;     // MMA1 done -> P/O group
+  uint64_t* mma3done = bars + 30;  // [2] per O buffer: MMA3 done -> V group (y)
   uint64_t* ocross = bars + 32;    // MMA5 + MMA4 done -> P/O group, S group
   uint64_t* pready = bars + 33;    // P/O group: P~ (and xi O) written -> MMA3
   uint64_t* sready = bars + 35;    // S group: state copy + rescaled state written -> MMA5, MMA4
-  uint64_t* mma3done = bars + 36;  // MMA3 done -> P/O group (y)
-  uint64_t* ofree = bars + 37;     // P/O group: O read out -> V group, MMA4 of the next block
+  uint64_t* ofree = bars + 36;     // [2] per O buffer: V group read y out -> MMA4 two blocks later
   uint64_t* fin = bars + 38;       // teardown drain of the MMA pipe
-  uint64_t* ystaged = bars + 41;   // [4] P/O group: y of the block staged in its V buffer -> producer (TMA store)
+  uint64_t* ystaged = bars + 41;   // [4] V group: y of the block staged in its V buffer -> producer (TMA store)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 39);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 39) + 1;
   float* pw = reinterpret_cast<float*>(bars + 48);  // gamma^0 .. gamma^128
@@ -285,18 +289,16 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       mbar_init(&fullV[i], 1);
       mbar_init(&emptyQ[i], 1);
       mbar_init(&emptyK[i], 1);
-      mbar_init(&emptyV[i], 1);
     }
     for (int i = 0; i < 4; ++i) mbar_init(&zready[i], 128);
+    mbar_init(pfull, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&pfull[i], 1);
-      mbar_init(&pfree[i], 1);
+      mbar_init(&mma3done[i], 1);
+      mbar_init(&ofree[i], 128);
     }
     mbar_init(ocross, 1);
     mbar_init(pready, 128);
     mbar_init(sready, 128);
-    mbar_init(mma3done, 1);
-    mbar_init(ofree, 128);
     for (int i = 0; i < 4; ++i) mbar_init(&ystaged[i], 128);
     mbar_init(fin, 1);
     *abort_flag = 0;
@@ -361,19 +363,15 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         for (int b = 0; b < DK / 64; ++b)
           tma_load_3d(sQ + s * sp.q_stage + b * 16384, &mapQ, &fullQ[s], b * 64, t0, bh);
         if (it >= NS) {
-          if (NS >= 2) {
-            // the V buffer holds y of block it - NS (staged there after MMA3):
-            // store it with two TMA tensor stores, and reload the buffer once
-            // they have read it
-            if (!mbar_wait(&ystaged[s], par, abort_flag, a.lim)) break;
-            const int ty = blk_t0(it - NS);
-            tma_store_3d(&mapY, sV + s * sp.v_stage, vt * kCW_DVT, ty, bh);
-            tma_store_3d(&mapY, sV + s * sp.v_stage + C * 128, vt * kCW_DVT + 64, ty, bh);
-            bulk_commit_group();
-            bulk_wait_read_all();
-          } else if (!mbar_wait(&emptyV[s], par, abort_flag, a.lim)) {
-            break;
-          }
+          // the V buffer holds y of block it - NS (staged there after MMA3):
+          // store it with two TMA tensor stores, and reload the buffer once
+          // they have read it
+          if (!mbar_wait(&ystaged[s], par, abort_flag, a.lim)) break;
+          const int ty = blk_t0(it - NS);
+          tma_store_3d(&mapY, sV + s * sp.v_stage, vt * kCW_DVT, ty, bh);
+          tma_store_3d(&mapY, sV + s * sp.v_stage + C * 128, vt * kCW_DVT + 64, ty, bh);
+          bulk_commit_group();
+          bulk_wait_read_all();
         }
         mbar_arrive_expect_tx(&fullV[s], v_bytes);
         for (int b = 0; b < 2; ++b)
@@ -389,7 +387,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         }
       }
       // y of the last blocks (those no later load had to wait for)
-      if (NS >= 2 && issued == nck) {
+      if (issued == nck) {
         for (int j = max(0, nck - NS); j < nck; ++j) {
           if (!mbar_wait(&ystaged[j % NS], (j / NS) & 1, abort_flag, a.lim)) break;
           const uint8_t* ys = sV + (j % NS) * sp.v_stage;
@@ -409,7 +407,10 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   } else if (warp == kWarpMma) {
     // ---------------------------------------------------------- MMA issuer
     // Order per block: MMA1 (P = Q K^T), MMA5 (state update; frees K), MMA4
-    // (Q S; frees Q), MMA3 (P~ V; frees V and P).
+    // (Q S into O buffer it % 2; frees Q), MMA3 (P~ V).  MMAs issued by one
+    // thread run in order, so MMA1 of the next block overwrites P only after
+    // MMA3 has read P~, and MMA4 overwrites an O buffer only after MMA5 has
+    // read (zeta V)^T from it.
     if (lane == 0 && nck > 0) {
       const uint32_t id1 = idesc_bf16(128, C, false, false);
       const uint32_t id4 = idesc_bf16(128, kCW_DVT, false, false);
@@ -417,11 +418,11 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       const uint32_t id5 = idesc_bf16(128, DK, rescaled, true);  // A = V^T (smem, MN-major) or TMEM
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aSb = smem_u32(sSb);
       for (int it = 0; it < nck; ++it) {
-        const int s = it % NS, pb = it % NP;
+        const int s = it % NS, ob = it & 1;
         const uint32_t par = (it / NS) & 1;
+        const uint32_t t_o = tm + TM_O + 128u * (uint32_t)ob;
         if (!mbar_wait(&fullK[s], par, abort_flag, a.lim)) break;
         if (!mbar_wait(&fullQ[s], par, abort_flag, a.lim)) break;
-        if (it >= NP && !mbar_wait(&pfree[pb], ((it / NP) - 1) & 1, abort_flag, a.lim)) break;
         RET_TRACE_STAMP(cta_id, it, 1);
         tc_fence_after();
         const uint32_t q_s = aQ + s * sp.q_stage, k_s = aK + s * sp.k_stage, v_s = aV + s * sp.v_stage;
@@ -430,13 +431,13 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(q_s + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(k_s + (kk / 4) * C * 128 + (kk % 4) * 32, 16, 1024);
-          mma_ss(tm + TM_P + pb * 128, ad, bd, id1, kk > 0);
+          mma_ss(tm + TM_P, ad, bd, id1, kk > 0);
         }
-        mma_commit(&pfull[pb]);
+        mma_commit(pfull);
         // MMA5: S^T += (zeta V)^T K, onto the state already rescaled by gamma^l.
         // Rescaled form: zeta V is the V tile itself (scaled in place), read
         // MN-major from shared memory.  Direct form: (zeta V)^T was built in the
-        // (free) O columns of TMEM.
+        // columns of this block's (free) O buffer.
         // zready is per stage: in the rescaled form the V group runs ahead by up
         // to NS blocks, so one barrier could complete two phases unobserved.
         if (!mbar_wait(&zready[s], par, abort_flag, a.lim)) break;
@@ -448,19 +449,17 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           if (rescaled)
             mma_ss(tm + TM_S, sdesc_sw128(v_s + kk * 2048, C * 128, 1024), bd, id5, 1);
           else
-            mma_ts(tm + TM_S, tm + TM_O + kk * 8, bd, id5, 1);
+            mma_ts(tm + TM_S, t_o + kk * 8, bd, id5, 1);
         }
         mma_commit(&emptyK[s]);
-        // MMA4: O = Q S_copy, once the previous block's O was drained.  It
-        // overwrites the O columns after MMA5 has read them (MMAs issued by one
-        // thread run in order).
-        if (!mbar_wait(ofree, it & 1, abort_flag, a.lim)) break;
+        // MMA4: O = Q S_copy into buffer ob, once y of block it - 2 left it
+        if (!mbar_wait(&ofree[ob], (it >> 1) & 1, abort_flag, a.lim)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(q_s + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(aSb + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
-          mma_ss(tm + TM_O, ad, bd, id4, kk > 0);
+          mma_ss(t_o, ad, bd, id4, kk > 0);
         }
         mma_commit(ocross);
         mma_commit(&emptyQ[s]);
@@ -470,46 +469,51 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         tc_fence_after();
         for (int kk = 0; kk < C / 16; ++kk) {
           const uint64_t bd = sdesc_sw128(v_s + kk * 2048, C * 128, 1024);
-          mma_ts(tm + TM_O, tm + TM_P + pb * 128 + kk * 8, bd, id3, 1);
+          mma_ts(t_o, tm + TM_P + kk * 8, bd, id3, 1);
         }
-        mma_commit(&pfree[pb]);
-        mma_commit(mma3done);
+        mma_commit(&mma3done[ob]);
       }
       mma_commit(fin);
       mbar_drain(fin, 0, a.lim);
     }
   } else if (warp >= kWarpZBase) {
     // ---------------------------------------------------- V group (4 warps)
+    // Two jobs, one block apart: zeta for block it + 1 (on V in the rescaled
+    // form, (zeta V)^T into that block's O buffer in the direct form), then y
+    // of block it out of its O buffer once MMA3 is done.  TMEM lane t = dv
+    // column t for (zeta V)^T, row t of the block for y.
     const uint32_t t = threadIdx.x - kWarpZBase * 32;
-    float rho = cw_rho_first(rescaled, pw[l_first]);
-    for (int it = 0; it < nck; ++it) {
+    const uint32_t lane_off = (uint32_t)((warp - kWarpZBase) * 32) << 16;
+    const int row_lo = (warp - kWarpZBase) * 32;
+    float rho_z = cw_rho_first(rescaled, pw[l_first]);  // rho of the block zeta is applied to
+    float rho_y = rho_z;                                 // rho of the block read out
+    mbar_arrive(&ofree[0]);  // both O buffers start free
+    mbar_arrive(&ofree[1]);
+    auto zeta_step = [&](int it) -> bool {
       const int s = it % NS;
-      if (!mbar_wait(&fullV[s], (it / NS) & 1, abort_flag, a.lim)) break;
-      // Direct form: (zeta V)^T goes into the O columns, free once the previous
-      // block's O was drained.
-      if (!rescaled && !mbar_wait(ofree, it & 1, abort_flag, a.lim)) break;
-      tc_fence_after();
+      if (!mbar_wait(&fullV[s], (it / NS) & 1, abort_flag, a.lim)) return false;
       const int l = min(C, a.L - blk_t0(it));
       uint8_t* vs = sV + s * sp.v_stage;
       if (rescaled) {
         // row j of the V tile scaled in place by zeta_j = gamma^(l-1-j) (0 past the end)
         if ((int)t < C && RET_BC(s < NS, 105)) {
-          const float zs = (((int)t < l) ? pw[REV ? (int)t : l - 1 - (int)t] : 0.f) * __frcp_rn(rho);  // zeta / rho
+          const float zs = (((int)t < l) ? pw[REV ? (int)t : l - 1 - (int)t] : 0.f) * __frcp_rn(rho_z);  // zeta / rho
           scale_row_sw128(vs, t, zs);
           scale_row_sw128(vs + C * 128, t, zs);
         }
         fence_proxy_async_smem();
       } else {
-        // (zeta V)^T into the O columns: lane v holds column v of V scaled
+        // (zeta V)^T into the block's O buffer (its y of two blocks before was
+        // read out by this group already): lane v holds column v of V scaled
         // row-wise by zeta_j, two rows per 32-bit column.  V is read from its
         // swizzled tile as 32-bit pairs (v0, v0+1) of rows j and j+1 and
         // re-paired by a byte permute.
-        const uint32_t lane_off = (uint32_t)((warp - kWarpZBase) * 32) << 16;
         const uint32_t vb = t / 64, vv = t % 64;
         const uint32_t vchunk = vv / 8;                // 16-byte chunk of the row
         const uint32_t vbyte = ((vv % 8) & ~1u) * 2u;  // byte of the pair (v0, v0+1): 0, 4, 8, 12
         const uint32_t sel = (t & 1) ? 0x7632u : 0x5410u;
         const uint8_t* vt_s = vs + vb * C * 128;
+        const uint32_t t_o = tm + lane_off + TM_O + 128u * (uint32_t)(it & 1);
         for (int j0 = 0; j0 < C; j0 += 32) {
           uint32_t w[16];
 #pragma unroll
@@ -527,14 +531,53 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           // When C % 32 == 16 the last piece covers 16 rows past C (zeta = 0
           // there, read from the next, allocated, part of shared memory); the
           // results land in columns MMA5 never reads.
-          tmem_st16(tm + lane_off + TM_O + j0 / 2, w);
+          tmem_st16(t_o + j0 / 2, w);
         }
         tmem_st_wait();
         tc_fence_before();
       }
       mbar_arrive(&zready[s]);
       if (t == 0) RET_TRACE_STAMP(cta_id, it, 3);
-      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[blk_len(it + 1)]);
+      if (it + 1 < nck && rescaled) rho_z = cw_rho_next(rho_z, pw[blk_len(it + 1)]);
+      return true;
+    };
+    // y = (gamma^(r+1-l) rho in the rescaled form) O, staged in the block's V
+    // buffer (dead after MMA3, not reloaded before the producer stored y out of
+    // it) for two TMA tensor stores by the producer.
+    auto y_step = [&](int it) -> bool {
+      const int s = it % NS, ob = it & 1;
+      if (!mbar_wait(&mma3done[ob], (it >> 1) & 1, abort_flag, a.lim)) return false;
+      if (t == 0) RET_TRACE_STAMP(cta_id, it, 9);
+      tc_fence_after();
+      const int l = blk_len(it);
+      const int r = (int)t;
+      const float yf = rescaled ? exp2f((float)(REV ? -r : r + 1 - l) * l2g) * rho_y : 1.f;
+      if (it + 1 < nck && rescaled) rho_y = cw_rho_next(rho_y, pw[blk_len(it + 1)]);
+      uint8_t* ystage = sV + s * sp.v_stage;
+      const uint32_t t_o = tm + lane_off + TM_O + 128u * (uint32_t)ob;
+#pragma unroll
+      for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(t_o + c0, o);
+        tmem_ld_wait();
+        float x[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) x[u] = yf * __uint_as_float(o[u]);
+        if (r < C) store_row32_sw128(ystage, (uint32_t)C * 128u, (uint32_t)r, (uint32_t)c0, x);
+      }
+      tc_fence_before();
+      mbar_arrive(&ofree[ob]);
+      fence_proxy_async_smem();
+      mbar_arrive(&ystaged[s]);  // the producer stores it
+      if (t == 0) RET_TRACE_STAMP(cta_id, it, 7);
+      (void)row_lo;
+      return true;
+    };
+    if (nck > 0 && zeta_step(0)) {
+      for (int it = 0; it < nck; ++it) {
+        if (it + 1 < nck && !zeta_step(it + 1)) break;
+        if (!y_step(it)) break;
+      }
     }
   } else if (warp >= kWarpSBase) {
     // ---------------------------------------------------- S group (4 warps)
@@ -548,6 +591,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     const float g0 = pw[l_first];
     float rho = cw_rho_first(rescaled, g0);
     {
+      // the segment states come from the launches before this one on the
+      // stream, which may still be running (programmatic dependent launch)
+      if (a.n_seg > 1) griddep_wait();
       const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
                                        : (a.state_in ? a.state_in + (size_t)bh * dkdv : nullptr);
       // rescaled: U = S_in (or gamma^l0 S_in when rho was reset), Sb = bf16(U);
@@ -622,24 +668,22 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     }
   } else {
     // -------------------------------------------------- P/O group (4 warps)
-    // TMEM lane r = row r of P and O (token t0 + r of the block).
+    // TMEM lane r = row r of P and O (token t0 + r of the block).  P -> P~ for
+    // MMA3 (and xi on O in the direct form); y is read out by the V group.
     const int r = (int)threadIdx.x;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int row_lo = warp * 32;  // rows of this warp: [row_lo, row_lo + 32)
-    float rho = cw_rho_first(rescaled, pw[l_first]);
-    mbar_arrive(ofree);            // O starts free
     for (int it = 0; it < nck; ++it) {
-      const int pb = it % NP;
       const int t0 = blk_t0(it);
       const int l = min(C, a.L - t0);
-      if (!mbar_wait(&pfull[pb], (it / NP) & 1, abort_flag, a.lim)) break;
+      if (!mbar_wait(pfull, it & 1, abort_flag, a.lim)) break;
       (void)RET_BC(l >= 1 && l <= C && t0 >= 0 && t0 < a.L, 107);
       tc_fence_after();
       // P -> P~ in place (two bf16 per column).  Rows past the block end read
       // zero Q rows and columns past it zero K rows, so P is already 0 there.
       // Rescaled form: P~ = P on and below the diagonal (decay lives in zeta V
       // and the row factor applied at the end).  Direct form: P~ = P gamma^(r-j).
-      const uint32_t tp = tm + lane_off + TM_P + pb * 128;
+      const uint32_t tp = tm + lane_off + TM_P;
       for (int j0 = 0; j0 < C; j0 += 32) {
         uint32_t pr[32];
         tmem_ld32(tp + j0, pr);
@@ -682,69 +726,24 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       }
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 5);
       if (!rescaled) {
-        // O *= xi_r = gamma^(r+1) once MMA4 wrote Q S_prev into O
+        // O *= xi_r = gamma^(r+1) once MMA4 wrote Q S_prev into this block's O buffer
         if (!mbar_wait(ocross, it & 1, abort_flag, a.lim)) break;
         tc_fence_after();
         const float xi = pw[REV ? max(l - r, 0) : r + 1];
+        const uint32_t t_o = tm + lane_off + TM_O + 128u * (uint32_t)(it & 1);
         for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
           uint32_t o[32];
-          tmem_ld32(tm + lane_off + TM_O + c0, o);
+          tmem_ld32(t_o + c0, o);
           tmem_ld_wait();
 #pragma unroll
           for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * xi);
-          tmem_st32(tm + lane_off + TM_O + c0, o);
+          tmem_st32(t_o + c0, o);
         }
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(pready);
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 6);
-      // O -> y once MMA3 added P~ V.  Rescaled form: y_r = gamma^(r+1-l) O_r.
-      if (!mbar_wait(mma3done, it & 1, abort_flag, a.lim)) break;
-      if (r == 0) RET_TRACE_STAMP(cta_id, it, 9);
-      tc_fence_after();
-      const int s = it % NS;
-      const float yf = rescaled ? exp2f((float)(REV ? -r : r + 1 - l) * l2g) * rho : 1.f;
-      if (it + 1 < nck && rescaled) rho = cw_rho_next(rho, pw[blk_len(it + 1)]);
-      if (NS >= 2) {
-        // The V tile is dead after MMA3 and its buffer is not needed again for
-        // NS-1 blocks: stage y there (bf16, 128B-swizzled) for two TMA tensor
-        // stores; the producer reloads the buffer once the stores have read it.
-        uint8_t* ystage = sV + s * sp.v_stage;
-#pragma unroll
-        for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(tm + lane_off + TM_O + c0, o);
-          tmem_ld_wait();
-          float x[32];
-#pragma unroll
-          for (int u = 0; u < 32; ++u) x[u] = yf * __uint_as_float(o[u]);
-          if (r < C) store_row32_sw128(ystage, (uint32_t)C * 128u, (uint32_t)r, (uint32_t)c0, x);
-        }
-        tc_fence_before();
-        mbar_arrive(ofree);
-        fence_proxy_async_smem();
-        mbar_arrive(&ystaged[s]);  // the producer stores it
-      } else {
-        // Single stage: the V buffer is reloaded at once, so y goes straight
-        // from registers to global memory (quad-transposed stores).
-        if (r == 0) mbar_arrive(&emptyV[s]);
-        __nv_bfloat16* wrow0 = a.y + ((size_t)bh * a.L + t0 + row_lo) * a.dv + vt * kCW_DVT;
-#pragma unroll
-        for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(tm + lane_off + TM_O + c0, o);
-          tmem_ld_wait();
-          // the factor differs per row: scale before the transpose
-#pragma unroll
-          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(yf * __uint_as_float(o[u]));
-          if (RET_BC(t0 + l <= a.L && vt * kCW_DVT + c0 + 32 <= a.dv, 102))
-            store_rows_bf16_quad(wrow0 + c0, (size_t)a.dv, lane, o, 1.f, l - row_lo);
-        }
-        tc_fence_before();
-        mbar_arrive(ofree);
-      }
-      if (r == 0) RET_TRACE_STAMP(cta_id, it, 7);
     }
   }
   if (threadIdx.x == 0) bulk_wait_all();  // no store is left in flight (the producer waited for its own)
@@ -972,6 +971,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
     const float g0 = pw[l_first];
     float rho = cw_rho_first(rescaled, g0);
     {
+      if (a.n_seg > 1) griddep_wait();  // segment states from the launches before (see above)
       const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
                                        : (a.state_in ? a.state_in + (size_t)bh * dkdv : nullptr);
       // TMEM starts as gu S_in: rescaled, U = S_in (or gamma^l0 S_in when rho
@@ -1349,6 +1349,9 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
       }
     }
   }
+  // The scan (or fold) that consumes the segment sums may be launched now; it
+  // waits for this grid's completion before it reads them.
+  if (threadIdx.x == 0) griddep_launch_dependents();
   tc_fence_before();
   __syncthreads();
   if (warp == 5) {
@@ -1376,6 +1379,7 @@ __global__ void state_scan_kernel(const float* __restrict__ state_in, float* __r
   // One element per thread; the segment sums are loaded eight at a time
   // ahead of the dependent multiply-adds, so the chain waits on arithmetic,
   // not on one memory round trip per segment.
+  griddep_wait();  // the segment sums of chunk_state_kernel
   const size_t total = (size_t)BH * dkdv;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (size_t)gridDim.x * blockDim.x) {
@@ -1413,6 +1417,8 @@ __global__ void state_scan_kernel(const float* __restrict__ state_in, float* __r
       }
     }
   }
+  // the main kernel, launched behind this one, waits for its completion
+  if (threadIdx.x == 0) griddep_launch_dependents();
 }
 
 }  // namespace ret

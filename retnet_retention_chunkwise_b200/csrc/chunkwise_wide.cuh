@@ -287,6 +287,7 @@ chunkwise_wide_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_con
     const float g0 = pw[max(min(C, a.L - c_begin * C), 0)];
     float rho = cw_rho_first(rescaled, g0);
     {
+      if (a.n_seg > 1) griddep_wait();  // segment states from the launches before this one
       const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
                                        : (a.state_in ? a.state_in + (size_t)bh * dkdv : nullptr);
       const float gu = (rho == 1.f) ? g0 : 1.f;

@@ -12,6 +12,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include <nvtx3/nvToolsExt.h>
@@ -139,6 +140,25 @@ void fill_l2g(CwDecay& d, const float* gamma, int H) {
 
 ret_status launch_status() { return cudaGetLastError() == cudaSuccess ? RET_OK : RET_ECUDA; }
 
+// Launch that may start while the previous launch on the stream is still
+// running (programmatic dependent launch).  The kernel must call griddep_wait
+// before it touches memory that launch writes or reads.
+template <typename... KArgs, typename... Args>
+ret_status launch_after(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                        Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? RET_OK : RET_ECUDA;
+}
+
 bool tc_shape_ok(const ret_shape& s) {
   return (s.dk == 64 || s.dk == 128 || s.dk == 256) && (s.dv % kCW_DVT) == 0;
 }
@@ -201,6 +221,9 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
   if (C <= 128) {
     for (int n = kCW_MaxStages; n >= 1; --n)
       if ((int)cw_smem_plan(DK, C, n).total <= smax) { ns = n; break; }
+    // the dk <= 128 kernel stages y in a V buffer while the next block's V
+    // loads into another: two stages at least
+    if (DK <= 128 && ns < 2) ns = 0;
   } else if (DK <= 128 && (int)cw_wide_smem_plan(DK, C).total <= smax) {
     ns = 1;  // blocks of 129..256 rows: one stage, two row halves
   }
@@ -253,12 +276,16 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
     dim3 g2(s.dv / kCW_DVT, BH, n_seg - 1);
     chunk_state_kernel<DK, REV><<<g2, kCW_Threads, smem2, st>>>(mk, mv, a2, dec, static_cast<float*>(ws));
     if (launch_status() != RET_OK) return RET_ECUDA;
+    // The scan and the main kernel are launched behind the kernel before them
+    // (programmatic dependent launch): their prologues overlap its tail, and
+    // each waits (griddep_wait) before it reads the segment states.
     const long long total = (long long)BH * DK * s.dv;
     const int blocks = (int)std::min<long long>((total + 255) / 256, 1LL << 20);  // one element per thread
-    state_scan_kernel<REV><<<blocks, 256, 0, st>>>(state_in, static_cast<float*>(ws), BH, s.H, DK * s.dv, n_seg,
-                                                   seg_chunks * C, s.L - (n_seg - 1) * seg_chunks * C, dec);
-    if (launch_status() != RET_OK) return RET_ECUDA;
+    if (launch_after(state_scan_kernel<REV>, dim3(blocks), dim3(256), 0, st, state_in, static_cast<float*>(ws), BH,
+                     s.H, DK * s.dv, n_seg, seg_chunks * C, s.L - (n_seg - 1) * seg_chunks * C, dec) != RET_OK)
+      return RET_ECUDA;
   }
+  const bool after = n_seg > 1;
   dim3 grid(s.dv / kCW_DVT, BH, n_seg);
   if constexpr (DK == 256) {
     // one stage; scores and cross-block term fused into one wide MMA
@@ -268,6 +295,8 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
     if (cudaFuncSetAttribute(chunkwise_tc256_kernel<REV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)p256.total) != cudaSuccess)
       return RET_ECUDA;
+    if (after) return launch_after(chunkwise_tc256_kernel<REV>, grid, dim3(kCW_MainThreads), p256.total, st, mq, mk,
+                                   mv, a, dec);
     chunkwise_tc256_kernel<REV><<<grid, kCW_MainThreads, p256.total, st>>>(mq, mk, mv, a, dec);
     return launch_status();
   } else {
@@ -276,12 +305,16 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
       if (cudaFuncSetAttribute(chunkwise_wide_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)pw.total) != cudaSuccess)
         return RET_ECUDA;
+      if (after) return launch_after(chunkwise_wide_kernel<DK>, grid, dim3(kCW_MainThreads), pw.total, st, mq, mk,
+                                     mv, a, dec);
       chunkwise_wide_kernel<DK><<<grid, kCW_MainThreads, pw.total, st>>>(mq, mk, mv, a, dec);
       return launch_status();
     }
     if (cudaFuncSetAttribute(chunkwise_tc_kernel<DK, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)plan.total) != cudaSuccess)
       return RET_ECUDA;
+    if (after) return launch_after(chunkwise_tc_kernel<DK, REV>, grid, dim3(kCW_MainThreads), plan.total, st, mq,
+                                   mk, mv, my, a, dec);
     chunkwise_tc_kernel<DK, REV><<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, my, a, dec);
     return launch_status();
   }
@@ -290,7 +323,7 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
 // Launch state_fold_kernel: out = fold of n parts (see state_fold.cuh).
 ret_status launch_state_fold(const float* state_in, const float* parts, float* out, const ret_shape& s,
                              const float* gamma, int n, const int* lens, long long part_stride,
-                             long long bh_stride, cudaStream_t st) {
+                             long long bh_stride, cudaStream_t st, bool after = false) {
   HeadLog2 hl;
   FoldLens fl;
   for (int h = 0; h < s.H; ++h) hl.l2g[h] = log2_gamma(gamma[h]);
@@ -299,6 +332,8 @@ ret_status launch_state_fold(const float* state_in, const float* parts, float* o
   const long long BH = (long long)s.B * s.H;
   const long long total = BH * s.dk * s.dv;
   const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>((total + 255) / 256, 8LL * sm_count()));
+  if (after) return launch_after(state_fold_kernel, dim3(grid), dim3(256), 0, st, state_in, parts, out, BH, s.H,
+                                 s.dk * s.dv, n, part_stride, bh_stride, hl, fl);
   state_fold_kernel<<<grid, 256, 0, st>>>(state_in, parts, out, BH, s.H, s.dk * s.dv, n, part_stride, bh_stride,
                                           hl, fl);
   return launch_status();
@@ -371,7 +406,7 @@ ret_status launch_chunk_state(const void* k, const void* v, const float* gamma, 
   for (int g = 0; g < n_seg; ++g) lens[g] = std::min(s.L, (g + 1) * seg_chunks * C) - g * seg_chunks * C;
   const long long dkdv = (long long)DK * s.dv;
   return launch_state_fold(state_in, static_cast<const float*>(ws) + dkdv, state_out, s, gamma, n_seg, lens, dkdv,
-                           (long long)(n_seg + 1) * dkdv, st);
+                           (long long)(n_seg + 1) * dkdv, st, /*after=*/true);
 }
 
 template <int DK, int DVT, bool REV>

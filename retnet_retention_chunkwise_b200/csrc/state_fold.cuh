@@ -16,6 +16,7 @@
 #include <stdint.h>
 
 #include "simt_f32.cuh"  // HeadLog2, decay_pow
+#include "tc_common.cuh"  // griddep_wait
 
 namespace ret {
 
@@ -33,6 +34,7 @@ __global__ void __launch_bounds__(256) state_fold_kernel(const float* state_in, 
                                                          long long part_stride, long long bh_stride,
                                                          const __grid_constant__ HeadLog2 hl,
                                                          const __grid_constant__ FoldLens fl) {
+  griddep_wait();  // parts written by the launch before this one (if it was programmatic)
   const long long total = BH * dkdv;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (long long)gridDim.x * blockDim.x) {
