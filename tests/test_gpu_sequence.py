@@ -31,6 +31,7 @@ TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
     (torch.bfloat16, 2, 3, 1000, 128, 256, 64),    # ragged tail
     (torch.bfloat16, 1, 2, 777, 64, 128, 256),     # 256-row blocks
     (torch.bfloat16, 1, 1, 100, 128, 128, 128),    # one block
+    (torch.bfloat16, 1, 2, 500, 64, 256, 64),      # dk = 64, two dv slices per CTA
     (torch.float32, 1, 2, 300, 64, 48, 32),
 ])
 def test_chunkwise_state_matches_state_out(dt, B, H, L, dk, dv, C):
