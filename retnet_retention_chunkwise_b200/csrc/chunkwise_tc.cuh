@@ -257,10 +257,17 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   uint64_t* sready = bars + 35;    // S group: state copy + rescaled state written -> MMA5, MMA4
   uint64_t* ofree = bars + 36;     // [2] per O buffer: V group read y out -> MMA4 two blocks later
   uint64_t* fin = bars + 38;       // teardown drain of the MMA pipe
-  uint64_t* ystaged = bars + 41;   // [4] V group: y of the block staged in its V buffer -> producer (TMA store)
+  uint64_t* ystaged = bars + 41;   // [4] V group: y of the block staged -> producer (TMA store)
+  uint64_t* emptyV = bars + 45;    // [4] MMA3 done -> producer (y staged in the Q buffer)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 39);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 39) + 1;
-  float* pw = reinterpret_cast<float*>(bars + 48);  // gamma^0 .. gamma^128
+  float* pw = reinterpret_cast<float*>(bars + 52);  // gamma^0 .. gamma^128
+  // y of a block is staged for its TMA store in a buffer that is dead after
+  // MMA3: the block's Q buffer when it holds a C x 128 bf16 tile (DK = 128),
+  // so that the V buffer can be reloaded as soon as MMA3 is done, else the
+  // block's V buffer.
+  constexpr bool kYinQ = DK >= 128;
+  const uint32_t y_box = kYinQ ? 16384u : (uint32_t)C * 128u;  // bytes between the two 64-column boxes of y
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int vt = blockIdx.x, bh = blockIdx.y, seg = blockIdx.z;
@@ -299,7 +306,10 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     mbar_init(ocross, 1);
     mbar_init(pready, 128);
     mbar_init(sready, 128);
-    for (int i = 0; i < 4; ++i) mbar_init(&ystaged[i], 128);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&ystaged[i], 128);
+      mbar_init(&emptyV[i], 1);
+    }
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -328,8 +338,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
     // Q, K, V of each block go to their own stage buffers with their own
-    // barriers, so each is reloaded as soon as its last reader is done:
-    // K after MMA5, Q after MMA4, V after MMA3 (the order they are issued in).
+    // barriers, so each is reloaded as soon as its last reader is done: K
+    // after MMA5, V after MMA3, and the buffer that stages y (Q or V) after
+    // the TMA stores of that y have read it.
     // The next block's tiles are prefetched into L2 as soon as this block's
     // loads are issued, so a reload waits on L2 rather than on DRAM.
     if (lane == 0 && nck > 0) {
@@ -358,24 +369,41 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           for (int b = 0; b < DK / 64; ++b)
             tma_load_3d(sK + s * sp.k_stage + b * C * 128, &mapK, &fullK[s], b * 64, t0, bh);
         }
-        if (it >= NS && !mbar_wait(&emptyQ[s], par, abort_flag, a.lim)) break;
-        mbar_arrive_expect_tx(&fullQ[s], qk_bytes);
-        for (int b = 0; b < DK / 64; ++b)
-          tma_load_3d(sQ + s * sp.q_stage + b * 16384, &mapQ, &fullQ[s], b * 64, t0, bh);
-        if (it >= NS) {
-          // the V buffer holds y of block it - NS (staged there after MMA3):
-          // store it with two TMA tensor stores, and reload the buffer once
-          // they have read it
-          if (!mbar_wait(&ystaged[s], par, abort_flag, a.lim)) break;
+        // The staging buffer of stage s holds y of block it - NS (staged after
+        // MMA3): store it with two TMA tensor stores, and reload the buffer
+        // once they have read it.
+        uint8_t* ys = kYinQ ? sQ + s * sp.q_stage : sV + s * sp.v_stage;
+        auto store_y = [&]() -> bool {
+          if (!mbar_wait(&ystaged[s], par, abort_flag, a.lim)) return false;
           const int ty = blk_t0(it - NS);
-          tma_store_3d(&mapY, sV + s * sp.v_stage, vt * kCW_DVT, ty, bh);
-          tma_store_3d(&mapY, sV + s * sp.v_stage + C * 128, vt * kCW_DVT + 64, ty, bh);
+          tma_store_3d(&mapY, ys, vt * kCW_DVT, ty, bh);
+          tma_store_3d(&mapY, ys + y_box, vt * kCW_DVT + 64, ty, bh);
           bulk_commit_group();
           bulk_wait_read_all();
+          return true;
+        };
+        auto load_q = [&]() {
+          mbar_arrive_expect_tx(&fullQ[s], qk_bytes);
+          for (int b = 0; b < DK / 64; ++b)
+            tma_load_3d(sQ + s * sp.q_stage + b * 16384, &mapQ, &fullQ[s], b * 64, t0, bh);
+        };
+        auto load_v = [&]() {
+          mbar_arrive_expect_tx(&fullV[s], v_bytes);
+          for (int b = 0; b < 2; ++b)
+            tma_load_3d(sV + s * sp.v_stage + b * C * 128, &mapV, &fullV[s], vt * kCW_DVT + b * 64, t0, bh);
+        };
+        if (kYinQ) {
+          // V after MMA3 of block it - NS; Q after y of that block left its buffer
+          if (it >= NS && !mbar_wait(&emptyV[s], par, abort_flag, a.lim)) break;
+          load_v();
+          if (it >= NS && !store_y()) break;
+          load_q();
+        } else {
+          if (it >= NS && !mbar_wait(&emptyQ[s], par, abort_flag, a.lim)) break;
+          load_q();
+          if (it >= NS && !store_y()) break;
+          load_v();
         }
-        mbar_arrive_expect_tx(&fullV[s], v_bytes);
-        for (int b = 0; b < 2; ++b)
-          tma_load_3d(sV + s * sp.v_stage + b * C * 128, &mapV, &fullV[s], vt * kCW_DVT + b * 64, t0, bh);
         issued = it + 1;
         if (it + NS < nck) {
           const int tp = blk_t0(it + NS);
@@ -390,9 +418,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       if (issued == nck) {
         for (int j = max(0, nck - NS); j < nck; ++j) {
           if (!mbar_wait(&ystaged[j % NS], (j / NS) & 1, abort_flag, a.lim)) break;
-          const uint8_t* ys = sV + (j % NS) * sp.v_stage;
+          const uint8_t* ys = kYinQ ? sQ + (j % NS) * sp.q_stage : sV + (j % NS) * sp.v_stage;
           tma_store_3d(&mapY, ys, vt * kCW_DVT, blk_t0(j), bh);
-          tma_store_3d(&mapY, ys + C * 128, vt * kCW_DVT + 64, blk_t0(j), bh);
+          tma_store_3d(&mapY, ys + y_box, vt * kCW_DVT + 64, blk_t0(j), bh);
           bulk_commit_group();
         }
       }
@@ -472,6 +500,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           mma_ts(t_o, tm + TM_P + kk * 8, bd, id3, 1);
         }
         mma_commit(&mma3done[ob]);
+        if (kYinQ) mma_commit(&emptyV[s]);
       }
       mma_commit(fin);
       mbar_drain(fin, 0, a.lim);
@@ -541,9 +570,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       if (it + 1 < nck && rescaled) rho_z = cw_rho_next(rho_z, pw[blk_len(it + 1)]);
       return true;
     };
-    // y = (gamma^(r+1-l) rho in the rescaled form) O, staged in the block's V
-    // buffer (dead after MMA3, not reloaded before the producer stored y out of
-    // it) for two TMA tensor stores by the producer.
+    // y = (gamma^(r+1-l) rho in the rescaled form) O, staged in the block's Q
+    // or V buffer (dead after MMA3, not reloaded before the producer stored y
+    // out of it) for two TMA tensor stores by the producer.
     auto y_step = [&](int it) -> bool {
       const int s = it % NS, ob = it & 1;
       if (!mbar_wait(&mma3done[ob], (it >> 1) & 1, abort_flag, a.lim)) return false;
@@ -553,7 +582,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       const int r = (int)t;
       const float yf = rescaled ? exp2f((float)(REV ? -r : r + 1 - l) * l2g) * rho_y : 1.f;
       if (it + 1 < nck && rescaled) rho_y = cw_rho_next(rho_y, pw[blk_len(it + 1)]);
-      uint8_t* ystage = sV + s * sp.v_stage;
+      uint8_t* ystage = kYinQ ? sQ + s * sp.q_stage : sV + s * sp.v_stage;
       const uint32_t t_o = tm + lane_off + TM_O + 128u * (uint32_t)ob;
 #pragma unroll
       for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
@@ -563,7 +592,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         float x[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) x[u] = yf * __uint_as_float(o[u]);
-        if (r < C) store_row32_sw128(ystage, (uint32_t)C * 128u, (uint32_t)r, (uint32_t)c0, x);
+        if (r < C) store_row32_sw128(ystage, y_box, (uint32_t)r, (uint32_t)c0, x);
       }
       tc_fence_before();
       mbar_arrive(&ofree[ob]);
