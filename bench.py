@@ -92,10 +92,16 @@ def load_peaks():
                 "source": "fallback (earlier measurement on this pool)"}
 
 
-# The headline kernel's source: chunkwise_tc.cuh up to the start of the
-# sequence-split helpers that follow chunkwise_tc256_kernel (everything the
-# kernel can use is declared above it), plus tc_common.cuh.
-HEADLINE_SOURCE_END = b"// Segment sums for the sequence split"
+# The headline kernel's source: in chunkwise_tc.cuh the shared helpers (from
+# the namespace opening to the dk <= 128 kernel) and chunkwise_tc256_kernel's
+# own section (up to the sequence-split helpers that follow it), plus
+# tc_common.cuh.  Comments outside those regions and the other kernels of the
+# file do not enter it.
+HEADLINE_SOURCE_REGIONS = (
+    (b"namespace ret {",
+     b"template <int DK, bool REV>\n__global__ void __launch_bounds__(kCW_MainThreads, 1)\nchunkwise_tc_kernel("),
+    (b"// dk = 256: one stage", b"// Segment sums for the sequence split"),
+)
 
 
 def kernel_source_digest():
@@ -104,8 +110,9 @@ def kernel_source_digest():
     d = os.path.join(ROOT, "retnet_retention_chunkwise_b200", "csrc")
     with open(os.path.join(d, "chunkwise_tc.cuh"), "rb") as fh:
         src = fh.read()
-    cut = src.find(HEADLINE_SOURCE_END)
-    h.update(src if cut < 0 else src[:cut])
+    for start, end in HEADLINE_SOURCE_REGIONS:
+        i, j = src.find(start), src.find(end)
+        h.update(src if i < 0 or j < i else src[i:j])  # a missing marker hashes the whole file
     with open(os.path.join(d, "tc_common.cuh"), "rb") as fh:
         h.update(fh.read())
     return h.hexdigest()[:16]
