@@ -85,6 +85,13 @@ struct CwArgs {
   const float* state_in;    // initial state when n_seg == 1 (may be null = zeros)
   float* state_out;         // may be null
   const float* seg_state;   // [BH][n_seg][dk][dv] initial states when n_seg > 1
+  // Anti-causal sums (REV) only, dk <= 128 kernel: when set (and seg_state is
+  // null), segment g starts from the transpose of the state in slot
+  // seg_tr_step * (g + 1) - 1 (the last segment: slot seg_tr_nseg - 1) of
+  // seg_tr, laid out [BH][seg_tr_nseg][dv][dk]: the scanned segment states of
+  // an anti-causal sum whose state is the transpose of this one.
+  const float* seg_tr;
+  int seg_tr_nseg, seg_tr_step;
   WaitLimit lim;
   int debug_drop_block;     // fault injection: block whose K load is never issued (-1 = none)
 };
@@ -623,8 +630,16 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       // the segment states come from the launches before this one on the
       // stream, which may still be running (programmatic dependent launch)
       if (a.n_seg > 1) griddep_wait();
-      const float* src = (a.n_seg > 1) ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv
+      const bool tr = REV && a.n_seg > 1 && a.seg_state == nullptr && a.seg_tr != nullptr;
+      const float* src = (a.n_seg > 1) ? (a.seg_state ? a.seg_state + ((size_t)bh * a.n_seg + seg) * dkdv : nullptr)
                                        : (a.state_in ? a.state_in + (size_t)bh * dkdv : nullptr);
+      // transposed source: row v of the [dv][dk] state, contiguous in d
+      const float* src_tr = nullptr;
+      if (tr) {
+        const int slot = (seg == a.n_seg - 1) ? a.seg_tr_nseg - 1 : a.seg_tr_step * (seg + 1) - 1;
+        if (RET_BC(slot >= 0 && slot < a.seg_tr_nseg && v < a.dv, 108))
+          src_tr = a.seg_tr + ((size_t)bh * a.seg_tr_nseg + slot) * dkdv + (size_t)v * DK;
+      }
       // rescaled: U = S_in (or gamma^l0 S_in when rho was reset), Sb = bf16(U);
       // direct: TMEM holds gamma^l0 S_in, Sb = S_in
       const float gu = (rho == 1.f) ? g0 : 1.f;
@@ -632,9 +647,20 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       for (int d0 = 0; d0 < DK; d0 += 32) {
         float x[32];
         uint32_t w[32];
+        if (tr) {
+#pragma unroll
+          for (int u = 0; u < 32; u += 4) {
+            const float4 f4 = src_tr ? *reinterpret_cast<const float4*>(src_tr + d0 + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            x[u] = f4.x, x[u + 1] = f4.y, x[u + 2] = f4.z, x[u + 3] = f4.w;
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            x[u] = (src && RET_BC(d0 + u < DK && v < a.dv, 104)) ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
+        }
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          const float sv = (src && RET_BC(d0 + u < DK && v < a.dv, 104)) ? src[(size_t)(d0 + u) * a.dv + v] : 0.f;
+          const float sv = x[u];
           x[u] = gc * sv;
           w[u] = __float_as_uint(gu * sv);
         }

@@ -199,12 +199,34 @@ size_t seg_workspace_bytes(const ret_shape& s, int n_seg) {
   return (size_t)s.B * s.H * n_seg * (size_t)s.dk * s.dv * sizeof(float);
 }
 
+// Sequence-split plan of one chunkwise call: n_seg segments of seg_chunks
+// blocks (the last may be shorter).
+struct SegPlan {
+  int n_seg, seg_chunks;
+};
+
+// Segment states taken from another anti-causal sum whose state is the
+// transpose of this one's (the two anti-causal sums of the backward pass):
+// its scanned workspace [BH][n_src][dv][dk], its segments `step` times
+// shorter than this call's (plan).
+struct SegReuse {
+  const float* src;
+  int n_src, step;
+  SegPlan plan;
+};
+
 // REV = true runs the anti-causal sum (see chunkwise_dir); blocks longer than
-// 128 rows have no anti-causal kernel.
+// 128 rows have no anti-causal kernel.  force: use this sequence-split plan
+// instead of the default one (still reduced if the workspace is short);
+// used: the plan run; reuse: no segment-sum pass of its own (dk <= 128
+// anti-causal kernel only).
 template <int DK, bool REV>
 ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, const float* gamma,
                                void* y, const float* state_in, float* state_out, int C,
-                               const ret_shape& s, void* ws, size_t ws_bytes, cudaStream_t st) {
+                               const ret_shape& s, void* ws, size_t ws_bytes, cudaStream_t st,
+                               const SegPlan* force = nullptr, SegPlan* used = nullptr,
+                               const SegReuse* reuse = nullptr) {
+  if (reuse && (!REV || DK > 128 || C > 128)) return RET_EINVAL;
   if (REV && C > 128) return RET_EUNSUPPORTED;
   const int BH = s.B * s.H;
   CUtensorMap mq, mk, mv, my;
@@ -232,7 +254,9 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
 
   int n_seg = 1, seg_chunks = 0;
   plan_segments(s, C, &n_seg, &seg_chunks);
-  while (n_seg > 1 && (ws == nullptr || seg_workspace_bytes(s, n_seg) > ws_bytes)) {
+  if (force) n_seg = force->n_seg, seg_chunks = force->seg_chunks;
+  if (reuse) n_seg = reuse->plan.n_seg, seg_chunks = reuse->plan.seg_chunks;
+  while (!reuse && n_seg > 1 && (ws == nullptr || seg_workspace_bytes(s, n_seg) > ws_bytes)) {
     // not enough workspace for this split: fall back to fewer segments
     const int n_chunks = (s.L + C - 1) / C;
     int g = n_seg - 1;
@@ -240,9 +264,11 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
     n_seg = (n_chunks + seg_chunks - 1) / seg_chunks;
   }
   if (n_seg <= 1) {
+    if (reuse) return RET_EINVAL;
     n_seg = 1;
     seg_chunks = (s.L + C - 1) / C;
   }
+  if (used) used->n_seg = n_seg, used->seg_chunks = seg_chunks;
 
   CwArgs a;
   a.B = s.B;
@@ -256,11 +282,14 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
   a.y = static_cast<__nv_bfloat16*>(y);
   a.state_in = state_in;
   a.state_out = state_out;
-  a.seg_state = static_cast<const float*>(ws);
+  a.seg_state = reuse ? nullptr : static_cast<const float*>(ws);
+  a.seg_tr = reuse ? reuse->src : nullptr;
+  a.seg_tr_nseg = reuse ? reuse->n_src : 0;
+  a.seg_tr_step = reuse ? reuse->step : 0;
   a.lim = wait_limit();
   a.debug_drop_block = debug_drop_block();
 
-  if (n_seg > 1) {
+  if (n_seg > 1 && !reuse) {
     // segment sums -> workspace slots 1..n_seg-1, then the scan fills every slot
     int ns2 = 0;
     const uint32_t per = (uint32_t)(DK / 64) * C * 128 + 2u * C * 128;
@@ -285,7 +314,7 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
                      s.H, DK * s.dv, n_seg, seg_chunks * C, s.L - (n_seg - 1) * seg_chunks * C, dec) != RET_OK)
       return RET_ECUDA;
   }
-  const bool after = n_seg > 1;
+  const bool after = n_seg > 1 && !reuse;
   dim3 grid(s.dv / kCW_DVT, BH, n_seg);
   if constexpr (DK == 256) {
     // one stage; scores and cross-block term fused into one wide MMA
@@ -531,7 +560,9 @@ ret_status parallel_dir(const void* q, const void* k, const void* v, const float
 template <bool REV>
 ret_status chunkwise_dir(const void* q, const void* k, const void* v, const float* gamma, void* y,
                          const float* state_in, float* state_out, int chunk, ret_shape s, ret_dtype dt,
-                         void* workspace, size_t workspace_bytes, cudaStream_t st) {
+                         void* workspace, size_t workspace_bytes, cudaStream_t st, const SegPlan* force = nullptr,
+                         SegPlan* used = nullptr, const SegReuse* reuse = nullptr) {
+  if (used) used->n_seg = 0, used->seg_chunks = 0;  // no split unless the tensor-core path reports one
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
   if ((rc = check_gamma(gamma, s.H)) != RET_OK) return rc;
@@ -572,9 +603,16 @@ ret_status chunkwise_dir(const void* q, const void* k, const void* v, const floa
     return launch_status();
   }
   switch (s.dk) {
-    case 64: return launch_chunkwise_tc<64, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
-    case 128: return launch_chunkwise_tc<128, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
-    default: return launch_chunkwise_tc<256, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace, workspace_bytes, st);
+    case 64:
+      return launch_chunkwise_tc<64, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace,
+                                          workspace_bytes, st, force, used, reuse);
+    case 128:
+      return launch_chunkwise_tc<128, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace,
+                                           workspace_bytes, st, force, used, reuse);
+    default:
+      if (reuse) return RET_EINVAL;
+      return launch_chunkwise_tc<256, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace,
+                                           workspace_bytes, st, force, used, nullptr);
   }
 }
 
@@ -1178,14 +1216,36 @@ ret_status retention_chunkwise_backward_state(const void* q, const void* k, cons
   if ((rc = chunkwise_dir<false>(dy, v, k, gamma, dq, state_in ? s0t : nullptr, nullptr, chunk, swapped, dt, sw,
                                  split, st)) != RET_OK)
     return rc;
+  // The two anti-causal sums carry transposed states (sum_n dy_n^T q_n and
+  // sum_n q_n^T dy_n, from (dS_out / gamma)^T and dS_out / gamma).  When both
+  // are split into segments, the dk sum runs with segments `step` times
+  // shorter than the dv sum's, and the dv sum starts each segment from the
+  // transpose of the dk sum's scanned state at the same token, with no
+  // segment-sum pass of its own.
+  SegPlan p3{}, p2{}, p2_used{};
+  int step = 0;
+  if (dt == RET_BF16 && s.dk <= 128) {
+    plan_segments(s, cr, &p3.n_seg, &p3.seg_chunks);
+    plan_segments(swapped, cr, &p2.n_seg, &p2.seg_chunks);
+    if (p3.n_seg > 1 && p2.n_seg >= p3.n_seg) {
+      for (step = p2.n_seg / p3.n_seg; step > 1 && p3.seg_chunks % step != 0; --step) {
+      }
+      const int n_chunks = (s.L + cr - 1) / cr;
+      p2.seg_chunks = p3.seg_chunks / step;
+      p2.n_seg = (n_chunks + p2.seg_chunks - 1) / p2.seg_chunks;
+      if (p2.n_seg <= 1) step = 0;
+    }
+  }
   // dk_m = sum_{n>=m} gamma^(n-m) (v_m . dy_n) q_n + gamma^(L-1-m) v_m dS_out^T:  anti-causal, state_in x2
   if ((rc = chunkwise_dir<true>(v, dy, q, gamma, dk, dstate_out ? x2 : nullptr, nullptr, cr, swapped, dt, sw, split,
-                                st)) != RET_OK)
+                                st, step ? &p2 : nullptr, &p2_used)) != RET_OK)
     return rc;
+  const bool reuse_ok = step > 0 && p2_used.n_seg == p2.n_seg && p2_used.seg_chunks == p2.seg_chunks;
+  const SegReuse reuse{static_cast<const float*>(sw), p2.n_seg, step, p3};
   // dv_m = sum_{n>=m} gamma^(n-m) (k_m . q_n) dy_n + gamma^(L-1-m) k_m dS_out:  anti-causal, state_in x3;
   // its state_out T = sum_n gamma^n q_n^T dy_n + gamma^(L-1) dS_out goes to x2 (dS0 = gamma T)
   if ((rc = chunkwise_dir<true>(k, q, dy, gamma, dv, dstate_out ? x3 : nullptr, dstate_in ? x2 : nullptr, cr, s, dt,
-                                sw, split, st)) != RET_OK)
+                                sw, split, st, nullptr, nullptr, reuse_ok ? &reuse : nullptr)) != RET_OK)
     return rc;
   if (dstate_out && any_small) {
     if (dt == RET_BF16)
