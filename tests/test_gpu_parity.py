@@ -515,3 +515,24 @@ def test_chunkwise_backward_state_chained_calls():
     for i in range(3):
         assert rel(torch.cat([g1[i], g2[i]], dim=2), ref[i]) <= 2e-2, i
     assert rel(g1[3], ref[3]) <= 2e-2
+
+
+def test_chunkwise_backward_state_reused_segment_states():
+    # 16 heads of dk 128, dv 256 over 2048 tokens in 64-row blocks: the dk sum
+    # runs 8 segments and the dv sum 4, each of the dv sum's segments starting
+    # from the transpose of the dk sum's scanned state at the same token.  dk_m
+    # and dv_m need only the tokens n >= m, so the oracle's backward of the
+    # window [512, 2048) (same dS_out) gives their exact rows there: rows of
+    # three segments whose initial states came from the dk sum.
+    B, H, L, dk, dv, C = 1, 16, 2048, 128, 256, 64
+    q, k, v, dy, s0, dso = _state_grad_inputs(torch.bfloat16, B, H, L, dk, dv, 77)
+    gam = inputs.multiscale_gammas(H)
+    qd, kd, vd, dyd, s0d, dsod = dev(q, k, v, dy, s0, dso)
+    _, dkk, dvv, _ = ret.chunkwise_backward_state(qd, kd, vd, gam, dyd, C, s0d, dsod)
+    assert ret.device_status() == 0
+    w0 = 512
+    for h in (0, 9):
+        sl = lambda t: t[:, h:h + 1, w0:]  # noqa: E731
+        _, dk_r, dv_r, _ = oracle.backward(sl(q), sl(k), sl(v), gam[h:h + 1], sl(dy), None, dso[:, h:h + 1])
+        assert rel(dkk[:, h:h + 1, w0:], dk_r) <= 2e-2, h
+        assert rel(dvv[:, h:h + 1, w0:], dv_r) <= 2e-2, h
