@@ -17,6 +17,9 @@ Also measured in the same run (same timing rules, reported under "forms"):
   chunkwise_backward_state_long_context -- the same with a carried state
                 (state_in, the gradient of state_out, the gradient of state_in);
   chunkwise_msr_core -- chunkwise C=64 on the same MSR-core shape;
+  chunkwise_gn_msr_core -- the same with the per-head GroupNorm fused into its
+                epilogue, beside the chunkwise call followed by the GroupNorm
+                kernel (two_kernel_ms);
   long_context_C{64,128,256} -- B=1, H=16, L=65536, dk=128, dv=256 as four
                 16384-token calls with the state carried in place;
   chunkwise_state_headline -- the state-only call (no y) on the headline shape;
@@ -456,6 +459,19 @@ def bench_small(ret, args, dist, peaks):
     out["chunkwise_msr_core"] = {"workload": "B2 H8 L2048 dk64 dv128 C64, L2 flushed",
                                  "tokens_per_s": dist.sum(w.B * w.L) / (t * 1e-3), "call_ms": round(t, 4),
                                  "hbm_frac": round(nb / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    per, _ = time_calls(lambda: ret.chunkwise_groupnorm(q, k, v, gam, w.chunk, 1e-5, out=y, return_state=False),
+                        n, max(args.warmup, 3), dist, flush=True)
+    t_f = dist.max(statistics.median(per))
+
+    def two_calls():
+        ret.chunkwise(q, k, v, gam, w.chunk, out=y, return_state=False)
+        ret.groupnorm(y, 1e-5, out=y)
+    per, _ = time_calls(two_calls, n, max(args.warmup, 3), dist, flush=True)
+    t_2 = dist.max(statistics.median(per))
+    out["chunkwise_gn_msr_core"] = {"workload": "B2 H8 L2048 dk64 dv128 C64 + GroupNorm, L2 flushed",
+                                    "tokens_per_s": dist.sum(w.B * w.L) / (t_f * 1e-3),
+                                    "call_ms": round(t_f, 4), "two_kernel_ms": round(t_2, 4),
+                                    "hbm_frac": round(nb / (t_f * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
     del q, k, v, y
     w = inputs.WORKLOADS["long_context_bf16"]
     q, k, v = gpu_qkv(w.B, w.H, w.L, w.dk, w.dv, seed=0)

@@ -265,7 +265,11 @@ RET_API ret_status retention_groupnorm_gated(const void* y, const void* gate, vo
 /*
  * Chunkwise form followed by retention_groupnorm on its output, in place: y
  * receives the normalised output.  The other arguments are as for
- * retention_chunkwise; the normalisation runs as a second kernel on the stream.
+ * retention_chunkwise.  With bf16, dv = 128 (one head = one 128-column slice),
+ * dk <= 128, chunk <= 128 and weight and bias 16-byte aligned (or NULL) the
+ * chunkwise kernel normalises each row in its epilogue, before y is stored
+ * (one launch, no extra pass over y); otherwise the normalisation runs as a
+ * second kernel on the stream.
  */
 RET_API ret_status retention_chunkwise_gn(const void* q, const void* k, const void* v, const float* gamma,
                                           void* y, const float* state_in, float* state_out, int chunk,
@@ -278,7 +282,8 @@ RET_API size_t retention_chunkwise_gn_workspace_bytes(int chunk, ret_shape s, re
 
 /*
  * retention_chunkwise_gn with the output gate: y receives
- * GroupNorm(y) * act(gate) (see retention_groupnorm_gated), in place.  gate:
+ * GroupNorm(y) * act(gate) (see retention_groupnorm_gated), in place; with a
+ * gate the normalisation and gate always run as a second kernel.  gate:
  * device [B][H][L][dv] in the call's dtype, 16-byte aligned, sharing no byte
  * with y (RET_EINVAL otherwise: y is normalised in place while the gate is
  * read); NULL for no gate.  act: a ret_gate_act.  Workspace:

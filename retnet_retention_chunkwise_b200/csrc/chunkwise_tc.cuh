@@ -92,6 +92,13 @@ struct CwArgs {
   // an anti-causal sum whose state is the transpose of this one.
   const float* seg_tr;
   int seg_tr_nseg, seg_tr_step;
+  // Causal dk <= 128 kernel with one 128-column dv slice per head, built
+  // with GN: the per-head group normalisation of each y row in the epilogue,
+  // before the store, with eps and the optional per-channel weight and bias
+  // [H][dv].
+  float gn_eps;
+  const float* gn_w;
+  const float* gn_b;
   WaitLimit lim;
   int debug_drop_block;     // fault injection: block whose K load is never issued (-1 = none)
 };
@@ -230,7 +237,7 @@ __device__ __forceinline__ float cw_rho_first(bool rescaled, float g0) {
   return (rescaled && g0 >= 0x1p-64f) ? g0 : 1.f;
 }
 
-template <int DK, bool REV>
+template <int DK, bool REV, bool GN = false>
 __global__ void __launch_bounds__(kCW_MainThreads, 1)
 chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapY,
@@ -591,14 +598,65 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       if (it + 1 < nck && rescaled) rho_y = cw_rho_next(rho_y, pw[blk_len(it + 1)]);
       uint8_t* ystage = kYinQ ? sQ + s * sp.q_stage : sV + s * sp.v_stage;
       const uint32_t t_o = tm + lane_off + TM_O + 128u * (uint32_t)ob;
+      // Group normalisation of the row (the head's whole dv), with y = yf * o
+      // for the accumulator row o: the mean and biased variance of o from
+      // one pass over the row in TMEM (sums shifted by the row's first value,
+      // eight partial sums to keep the dependent chains short), scaled by yf;
+      // then z = o * (yf rstd) - mean rstd in the second pass.
+      float gn_a = 1.f, gn_b = 0.f;
+      if constexpr (GN) {
+        float sh = 0.f, s1[8], s2[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s1[j] = 0.f, s2[j] = 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c0, o);
+          tmem_ld_wait();
+          if (c0 == 0) sh = __uint_as_float(o[0]);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const float d = __uint_as_float(o[u]) - sh;
+            s1[u & 7] += d;
+            s2[u & 7] = fmaf(d, d, s2[u & 7]);
+          }
+        }
+#pragma unroll
+        for (int j = 1; j < 8; ++j) s1[0] += s1[j], s2[0] += s2[j];
+        const float m1 = s1[0] * (1.f / kCW_DVT);
+        const float var = fmaxf(s2[0] * (1.f / kCW_DVT) - m1 * m1, 0.f) * (yf * yf);
+        const float rstd = rsqrtf(var + a.gn_eps);
+        gn_a = yf * rstd;
+        gn_b = -(sh + m1) * gn_a;
+      }
 #pragma unroll
       for (int c0 = 0; c0 < kCW_DVT; c0 += 32) {
         uint32_t o[32];
         tmem_ld32(t_o + c0, o);
         tmem_ld_wait();
         float x[32];
+        if constexpr (GN) {
 #pragma unroll
-        for (int u = 0; u < 32; ++u) x[u] = yf * __uint_as_float(o[u]);
+          for (int u = 0; u < 32; ++u) x[u] = fmaf(__uint_as_float(o[u]), gn_a, gn_b);
+          const int ch = (bh % a.H) * kCW_DVT + c0;  // this head's channels
+          if (a.gn_w) {
+#pragma unroll
+            for (int u = 0; u < 32; u += 4) {
+              const float4 w4 = __ldg(reinterpret_cast<const float4*>(a.gn_w + ch + u));
+              x[u] *= w4.x, x[u + 1] *= w4.y, x[u + 2] *= w4.z, x[u + 3] *= w4.w;
+            }
+          }
+          if (a.gn_b) {
+#pragma unroll
+            for (int u = 0; u < 32; u += 4) {
+              const float4 b4 = __ldg(reinterpret_cast<const float4*>(a.gn_b + ch + u));
+              x[u] += b4.x, x[u + 1] += b4.y, x[u + 2] += b4.z, x[u + 3] += b4.w;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) x[u] = yf * __uint_as_float(o[u]);
+        }
         if (r < C) store_row32_sw128(ystage, y_box, (uint32_t)r, (uint32_t)c0, x);
       }
       tc_fence_before();

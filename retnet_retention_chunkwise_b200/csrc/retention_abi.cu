@@ -215,8 +215,16 @@ struct SegReuse {
   SegPlan plan;
 };
 
+// Group normalisation in the chunkwise epilogue (see CwArgs::gn).
+struct GnParams {
+  float eps;
+  const float* weight;
+  const float* bias;
+};
+
 // REV = true runs the anti-causal sum (see chunkwise_dir); blocks longer than
-// 128 rows have no anti-causal kernel.  force: use this sequence-split plan
+// 128 rows have no anti-causal kernel.  gn: normalise y in the epilogue (the
+// causal dk <= 128 kernel with one dv slice per head).  force: use this sequence-split plan
 // instead of the default one (still reduced if the workspace is short);
 // used: the plan run; reuse: no segment-sum pass of its own (dk <= 128
 // anti-causal kernel only).
@@ -225,8 +233,9 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
                                void* y, const float* state_in, float* state_out, int C,
                                const ret_shape& s, void* ws, size_t ws_bytes, cudaStream_t st,
                                const SegPlan* force = nullptr, SegPlan* used = nullptr,
-                               const SegReuse* reuse = nullptr) {
+                               const SegReuse* reuse = nullptr, const GnParams* gn = nullptr) {
   if (reuse && (!REV || DK > 128 || C > 128)) return RET_EINVAL;
+  if (gn && (REV || DK > 128 || C > 128 || s.dv != kCW_DVT)) return RET_EUNSUPPORTED;
   if (REV && C > 128) return RET_EUNSUPPORTED;
   const int BH = s.B * s.H;
   CUtensorMap mq, mk, mv, my;
@@ -286,6 +295,9 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
   a.seg_tr = reuse ? reuse->src : nullptr;
   a.seg_tr_nseg = reuse ? reuse->n_src : 0;
   a.seg_tr_step = reuse ? reuse->step : 0;
+  a.gn_eps = gn ? gn->eps : 0.f;
+  a.gn_w = gn ? gn->weight : nullptr;
+  a.gn_b = gn ? gn->bias : nullptr;
   a.lim = wait_limit();
   a.debug_drop_block = debug_drop_block();
 
@@ -339,12 +351,13 @@ ret_status launch_chunkwise_tc(const void* q, const void* k, const void* v, cons
       chunkwise_wide_kernel<DK><<<grid, kCW_MainThreads, pw.total, st>>>(mq, mk, mv, a, dec);
       return launch_status();
     }
-    if (cudaFuncSetAttribute(chunkwise_tc_kernel<DK, REV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)plan.total) != cudaSuccess)
+    // the normalising epilogue is its own instance, so the plain kernels keep
+    // their register allocation
+    auto* kern = gn ? chunkwise_tc_kernel<DK, false, true> : chunkwise_tc_kernel<DK, REV>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.total) != cudaSuccess)
       return RET_ECUDA;
-    if (after) return launch_after(chunkwise_tc_kernel<DK, REV>, grid, dim3(kCW_MainThreads), plan.total, st, mq,
-                                   mk, mv, my, a, dec);
-    chunkwise_tc_kernel<DK, REV><<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, my, a, dec);
+    if (after) return launch_after(kern, grid, dim3(kCW_MainThreads), plan.total, st, mq, mk, mv, my, a, dec);
+    kern<<<grid, kCW_MainThreads, plan.total, st>>>(mq, mk, mv, my, a, dec);
     return launch_status();
   }
 }
@@ -561,7 +574,7 @@ template <bool REV>
 ret_status chunkwise_dir(const void* q, const void* k, const void* v, const float* gamma, void* y,
                          const float* state_in, float* state_out, int chunk, ret_shape s, ret_dtype dt,
                          void* workspace, size_t workspace_bytes, cudaStream_t st, const SegPlan* force = nullptr,
-                         SegPlan* used = nullptr, const SegReuse* reuse = nullptr) {
+                         SegPlan* used = nullptr, const SegReuse* reuse = nullptr, const GnParams* gn = nullptr) {
   if (used) used->n_seg = 0, used->seg_chunks = 0;  // no split unless the tensor-core path reports one
   ret_status rc = check_shape(s, true);
   if (rc != RET_OK) return rc;
@@ -588,6 +601,7 @@ ret_status chunkwise_dir(const void* q, const void* k, const void* v, const floa
                              : cudaMemsetAsync(state_out, 0, sbytes, st);
     return e == cudaSuccess ? RET_OK : RET_ECUDA;
   }
+  if (gn && (dt != RET_BF16 || s.dk > 128)) return RET_EUNSUPPORTED;
   if (dt == RET_F32) {
     static HeadLog2 hl;
     static std::mutex mu;
@@ -605,10 +619,10 @@ ret_status chunkwise_dir(const void* q, const void* k, const void* v, const floa
   switch (s.dk) {
     case 64:
       return launch_chunkwise_tc<64, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace,
-                                          workspace_bytes, st, force, used, reuse);
+                                          workspace_bytes, st, force, used, reuse, gn);
     case 128:
       return launch_chunkwise_tc<128, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace,
-                                           workspace_bytes, st, force, used, reuse);
+                                           workspace_bytes, st, force, used, reuse, gn);
     default:
       if (reuse) return RET_EINVAL;
       return launch_chunkwise_tc<256, REV>(q, k, v, gamma, y, state_in, state_out, chunk, s, workspace,
@@ -1062,6 +1076,16 @@ ret_status retention_chunkwise_gn_gated(const void* q, const void* k, const void
     const size_t bytes = (size_t)s.B * s.H * s.L * s.dv * (dt == RET_BF16 ? 2 : 4);
     const uintptr_t g0 = reinterpret_cast<uintptr_t>(gate), y0 = reinterpret_cast<uintptr_t>(y);
     if (!aligned16(gate) || (g0 < y0 + bytes && y0 < g0 + bytes)) return RET_EINVAL;
+  }
+  // One dv slice per head (dv = 128), bf16, dk <= 128, blocks of at most 128
+  // rows, no gate, weight and bias 16-byte aligned (read as float4): the
+  // chunkwise kernel normalises each row before it stores y (one kernel).
+  // Otherwise the normalisation (and the gate) run as a second kernel over y.
+  if (!gate && (!weight || aligned16(weight)) && (!bias || aligned16(bias)) && dt == RET_BF16 && s.dv == kCW_DVT && s.dk <= 128 && chunk >= 16 && chunk <= 128 && s.L > 0 &&
+      tc_chunk_ok(chunk, s.dk) && tc_shape_ok(s) && check_shape(s, true) == RET_OK) {
+    const GnParams gn{eps, weight, bias};
+    return chunkwise_dir<false>(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, workspace, workspace_bytes,
+                                static_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr, &gn);
   }
   ret_status rc = retention_chunkwise(q, k, v, gamma, y, state_in, state_out, chunk, s, dt, workspace,
                                       workspace_bytes, stream);

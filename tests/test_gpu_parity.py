@@ -536,3 +536,28 @@ def test_chunkwise_backward_state_reused_segment_states():
         _, dk_r, dv_r, _ = oracle.backward(sl(q), sl(k), sl(v), gam[h:h + 1], sl(dy), None, dso[:, h:h + 1])
         assert rel(dkk[:, h:h + 1, w0:], dk_r) <= 2e-2, h
         assert rel(dvv[:, h:h + 1, w0:], dv_r) <= 2e-2, h
+
+
+@pytest.mark.parametrize("B,H,L,dk,C,affine,gammas", [
+    (2, 8, 2048, 64, 64, False, None),            # the MSR core, sequence split
+    (1, 3, 1000, 128, 128, True, None),           # ragged tail, weight and bias
+    (1, 2, 77, 64, 16, True, [0.5, 0.01]),        # gamma 0.01: the direct form; short blocks
+])
+def test_chunkwise_groupnorm_fused_epilogue(B, H, L, dk, C, affine, gammas):
+    # dv = 128: one dv slice per head, so the chunkwise kernel normalises each
+    # y row in its epilogue before the store (no second kernel); normalised
+    # rows share one scale, so one relative bound covers every head
+    dv = 128
+    q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed=L + 21)
+    gam = inputs.multiscale_gammas(H) if gammas is None else torch.tensor(gammas)
+    s_in = inputs.state(B, H, dk, dv, seed=22, scale=0.5)
+    g = torch.Generator("cpu").manual_seed(23)
+    w = torch.rand(H * dv, generator=g) + 0.5 if affine else None
+    b = torch.randn(H * dv, generator=g) * 0.1 if affine else None
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam, s_in)
+    z_ref = oracle.groupnorm(y_ref, eps=1e-5, weight=w, bias=b)
+    qd, kd, vd, sd = dev(q, k, v, s_in)
+    z, s = ret.chunkwise_groupnorm(qd, kd, vd, gam, C, 1e-5, weight=None if w is None else w.cuda(),
+                                   bias=None if b is None else b.cuda(), state_in=sd)
+    assert ret.device_status() == 0
+    assert rel(z, z_ref) <= 2e-2 and rel(s, s_ref) <= 2e-2
