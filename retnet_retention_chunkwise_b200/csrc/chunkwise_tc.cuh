@@ -138,15 +138,17 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, WaitL
 
 // Scale the 128-byte row r of a 128B-swizzled bf16 tile in place by f.
 __device__ __forceinline__ void scale_row_sw128(uint8_t* tile, uint32_t r, float f) {
+  // all eight loads first, so the row costs one shared-memory round trip
+  uint4 w[8];
+#pragma unroll
+  for (uint32_t c = 0; c < 8; ++c) w[c] = *reinterpret_cast<const uint4*>(tile + sw128_off(r, c));
 #pragma unroll
   for (uint32_t c = 0; c < 8; ++c) {
-    uint4* p = reinterpret_cast<uint4*>(tile + sw128_off(r, c));
-    uint4 w = *p;
-    w.x = pack_bf16x2(bf16lo_to_f32(w.x) * f, bf16hi_to_f32(w.x) * f);
-    w.y = pack_bf16x2(bf16lo_to_f32(w.y) * f, bf16hi_to_f32(w.y) * f);
-    w.z = pack_bf16x2(bf16lo_to_f32(w.z) * f, bf16hi_to_f32(w.z) * f);
-    w.w = pack_bf16x2(bf16lo_to_f32(w.w) * f, bf16hi_to_f32(w.w) * f);
-    *p = w;
+    w[c].x = pack_bf16x2(bf16lo_to_f32(w[c].x) * f, bf16hi_to_f32(w[c].x) * f);
+    w[c].y = pack_bf16x2(bf16lo_to_f32(w[c].y) * f, bf16hi_to_f32(w[c].y) * f);
+    w[c].z = pack_bf16x2(bf16lo_to_f32(w[c].z) * f, bf16hi_to_f32(w[c].z) * f);
+    w[c].w = pack_bf16x2(bf16lo_to_f32(w[c].w) * f, bf16hi_to_f32(w[c].w) * f);
+    *reinterpret_cast<uint4*>(tile + sw128_off(r, c)) = w[c];
   }
 }
 
@@ -263,7 +265,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   uint64_t* fullV = bars + 8;      // [4] TMA -> V group, MMA
   uint64_t* emptyQ = bars + 12;    // [4] MMA4 done -> producer
   uint64_t* emptyK = bars + 16;    // [4] MMA5 done -> producer
-  uint64_t* zready = bars + 24;    // [4] V group: scaled V of stage s written -> MMA5 (and MMA3)
+  uint64_t* zready = bars + 24;    // [4] V group: scaled V (K) of stage s written -> MMA5 (MMA1)
   uint64_t* pfull = bars + 28;     // MMA1 done -> P/O group
   uint64_t* mma3done = bars + 30;  // [2] per O buffer: MMA3 done -> V group (y)
   uint64_t* ocross = bars + 32;    // MMA5 + MMA4 done -> P/O group, S group
@@ -281,6 +283,11 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   // so that the V buffer can be reloaded as soon as MMA3 is done, else the
   // block's V buffer.
   constexpr bool kYinQ = DK >= 128;
+  // Rescaled form at dk = 64: zeta / rho goes on the rows of K (half the bytes
+  // of V's rows) as soon as K lands, before MMA1, so that P = Q (zeta K)^T
+  // carries it into P~ V and V stays as loaded; MMA5 takes V and zeta K.
+  // Elsewhere it goes on V's rows.
+  constexpr bool kZetaK = DK == 64;
   const uint32_t y_box = kYinQ ? 16384u : (uint32_t)C * 128u;  // bytes between the two 64-column boxes of y
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -289,6 +296,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   // Rescaled form (see the file header) when gamma^(C-1) >= 2^-64; else the
   // direct form.  Uniform over the CTA (one head).
   const bool rescaled = (float)(C - 1) * l2g >= -64.f;
+  const bool zeta_k = kZetaK && rescaled;
   const int n_total = (a.L + C - 1) / C;
   const int c_begin = seg * a.seg_chunks;
   const int c_end = min(c_begin + a.seg_chunks, n_total);
@@ -465,6 +473,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         const uint32_t t_o = tm + TM_O + 128u * (uint32_t)ob;
         if (!mbar_wait(&fullK[s], par, abort_flag, a.lim)) break;
         if (!mbar_wait(&fullQ[s], par, abort_flag, a.lim)) break;
+        if (zeta_k && !mbar_wait(&zready[s], par, abort_flag, a.lim)) break;
         RET_TRACE_STAMP(cta_id, it, 1);
         tc_fence_after();
         const uint32_t q_s = aQ + s * sp.q_stage, k_s = aK + s * sp.k_stage, v_s = aV + s * sp.v_stage;
@@ -477,12 +486,15 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         }
         mma_commit(pfull);
         // MMA5: S^T += (zeta V)^T K, onto the state already rescaled by gamma^l.
-        // Rescaled form: zeta V is the V tile itself (scaled in place), read
-        // MN-major from shared memory.  Direct form: (zeta V)^T was built in the
-        // columns of this block's (free) O buffer.
+        // Rescaled form: zeta sits on the V tile (or on the K tile at dk = 64)
+        // in place, V read MN-major from shared memory.  Direct form:
+        // (zeta V)^T was built in the columns of this block's (free) O buffer.
         // zready is per stage: in the rescaled form the V group runs ahead by up
         // to NS blocks, so one barrier could complete two phases unobserved.
-        if (!mbar_wait(&zready[s], par, abort_flag, a.lim)) break;
+        if (!zeta_k && !mbar_wait(&zready[s], par, abort_flag, a.lim)) break;
+        // with zeta on K nothing else has waited for this block's V tile: MMA5
+        // and MMA3 read it, so wait for its load here
+        if (zeta_k && !mbar_wait(&fullV[s], par, abort_flag, a.lim)) break;
         if (!mbar_wait(sready, it & 1, abort_flag, a.lim)) break;
         RET_TRACE_STAMP(cta_id, it, 2);
         tc_fence_after();
@@ -496,6 +508,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         mma_commit(&emptyK[s]);
         // MMA4: O = Q S_copy into buffer ob, once y of block it - 2 left it
         if (!mbar_wait(&ofree[ob], (it >> 1) & 1, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, it, 11);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
@@ -534,15 +547,38 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     mbar_arrive(&ofree[1]);
     auto zeta_step = [&](int it) -> bool {
       const int s = it % NS;
-      if (!mbar_wait(&fullV[s], (it / NS) & 1, abort_flag, a.lim)) return false;
+      if (!mbar_wait(zeta_k ? &fullK[s] : &fullV[s], (it / NS) & 1, abort_flag, a.lim)) return false;
+      if (t == 0) RET_TRACE_STAMP(cta_id, it, 13);
       const int l = min(C, a.L - blk_t0(it));
       uint8_t* vs = sV + s * sp.v_stage;
-      if (rescaled) {
-        // row j of the V tile scaled in place by zeta_j = gamma^(l-1-j) (0 past the end)
-        if ((int)t < C && RET_BC(s < NS, 105)) {
-          const float zs = (((int)t < l) ? pw[REV ? (int)t : l - 1 - (int)t] : 0.f) * __frcp_rn(rho_z);  // zeta / rho
-          scale_row_sw128(vs, t, zs);
-          scale_row_sw128(vs + C * 128, t, zs);
+      if (zeta_k) {
+        // row j of the K tile (one 64-column box) scaled in place by zeta_j / rho
+        const float rinv = __frcp_rn(rho_z);
+        if (RET_BC(s < NS, 105)) {
+          for (int j = (int)t; j < C; j += 128) {
+            const float zs = ((j < l) ? pw[REV ? j : l - 1 - j] : 0.f) * rinv;
+            scale_row_sw128(sK + s * sp.k_stage, (uint32_t)j, zs);
+          }
+        }
+        fence_proxy_async_smem();
+      } else if (rescaled) {
+        // row j of the V tile scaled in place by zeta_j = gamma^(l-1-j) (0 past
+        // the end), divided by rho.  C = 128: thread t takes both 64-column
+        // boxes of row t, one after the other (sixteen loads in flight were
+        // slower); shorter blocks spread (row, box) over all threads.
+        const float rinv = __frcp_rn(rho_z);
+        if (RET_BC(s < NS, 105)) {
+          if (C == 128) {
+            const float zs = (((int)t < l) ? pw[REV ? (int)t : l - 1 - (int)t] : 0.f) * rinv;
+            scale_row_sw128(vs, t, zs);
+            scale_row_sw128(vs + C * 128, t, zs);
+          } else {
+            for (int w = (int)t; w < 2 * C; w += 128) {
+              const int j = w % C;
+              const float zs = ((j < l) ? pw[REV ? j : l - 1 - j] : 0.f) * rinv;
+              scale_row_sw128(vs + (w / C) * C * 128, (uint32_t)j, zs);
+            }
+          }
         }
         fence_proxy_async_smem();
       } else {
@@ -790,6 +826,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       const int t0 = blk_t0(it);
       const int l = min(C, a.L - t0);
       if (!mbar_wait(pfull, it & 1, abort_flag, a.lim)) break;
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 12);
       (void)RET_BC(l >= 1 && l <= C && t0 >= 0 && t0 < a.L, 107);
       tc_fence_after();
       // P -> P~ in place (two bf16 per column).  Rows past the block end read

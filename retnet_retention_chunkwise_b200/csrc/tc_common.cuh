@@ -45,8 +45,9 @@ __device__ __forceinline__ bool bc_ok(bool ok, unsigned int site) {
 #define RET_BC(cond, site) (true)
 #endif
 
-// Optional event trace (builds with -DRET_TRACE only): %globaltimer stamps per
-// (CTA, block, event) written to a caller-provided buffer.  RET_TRACE_INIT reads
+// Optional event trace (builds with -DRET_TRACE only): %clock64 stamps (SM
+// cycles; compare stamps of one CTA only) per (CTA, block, event) written to a
+// caller-provided buffer.  RET_TRACE_INIT reads
 // the buffer description once into registers; the stamps are plain stores.
 // Both compile to nothing in the normal build.
 #ifdef RET_TRACE
@@ -61,7 +62,7 @@ __device__ int g_trace_blocks = 0;   // block slots per CTA
   do {                                                                                     \
     if (trace_buf_ && (it) < trace_bl_ && (ev) < trace_ev_) {                              \
       unsigned long long t_;                                                               \
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                             \
+      asm volatile("mov.u64 %0, %%clock64;" : "=l"(t_));                             \
       trace_buf_[((size_t)(cta) * trace_bl_ + (it)) * trace_ev_ + (ev)] = t_;              \
     }                                                                                      \
   } while (0)

@@ -561,3 +561,30 @@ def test_chunkwise_groupnorm_fused_epilogue(B, H, L, dk, C, affine, gammas):
                                    bias=None if b is None else b.cuda(), state_in=sd)
     assert ret.device_status() == 0
     assert rel(z, z_ref) <= 2e-2 and rel(s, s_ref) <= 2e-2
+
+
+@pytest.mark.parametrize("B,H,L,dk,dv,C", [
+    (2, 8, 2048, 64, 128, 64),     # MSR core: sequence split, zeta on K's rows
+    (8, 16, 1024, 64, 128, 64),    # 128 CTAs, no split
+    (1, 4, 4096, 128, 256, 128),   # dk = 128, two dv slices, split
+    (2, 4, 1024, 256, 512, 128),   # dk = 256 kernel
+])
+def test_chunkwise_cold_cache_repeatable(B, H, L, dk, dv, C):
+    # Every call starts with q, k, v evicted from L2 (a 256 MB write), so the
+    # first blocks' tiles arrive from DRAM as late as they can: an operand read
+    # before its load has landed shows up as calls that differ from one another
+    # or from the oracle.
+    q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed=31)
+    gam = inputs.multiscale_gammas(H)
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam)
+    qd, kd, vd = dev(q, k, v)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    outs = []
+    for _ in range(4):
+        flush.fill_(1.0)
+        outs.append(ret.chunkwise(qd, kd, vd, gam, C))
+    torch.cuda.synchronize()
+    assert ret.device_status() == 0
+    for y, s in outs[1:]:
+        assert torch.equal(y, outs[0][0]) and torch.equal(s, outs[0][1])
+    assert rel(outs[0][0], y_ref) <= 2e-2 and rel(outs[0][1], s_ref) <= 2e-2
