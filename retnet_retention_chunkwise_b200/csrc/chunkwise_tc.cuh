@@ -485,6 +485,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
           mma_ss(tm + TM_P, ad, bd, id1, kk > 0);
         }
         mma_commit(pfull);
+        RET_TRACE_STAMP(cta_id, it, 14);
         // MMA5: S^T += (zeta V)^T K, onto the state already rescaled by gamma^l.
         // Rescaled form: zeta sits on the V tile (or on the K tile at dk = 64)
         // in place, V read MN-major from shared memory.  Direct form:
@@ -528,6 +529,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         }
         mma_commit(&mma3done[ob]);
         if (kYinQ) mma_commit(&emptyV[s]);
+        RET_TRACE_STAMP(cta_id, it, 15);
       }
       mma_commit(fin);
       mbar_drain(fin, 0, a.lim);
@@ -1077,6 +1079,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         }
         mma_commit(pxfull);
         mma_commit(emptyQ);
+        RET_TRACE_STAMP(cta_id, it, 12);
         // MMA5: S^T += (zeta V)^T K  (rescaled: zeta on V; direct: zeta on K)
         if (!mbar_wait(zready, par, abort_flag, a.lim)) break;
         RET_TRACE_STAMP(cta_id, it, 2);
@@ -1088,6 +1091,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         }
         mma_commit(mma5done);
         mma_commit(emptyK);
+        RET_TRACE_STAMP(cta_id, it, 13);
         // MMA3: X += P~ V
         if (!mbar_wait(pready, par, abort_flag, a.lim)) break;
         RET_TRACE_STAMP(cta_id, it, 4);
@@ -1098,6 +1102,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
         }
         mma_commit(mma3done);
         mma_commit(emptyV);
+        RET_TRACE_STAMP(cta_id, it, 14);
       }
       mma_commit(fin);
       mbar_drain(fin, 0, a.lim);
