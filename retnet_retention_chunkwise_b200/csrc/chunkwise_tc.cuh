@@ -471,9 +471,9 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         const int s = it % NS, ob = it & 1;
         const uint32_t par = (it / NS) & 1;
         const uint32_t t_o = tm + TM_O + 128u * (uint32_t)ob;
-        if (!mbar_wait(&fullK[s], par, abort_flag, a.lim)) break;
-        if (!mbar_wait(&fullQ[s], par, abort_flag, a.lim)) break;
-        if (zeta_k && !mbar_wait(&zready[s], par, abort_flag, a.lim)) break;
+        if (!mbar_wait4(&fullK[s], par, &fullQ[s], par, zeta_k ? &zready[s] : &fullQ[s], par, &fullQ[s], par,
+                        abort_flag, a.lim))
+          break;
         RET_TRACE_STAMP(cta_id, it, 1);
         tc_fence_after();
         const uint32_t q_s = aQ + s * sp.q_stage, k_s = aK + s * sp.k_stage, v_s = aV + s * sp.v_stage;
@@ -492,11 +492,12 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         // (zeta V)^T was built in the columns of this block's (free) O buffer.
         // zready is per stage: in the rescaled form the V group runs ahead by up
         // to NS blocks, so one barrier could complete two phases unobserved.
-        if (!zeta_k && !mbar_wait(&zready[s], par, abort_flag, a.lim)) break;
-        // with zeta on K nothing else has waited for this block's V tile: MMA5
-        // and MMA3 read it, so wait for its load here
-        if (zeta_k && !mbar_wait(&fullV[s], par, abort_flag, a.lim)) break;
-        if (!mbar_wait(sready, it & 1, abort_flag, a.lim)) break;
+        // (with zeta on K nothing else has waited for this block's V tile: MMA5
+        // and MMA3 read it, so wait for its load here).  The wait for MMA4's O
+        // buffer (y of block it - 2 read out of it) goes with these.
+        if (!mbar_wait4(zeta_k ? &fullV[s] : &zready[s], par, sready, it & 1, &ofree[ob], (it >> 1) & 1, sready,
+                        it & 1, abort_flag, a.lim))
+          break;
         RET_TRACE_STAMP(cta_id, it, 2);
         tc_fence_after();
         for (int kk = 0; kk < C / 16; ++kk) {
@@ -507,8 +508,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
             mma_ts(tm + TM_S, t_o + kk * 8, bd, id5, 1);
         }
         mma_commit(&emptyK[s]);
-        // MMA4: O = Q S_copy into buffer ob, once y of block it - 2 left it
-        if (!mbar_wait(&ofree[ob], (it >> 1) & 1, abort_flag, a.lim)) break;
+        // MMA4: O = Q S_copy into buffer ob (y of block it - 2 has left it)
         RET_TRACE_STAMP(cta_id, it, 11);
         tc_fence_after();
 #pragma unroll
@@ -1064,10 +1064,7 @@ chunkwise_tc256_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_co
       const uint32_t aQ = smem_u32(sQ), aKS = smem_u32(sKS), aV = smem_u32(sV);
       for (int it = 0; it < nck; ++it) {
         const uint32_t par = it & 1;
-        if (!mbar_wait(fullQ, par, abort_flag, a.lim)) break;
-        if (!mbar_wait(fullK, par, abort_flag, a.lim)) break;
-        if (!mbar_wait(sready, par, abort_flag, a.lim)) break;
-        if (!mbar_wait(ofree, par, abort_flag, a.lim)) break;
+        if (!mbar_wait4(fullQ, par, fullK, par, sready, par, ofree, par, abort_flag, a.lim)) break;
         RET_TRACE_STAMP(cta_id, it, 1);
         tc_fence_after();
         // MMA14: [P | X] = Q [K ; Sb]^T

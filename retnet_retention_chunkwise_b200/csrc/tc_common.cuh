@@ -128,6 +128,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of four phases at once (a barrier may be repeated): the
+// four tests go out back to back, so when every phase is already complete the
+// answer costs one shared-memory round trip instead of four in a row.
+__device__ __forceinline__ bool mbar_test4(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint64_t* b2,
+                                           uint32_t p2, uint64_t* b3, uint32_t p3) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred q0, q1, q2, q3;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q0, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q1, [%3], %4;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q2, [%5], %6;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q3, [%7], %8;\n\t"
+      "and.pred q0, q0, q1;\n\t"
+      "and.pred q2, q2, q3;\n\t"
+      "and.pred q0, q0, q2;\n\t"
+      "selp.u32 %0, 1, 0, q0;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b0)), "r"(p0), "r"(smem_u32(b1)), "r"(p1), "r"(smem_u32(b2)), "r"(p2), "r"(smem_u32(b3)),
+        "r"(p3)
+      : "memory");
+  return ok != 0;
+}
+
 struct WaitLimit {
   uint64_t ns;        // wall-clock budget of one wait
   uint32_t max_iter;  // hard cap on polls, whatever the clock says
@@ -147,6 +170,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   *abort = 1;
   atomicExch(&g_device_status, 4);
   return false;
+}
+
+// Bounded wait for four phases (a barrier may be repeated): one joint test,
+// then, only if some phase is not yet complete, the waits one by one.
+__device__ __forceinline__ bool mbar_wait4(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1, uint64_t* b2,
+                                           uint32_t p2, uint64_t* b3, uint32_t p3, volatile int* abort,
+                                           WaitLimit lim) {
+  if (mbar_test4(b0, p0, b1, p1, b2, p2, b3, p3)) return true;
+  return mbar_wait(b0, p0, abort, lim) && mbar_wait(b1, p1, abort, lim) && mbar_wait(b2, p2, abort, lim) &&
+         mbar_wait(b3, p3, abort, lim);
 }
 
 // --------------------------------------------------------------------- TMA
