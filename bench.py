@@ -102,7 +102,8 @@ def load_peaks():
 # file do not enter it.
 HEADLINE_SOURCE_REGIONS = (
     (b"namespace ret {",
-     b"template <int DK, bool REV>\n__global__ void __launch_bounds__(kCW_MainThreads, 1)\nchunkwise_tc_kernel("),
+     b"template <int DK, bool REV, bool GN = false>\n__global__ void __launch_bounds__(kCW_MainThreads, 1)\n"
+     b"chunkwise_tc_kernel("),
     (b"// dk = 256: one stage", b"// Segment sums for the sequence split"),
 )
 

@@ -40,3 +40,15 @@ def test_traffic_is_read_only_for_the_current_kernel_source():
             assert bench.measured_traffic() is None
     finally:
         bench.TRAFFIC_FILE = orig
+
+
+def test_digest_regions_are_found_in_the_kernel_source():
+    # every region marker must be present, or the digest silently covers the
+    # whole file and any edit elsewhere voids the traffic record
+    path = os.path.join(bench.ROOT, "retnet_retention_chunkwise_b200", "csrc", "chunkwise_tc.cuh")
+    with open(path, "rb") as f:
+        src = f.read()
+    for start, end in bench.HEADLINE_SOURCE_REGIONS:
+        i, j = src.find(start), src.find(end)
+        assert 0 <= i < j, (start[:40], end[:40])
+    assert b"chunkwise_tc256_kernel(" in src[src.find(bench.HEADLINE_SOURCE_REGIONS[1][0]):]
