@@ -1374,6 +1374,9 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
   const int nck = max(c_end - c_begin, 0);
   const int seg_last = min(c_end * C, a.L) - 1;  // e_g
   const int seg_first = c_begin * C;              // s_g
+  const int cta_id = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  (void)cta_id;
+  RET_TRACE_INIT();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) {
@@ -1402,6 +1405,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
         const int s = it % NS;
         if (it >= NS && !mbar_wait(&empty[s], ((it / NS) - 1) & 1, abort_flag, a.lim)) break;
         const int t0 = (c_begin + it) * C;
+        RET_TRACE_STAMP(cta_id, it, 0);
         mbar_arrive_expect_tx(&full[s], bytes);
         for (int b = 0; b < DK / 64; ++b)
           tma_load_3d(sK + s * k_stage + b * C * 128, &mapK, &full[s], b * 64, t0, bh);
@@ -1419,6 +1423,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
         const int s = it % NS;
         if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) break;
         if (!mbar_wait(&kready[s], (it / NS) & 1, abort_flag, a.lim)) break;
+        RET_TRACE_STAMP(cta_id, it, 1);
         tc_fence_after();
         for (int kk = 0; kk < C / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(aV + s * v_stage + kk * 2048, C * 128, 1024);
@@ -1426,6 +1431,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
           mma_ss(tm, ad, bd, id5, (it > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&empty[s]);
+        RET_TRACE_STAMP(cta_id, it, 4);
       }
       mma_commit(done);
     }
@@ -1435,6 +1441,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
     for (int it = 0; it < nck; ++it) {
       const int s = it % NS;
       if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) { ok = false; break; }
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 2);
       // Row j of the narrower operand times gamma^(e_g - t).  DK <= 128: rows
       // of K, one row per thread.  DK = 256: rows of V (half the bytes of K's),
       // 2 boxes x 8 chunks of 16 bytes per row, chunk e = 16 j + 8 box + c; each
@@ -1484,6 +1491,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
       }
       fence_proxy_async_smem();
       mbar_arrive(&kready[s]);
+      if (r == 0) RET_TRACE_STAMP(cta_id, it, 3);
     }
     if (ok && nck > 0 && mbar_wait(done, 0, abort_flag, a.lim)) {
       tc_fence_after();

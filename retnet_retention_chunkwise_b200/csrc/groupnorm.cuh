@@ -89,13 +89,77 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Value e (0..7) of 8 bf16 packed in a uint4.
+__device__ __forceinline__ float bf8_at(const uint4& v, int e) {
+  const uint32_t w = e < 2 ? v.x : e < 4 ? v.y : e < 6 ? v.z : v.w;
+  return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+}
+
+// bf16 rows with dv % 256 == 0: each lane keeps its 8 values per step (and
+// the gate's) as the packed 16-byte words it loaded, and widens them where
+// they are used; half the registers of fp32 copies, so more rows are resident
+// per SM and more loads are in flight.
+template <int STEPS, bool GATE>
+__device__ __forceinline__ void groupnorm_row_bf16x8(const __nv_bfloat16* yr, __nv_bfloat16* orow, int lane,
+                                                     int dv, float eps, const float* wr, const float* br,
+                                                     const __nv_bfloat16* gr, int act) {
+  uint4 xv[STEPS], gv[GATE ? STEPS : 1];
+#pragma unroll
+  for (int i = 0; i < STEPS; ++i) {
+    const int c = (i * 32 + lane) * 8;
+    xv[i] = make_uint4(0, 0, 0, 0);
+    if (c < dv) {
+      xv[i] = *reinterpret_cast<const uint4*>(yr + c);
+      if constexpr (GATE) gv[i] = *reinterpret_cast<const uint4*>(gr + c);
+    }
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < STEPS; ++i)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s += bf8_at(xv[i], e);  // zeros past dv
+  const float mean = warp_sum(s) / (float)dv;
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < STEPS; ++i) {
+    if ((i * 32 + lane) * 8 < dv) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = bf8_at(xv[i], e) - mean;
+        q += d * d;
+      }
+    }
+  }
+  const float rstd = rsqrtf(warp_sum(q) / (float)dv + eps);
+#pragma unroll
+  for (int i = 0; i < STEPS; ++i) {
+    const int c = (i * 32 + lane) * 8;
+    if (c < dv) {
+      float z[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        z[e] = (bf8_at(xv[i], e) - mean) * rstd;
+        if (wr) z[e] *= wr[c + e];
+        if (br) z[e] += br[c + e];
+      }
+      if constexpr (GATE) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z[e] *= gate_act(bf8_at(gv[i], e), act);
+      }
+      gn_store8(orow + c, z);
+    }
+  }
+}
+
 // One warp per (b, h, n) row.  Vectorised (VEC values per lane per step: 8
 // for bf16 when dv % 256 == 0, 4 when dv % 128 == 0), else one value per lane
 // per step; STEPS steps cover dv (<= 1024), so the row lives in VEC * STEPS
-// registers per lane (x2 with the gate).  out may alias y.  GATE: act(gate)
-// multiplies the result.
+// registers per lane (x2 with the gate; packed bf16 words for VEC = 8).  out
+// may alias y.  GATE: act(gate) multiplies the result.
+// Packed bf16 rows of up to 512 values fit in 40 registers a thread, six
+// blocks of 8 rows per SM (the gated form needs that bound to get there).
 template <typename T, int VEC, int STEPS, bool GATE>
-__global__ void __launch_bounds__(32 * kGN_RowsPerBlock)
+__global__ void __launch_bounds__(32 * kGN_RowsPerBlock, (VEC == 8 && STEPS <= 2) ? 6 : 1)
 groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, float eps,
                       const float* __restrict__ w, const float* __restrict__ bias, const T* __restrict__ gate,
                       int act) {
@@ -106,6 +170,11 @@ groupnorm_rows_kernel(const T* y, T* out, long long rows, int H, int L, int dv, 
   const T* yr = y + row * dv;
   const T* gr = GATE ? gate + row * dv : nullptr;
   T* orow = out + row * dv;
+  if constexpr (VEC == 8) {
+    groupnorm_row_bf16x8<STEPS, GATE>(yr, orow, lane, dv, eps, w ? w + (size_t)h * dv : nullptr,
+                                      bias ? bias + (size_t)h * dv : nullptr, gr, act);
+    return;
+  }
   float x[STEPS][VEC], gv[GATE ? STEPS : 1][VEC];
   float s = 0.f;
 #pragma unroll
