@@ -1443,11 +1443,9 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
       if (!mbar_wait(&full[s], (it / NS) & 1, abort_flag, a.lim)) { ok = false; break; }
       if (r == 0) RET_TRACE_STAMP(cta_id, it, 2);
       // Row j of the narrower operand times gamma^(e_g - t).  DK <= 128: rows
-      // of K, one row per thread.  DK = 256: rows of V (half the bytes of K's),
-      // 2 boxes x 8 chunks of 16 bytes per row, chunk e = 16 j + 8 box + c; each
-      // thread takes every 128th chunk, 8 at a time (all 8 loads first).  A
-      // row's chunks share its factor, so the swizzle (a permutation within the
-      // row) plays no part.
+      // of K, one row per thread.  DK = 256: rows of V (half the bytes of
+      // K's): thread r takes 64-column box (r & 1) of row (r >> 1), all 8
+      // loads first, one factor per thread.
       if constexpr (DK <= kCW_DVT) {
         for (uint32_t j = r; j < (uint32_t)C; j += 128) {  // rows j and j + 128 (blocks up to 256)
           const int t = (c_begin + it) * C + (int)j;
@@ -1457,36 +1455,12 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_consta
         }
       } else {
         uint8_t* vs = sV + s * v_stage;
-        const uint32_t n_chunks = (uint32_t)C * 16u;
-        for (uint32_t e0 = r; e0 < n_chunks; e0 += 8u * 128u) {
-          uint4 w[8];
-          float f[8];
-#pragma unroll
-          for (uint32_t u = 0; u < 8; ++u) {
-            const uint32_t e = e0 + u * 128u;
-            if (e < n_chunks) {
-              const uint32_t j = e >> 4;
-              w[u] = *reinterpret_cast<const uint4*>(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u +
-                                                      (e & 7u) * 16u);
-              const int t = (c_begin + it) * C + (int)j;
-              const int ex = REV ? t - seg_first : seg_last - t;
-              f[u] = (t <= seg_last) ? (ex == 0 ? 1.f : exp2f((float)ex * l2g)) : 0.f;
-            }
-          }
-#pragma unroll
-          for (uint32_t u = 0; u < 8; ++u) {
-            const uint32_t e = e0 + u * 128u;
-            if (e < n_chunks) {
-              const uint32_t j = e >> 4;
-              const float g = f[u];
-              uint4 x = w[u];
-              x.x = pack_bf16x2(bf16lo_to_f32(x.x) * g, bf16hi_to_f32(x.x) * g);
-              x.y = pack_bf16x2(bf16lo_to_f32(x.y) * g, bf16hi_to_f32(x.y) * g);
-              x.z = pack_bf16x2(bf16lo_to_f32(x.z) * g, bf16hi_to_f32(x.z) * g);
-              x.w = pack_bf16x2(bf16lo_to_f32(x.w) * g, bf16hi_to_f32(x.w) * g);
-              *reinterpret_cast<uint4*>(vs + ((e >> 3) & 1u) * (uint32_t)C * 128u + j * 128u + (e & 7u) * 16u) = x;
-            }
-          }
+        for (uint32_t pr = r; pr < 2u * (uint32_t)C; pr += 128) {
+          const uint32_t j = pr >> 1;
+          const int t = (c_begin + it) * C + (int)j;
+          const int ex = REV ? t - seg_first : seg_last - t;
+          const float f = (t <= seg_last) ? (ex == 0 ? 1.f : exp2f((float)ex * l2g)) : 0.f;
+          scale_row_sw128(vs + (pr & 1u) * (uint32_t)C * 128u, j, f);
         }
       }
       fence_proxy_async_smem();
