@@ -383,11 +383,12 @@ ret_status launch_state_fold(const float* state_in, const float* parts, float* o
 
 // Plan of a state-only call.  Its result does not depend on the block length
 // (every row of K is scaled by its own decay to the segment end, and the sums
-// accumulate in fp32 across blocks), so it runs blocks of kStateC rows, which
-// keep four stages or two CTAs per SM in flight, and enough segments for about
-// two CTAs per SM; fewer when the workspace (n_seg + 1 states per (b, h)) is
-// short.  Returns n_seg, 0 when even one segment does not fit.
-constexpr int kStateC = 64;
+// accumulate in fp32 across blocks), so it runs blocks of kStateC rows, short
+// enough for two CTAs per SM with three stages each at dk = 256, and enough
+// segments for about two CTAs per SM; fewer when the workspace (n_seg + 1
+// states per (b, h)) is short.  Returns n_seg, 0 when even one segment does
+// not fit.
+constexpr int kStateC = 48;
 
 int state_only_segments(const ret_shape& s, size_t ws_bytes, int* seg_chunks) {
   const size_t per = (size_t)s.B * s.H * s.dk * s.dv * sizeof(float);
@@ -419,10 +420,13 @@ ret_status launch_chunk_state(const void* k, const void* v, const float* gamma, 
   fill_l2g(dec, gamma, s.H);
   const int smax = max_smem_optin();
   const uint32_t per = (uint32_t)(DK / 64) * C * 128 + 2u * C * 128;
-  // two stages per CTA when two CTAs per SM are wanted and fit, else as many as fit
+  // as many stages as let two CTAs share an SM when there are more CTAs than
+  // SMs (and two stages fit so), else as many as fit
   int ns = 0;
   const long long ctas = (long long)(s.dv / kCW_DVT) * BH * n_seg;
-  const int cap = (ctas > sm_count() && 2 * (int)(2 * per + kMiscBytes + kSmemAlign) <= smax) ? 2 : kCW_MaxStages;
+  int cap = kCW_MaxStages;
+  if (ctas > sm_count() && 2 * (int)(2 * per + kMiscBytes + kSmemAlign) <= smax)
+    while (cap > 2 && 2 * (int)(cap * per + kMiscBytes + kSmemAlign) > smax) --cap;
   for (int n = cap; n >= 1; --n)
     if ((int)(n * per + kMiscBytes + kSmemAlign) <= smax) { ns = n; break; }
   if (ns == 0) return RET_EUNSUPPORTED;
