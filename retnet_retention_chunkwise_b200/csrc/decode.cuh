@@ -127,4 +127,62 @@ recurrent_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T*
   }
 }
 
+// Small grids (few heads, e.g. batch 1): a block of 32 state columns per CTA,
+// one column per lane (a warp still reads one 128-byte row segment per load),
+// so that the grid has four times as many CTAs to spread the state stream over
+// the SMs; eight rows in flight per warp.
+constexpr int kDecodeNarrowCols = 32;
+
+template <typename T>
+__global__ void __launch_bounds__(kDecodeThreads)
+recurrent_step_narrow_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                             T* __restrict__ y, float* __restrict__ S, int H, int dk, int dv,
+                             const __grid_constant__ HeadGamma hg) {
+  __shared__ float sq[kDecodeMaxDk];
+  __shared__ float sk[kDecodeMaxDk];
+  __shared__ float red[kDecodeThreads / 32][32];
+
+  const int bh = blockIdx.y;
+  const float g = hg.g[bh % H];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int col = blockIdx.x * kDecodeNarrowCols + lane;
+
+  for (int i = threadIdx.x; i < dk; i += kDecodeThreads) {
+    sq[i] = to_f32(q[(size_t)bh * dk + i]);
+    sk[i] = to_f32(k[(size_t)bh * dk + i]);
+  }
+  const float vv = (col < dv) ? to_f32(v[(size_t)bh * dv + col]) : 0.f;
+  __syncthreads();
+
+  float acc = 0.f;
+  float* Sh = S + (size_t)bh * dk * dv;
+  if (col < dv) {
+    int d = warp;
+    for (; d + 56 < dk; d += 64) {
+      float s[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s[u] = Sh[(size_t)(d + 8 * u) * dv + col];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        s[u] = fmaf(g, s[u], sk[d + 8 * u] * vv);
+        Sh[(size_t)(d + 8 * u) * dv + col] = s[u];
+        acc = fmaf(sq[d + 8 * u], s[u], acc);
+      }
+    }
+    for (; d < dk; d += 8) {
+      const float sv = fmaf(g, Sh[(size_t)d * dv + col], sk[d] * vv);
+      Sh[(size_t)d * dv + col] = sv;
+      acc = fmaf(sq[d], sv, acc);
+    }
+  }
+  red[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float t = red[0][lane];
+#pragma unroll
+    for (int w = 1; w < kDecodeThreads / 32; ++w) t += red[w][lane];
+    if (col < dv) from_f32(y + (size_t)bh * dv + col, t);
+  }
+}
+
 }  // namespace ret

@@ -790,6 +790,19 @@ ret_status retention_recurrent_step(const void* q, const void* k, const void* v,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   dim3 grid((s.dv + kDecodeCols - 1) / kDecodeCols, s.B * s.H);
   const bool vec = (s.dv % 4) == 0;
+  if ((long long)grid.x * grid.y < 2LL * sm_count()) {
+    // few heads: narrower column blocks, four times the CTAs
+    const dim3 gn((s.dv + kDecodeNarrowCols - 1) / kDecodeNarrowCols, s.B * s.H);
+    if (dt == RET_F32)
+      recurrent_step_narrow_kernel<float><<<gn, kDecodeThreads, 0, st>>>(
+          static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+          static_cast<float*>(y), state, s.H, s.dk, s.dv, hg);
+    else
+      recurrent_step_narrow_kernel<__nv_bfloat16><<<gn, kDecodeThreads, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+          static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(y), state, s.H, s.dk, s.dv, hg);
+    return launch_status();
+  }
   if (dt == RET_F32) {
     auto* qf = static_cast<const float*>(q);
     auto* kf = static_cast<const float*>(k);
