@@ -588,3 +588,25 @@ def test_chunkwise_cold_cache_repeatable(B, H, L, dk, dv, C):
     for y, s in outs[1:]:
         assert torch.equal(y, outs[0][0]) and torch.equal(s, outs[0][1])
     assert rel(outs[0][0], y_ref) <= 2e-2 and rel(outs[0][1], s_ref) <= 2e-2
+
+
+def test_chunkwise_groupnorm_unaligned_affine_takes_the_two_kernel_path():
+    # weight and bias that are not 16-byte aligned cannot be read as float4 in
+    # the fused epilogue: the call normalises in a second kernel instead, with
+    # the same result
+    B, H, L, dk, dv, C = 1, 2, 300, 64, 128, 64
+    q, k, v = inputs.qkv(B, H, L, dk, dv, torch.bfloat16, seed=41)
+    gam = inputs.multiscale_gammas(H)
+    g = torch.Generator("cpu").manual_seed(42)
+    w = torch.rand(H * dv, generator=g) + 0.5
+    b = torch.randn(H * dv, generator=g) * 0.1
+    y_ref, s_ref = oracle.recurrent(q, k, v, gam)
+    z_ref = oracle.groupnorm(y_ref, eps=1e-5, weight=w, bias=b)
+    wd = torch.empty(H * dv + 1, device="cuda")[1:]
+    bd = torch.empty(H * dv + 1, device="cuda")[1:]
+    wd.copy_(w)
+    bd.copy_(b)
+    assert wd.data_ptr() % 16 != 0 and bd.data_ptr() % 16 != 0
+    qd, kd, vd = dev(q, k, v)
+    z, s = ret.chunkwise_groupnorm(qd, kd, vd, gam, C, 1e-5, weight=wd, bias=bd)
+    assert rel(z, z_ref) <= 2e-2 and rel(s, s_ref) <= 2e-2
