@@ -310,6 +310,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   const int cta_id = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
   (void)cta_id;
   RET_TRACE_INIT();
+  if (threadIdx.x == 0) RET_TRACE_STAMP(cta_id, 255, 0);  // trace: kernel entry
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) {
@@ -356,6 +357,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tmem_slot;
+  if (threadIdx.x == 0) RET_TRACE_STAMP(cta_id, 255, 1);  // trace: prologue done
 
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
@@ -447,6 +449,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
         }
       }
       bulk_wait_all();  // the y stores issued by this thread are complete
+      RET_TRACE_STAMP(cta_id, 255, 3);  // trace: last y store complete
       // every load issued must land before the CTA may exit
       for (int it = max(0, issued - NS); it < issued; ++it) {
         mbar_drain(&fullQ[it % NS], (it / NS) & 1, a.lim);
@@ -767,6 +770,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(sready);
+      if (v_loc == 0) RET_TRACE_STAMP(cta_id, 255, 2);  // trace: initial state in place
     }
     for (int it = 0; it < nck; ++it) {
       // MMA5 (state update) and MMA4 (last reader of Sb) are both done
@@ -899,6 +903,7 @@ chunkwise_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_const
     }
   }
   if (threadIdx.x == 0) bulk_wait_all();  // no store is left in flight (the producer waited for its own)
+  if (threadIdx.x == 0) RET_TRACE_STAMP(cta_id, 255, 4);  // trace: end of the roles
   tc_fence_before();
   __syncthreads();
   if (warp == kWarpMma) {
